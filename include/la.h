@@ -1,0 +1,194 @@
+/*
+ * la.h -- C ABI of the causal Lightning Attention library for B200 (sm_100a).
+ *
+ * Sources cited by page title and section:
+ *   [MX01] "MiniMax-01与Lightning Attention": section 1.1 (128 attention heads,
+ *          32 kv heads), 2.2 (linear attention by associativity, kv_sum =
+ *          K^T V), 2.3 (tiled state updates), 4.1 (incremental kv state).
+ *   [VGX]  "如何理解MiniMax股价创历史新高？拆解国产大模型技术底座", section
+ *          "Lightning Attention：长上下文为什么突然变得便宜了": the causal
+ *          chunkwise sketch (per block: inter term Q_b S, masked intra term
+ *          tril(Q_b K_b^T) V_b, then S += K_b^T V_b; the state starts at zero;
+ *          the last block may be short).
+ *
+ * What the library computes.  For every batch b and query head h, with
+ * g = floor(h / (Hq/Hkv)) the kv head h shares:
+ *
+ *     O[b,h,t,:] = q[b,h,t] S0[b,g] + sum_{s <= t} (q[b,h,t] . k[b,g,s]) v[b,g,s,:]
+ *     S[b,g]     = S0[b,g] + sum_s k[b,g,s]^T v[b,g,s]          (final state)
+ *
+ * chunk by chunk as [VGX] lays it out: O_c = Q_c S_{<c} + tril(Q_c K_c^T) V_c,
+ * then S += K_c^T V_c.  No softmax, no normalisation, no decay, no scaling (the
+ * 1/sqrt(d) factor belongs to the inputs).  S0 is zero unless given.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are caller-owned DEVICE memory, contiguous, row-major:
+ *       q, o  [B, Hq,  N, d]      k, v  [B, Hkv, N, d]      S  [B, Hkv, d, d]
+ *     S[b,g][i][j] pairs key feature i with value feature j.  The library never
+ *     frees, reallocates or keeps pointers to caller memory after a call.
+ *   - la_bf16 is the bit pattern of a bfloat16.  Outputs have the input dtype;
+ *     states are fp32; all accumulation is fp32.
+ *   - Every tensor pointer must be 16-byte aligned (the bulk tensor copies
+ *     require it); o must not overlap q, k, v or S.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and launch on the device current to the calling thread.
+ *   - Return codes report argument validation and launch errors only.  A fault
+ *     during execution surfaces at the caller's next synchronisation; a bounded
+ *     device-side wait that expires sets the device status word, read with
+ *     la_device_status().
+ */
+#ifndef LIGHTNING_B200_LA_H
+#define LIGHTNING_B200_LA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, Hq % Hkv != 0, misalignment, overlap */
+  LA_ERR_UNSUPPORTED = 2, /* head dim or chunk size this build does not implement */
+  LA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  LA_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired (see la_device_status) */
+  LA_ERR_WORKSPACE = 5    /* workspace pointer missing, misaligned or too small */
+} la_status;
+
+typedef uint16_t la_bf16; /* bfloat16 bits */
+typedef void *la_stream;  /* cudaStream_t */
+
+/* Device status word bits, set by kernels, read by la_device_status(). */
+#define LA_DEV_TIMEOUT 0x1u /* a bounded mbarrier / flag wait gave up */
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *la_status_string(la_status s);
+
+/* Library ABI version (this header: 1). */
+int la_version(void);
+
+/* ------------------------------------------------------------------------
+ * Prefill, bf16 -- the hot path.  Tensor-core (tcgen05) kernels, d == 128.
+ *
+ * la_forward: O only, zero initial state ([VGX] sketch; rows a1-a9 of the
+ * method).  chunk is the block length of the masked intra-chunk product,
+ * 64 or 128; any N >= 1 is accepted (the last chunk may be short, as in the
+ * sketch's end = min(start + block, n)).
+ *
+ * Query heads are grouped with their kv head ([MX01] section 1.1, GQA): one
+ * 128-row tensor-core tile holds 128/chunk query heads of a group times chunk
+ * tokens.  A group with a single query head at chunk 64 stacks two
+ * consecutive 64-token chunks into one 128-token tile with the full causal
+ * mask -- the same sum in exact arithmetic, since the chunked form is exact for
+ * every block length.
+ *
+ * Uses a workspace for the per-span states; la_forward / la_forward_state
+ * keep one cached per device (grown on demand with cudaMalloc, freed by
+ * la_shutdown), la_forward_ws takes one from the caller.
+ *
+ * Errors: LA_ERR_INVALID_ARG (null or misaligned pointer, B/Hq/Hkv/N <= 0,
+ * Hq % Hkv, o overlapping an input), LA_ERR_UNSUPPORTED (d != 128, chunk not
+ * in {64, 128}), LA_ERR_CUDA (allocation or launch failure).
+ * ---------------------------------------------------------------------- */
+la_status la_forward(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o, int B,
+                     int Hq, int Hkv, int64_t N, int d, int chunk, la_stream stream);
+
+/* As la_forward, plus a state.  S (nullable) is [B,Hkv,d,d] fp32 device
+ * memory: on entry the initial state S0, on return the final state
+ * S0 + K^T V ([MX01] section 4.1: the state is the whole resume point, so a
+ * sequence may be processed in pieces).  S == NULL means S0 = 0, no state out. */
+la_status la_forward_state(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
+                           float *S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                           la_stream stream);
+
+/* Bytes of workspace la_forward_ws needs for this problem on the current device. */
+size_t la_forward_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d, int chunk);
+
+/* As la_forward_state with a caller-owned device workspace (256-byte aligned,
+ * at least la_forward_workspace_bytes()); LA_ERR_WORKSPACE otherwise.  The
+ * workspace must not be used by anything else until the call's work on
+ * `stream` has finished. */
+la_status la_forward_ws(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
+                        float *S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                        void *workspace, size_t workspace_bytes, la_stream stream);
+
+/* ------------------------------------------------------------------------
+ * The prefill's three stages, for callers that schedule or time them apart.
+ * la_forward_ws == plan, then span_states, scan, main on one stream.
+ *
+ * The sequence of every (batch, kv head) is cut into `nspan` spans of whole
+ * chunks.  span_states writes each span's K^T V into the workspace; scan turns
+ * those into the state entering each span (S0 + the spans before it) and, if S
+ * is given, writes the final state; main runs the chunked loop of every span
+ * from its entering state.  This split is not on the pages: the chunk loop of
+ * the [VGX] sketch is sequential, and spans let one sequence fill the GPU.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int32_t nspan;           /* spans per (batch, kv head) */
+  int32_t tile;            /* tokens per 128-row tile: chunk, or 128 when stacking two 64-chunks */
+  int32_t heads_per_tile;  /* query heads stacked in one tile (tile * heads_per_tile == 128) */
+  int32_t tiles_total;     /* ceil(N / tile) */
+  int64_t workspace_bytes; /* B * Hkv * nspan * d * d * 4 */
+} la_plan;
+
+/* Fill *plan for this problem on the current device.  Errors as la_forward. */
+la_status la_prefill_plan(int B, int Hq, int Hkv, int64_t N, int d, int chunk, la_plan *plan);
+
+/* Stage 1: ws[b,g,j] = sum over span j of K_c^T V_c (fp32, [B,Hkv,nspan,d,d]). */
+la_status la_prefill_span_states(const la_bf16 *k, const la_bf16 *v, int B, int Hkv, int64_t N,
+                                 int d, const la_plan *plan, float *ws, la_stream stream);
+
+/* Stage 2, in place: ws[b,g,j] <- S0[b,g] + sum_{i<j} ws[b,g,i].  S (nullable)
+ * supplies S0 on entry and receives S0 + sum_i ws[b,g,i] on return. */
+la_status la_prefill_scan(float *ws, float *S, int B, int Hkv, int d, const la_plan *plan,
+                          la_stream stream);
+
+/* Stage 3: O for every span, starting each from ws[b,g,j]. */
+la_status la_prefill_main(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
+                          const float *ws, int B, int Hq, int Hkv, int64_t N, int d,
+                          const la_plan *plan, la_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Prefill in fp32 (inputs, output and state fp32; SIMT fp32 arithmetic).
+ * Same definition and arguments as la_forward_state; d in {64, 128}, chunk in
+ * {64, 128}.  For checking at fp32 precision, not tuned for speed.
+ * ---------------------------------------------------------------------- */
+la_status la_forward_f32(const float *q, const float *k, const float *v, float *o, float *S,
+                         int B, int Hq, int Hkv, int64_t N, int d, int chunk, la_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Decode step: one new token per sequence on the recurrent state
+ * ([MX01] section 4.1, incremental kv state; update first, then read, which
+ * keeps the diagonal term of the causal mask).  For every (b, g):
+ *     S[b,g] += k[b,g]^T v[b,g];   o[b,h] = q[b,h] S[b,g]  for the heads h of g.
+ * S [B,Hkv,d,d] fp32 is updated in place; q, o [B,Hq,d] and k, v [B,Hkv,d]
+ * are bf16.  d in {64, 128}.  Errors as la_forward.
+ * ---------------------------------------------------------------------- */
+la_status la_decode_step(float *S, const la_bf16 *q, const la_bf16 *k, const la_bf16 *v,
+                         la_bf16 *o, int B, int Hq, int Hkv, int d, la_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Failure detection.
+ * la_device_status: synchronises the current device, then stores the device
+ * status word (LA_DEV_* bits, 0 = clean) in *flags and clears it if `clear`.
+ * Returns LA_ERR_TIMEOUT when LA_DEV_TIMEOUT is set, LA_ERR_CUDA if the
+ * synchronisation reports a fault, else LA_OK.
+ *
+ * la_selftest_wait: launches one warp that waits, bounded by timeout_ns of
+ * device time, on a device flag that nothing ever sets; when the limit passes
+ * it records LA_DEV_TIMEOUT and returns.  Exercises the same bounded-wait
+ * routine the kernels use, without faulting or hanging the GPU.
+ * ---------------------------------------------------------------------- */
+la_status la_device_status(unsigned int *flags, int clear);
+la_status la_selftest_wait(int64_t timeout_ns, la_stream stream);
+
+/* Frees the cached per-device workspace of la_forward / la_forward_state.
+ * Call only when no call of this library is in flight. */
+void la_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_B200_LA_H */

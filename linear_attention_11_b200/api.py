@@ -1,0 +1,201 @@
+"""Thin ctypes binding of ``include/la.h``: same names, argument marshalling only.
+
+Each function takes torch CUDA tensors, passes their device pointers, sizes and
+the current CUDA stream to the C ABI, and raises ``LAError`` on a non-zero
+status.  No arithmetic of the method happens here; there is no CPU fallback.
+The shared library is loaded on first use and a missing build is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIBNAME = "liblightning_b200.so"
+_lock = threading.Lock()
+_lib = None
+
+STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_CUDA",
+          4: "LA_ERR_TIMEOUT", 5: "LA_ERR_WORKSPACE"}
+
+# Every symbol include/la.h declares.
+EXPORTS = ("la_status_string", "la_version", "la_forward", "la_forward_state",
+           "la_forward_workspace_bytes", "la_forward_ws", "la_prefill_plan",
+           "la_prefill_span_states", "la_prefill_scan", "la_prefill_main", "la_forward_f32",
+           "la_decode_step", "la_device_status", "la_selftest_wait", "la_shutdown")
+
+
+class LAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class la_plan(ctypes.Structure):
+    _fields_ = [("nspan", ctypes.c_int32), ("tile", ctypes.c_int32),
+                ("heads_per_tile", ctypes.c_int32), ("tiles_total", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_int64)]
+
+
+def library_path() -> str:
+    return os.environ.get("LA_LIBRARY", os.path.join(_HERE, _LIBNAME))
+
+
+def _declare(lib):
+    P, I, L, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    PP = ctypes.POINTER(la_plan)
+    sig = {
+        "la_status_string": ([I], ctypes.c_char_p),
+        "la_version": ([], I),
+        "la_forward": ([P, P, P, P, I, I, I, L, I, I, P], I),
+        "la_forward_state": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
+        "la_forward_workspace_bytes": ([I, I, I, L, I, I], S),
+        "la_forward_ws": ([P, P, P, P, P, I, I, I, L, I, I, P, S, P], I),
+        "la_prefill_plan": ([I, I, I, L, I, I, PP], I),
+        "la_prefill_span_states": ([P, P, I, I, L, I, PP, P, P], I),
+        "la_prefill_scan": ([P, P, I, I, I, PP, P], I),
+        "la_prefill_main": ([P, P, P, P, P, I, I, I, L, I, PP, P], I),
+        "la_forward_f32": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
+        "la_decode_step": ([P, P, P, P, P, I, I, I, I, P], I),
+        "la_device_status": ([ctypes.POINTER(ctypes.c_uint), I], I),
+        "la_selftest_wait": ([L, P], I),
+        "la_shutdown": ([], None),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+def load_library(path: str | None = None):
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            p = path or library_path()
+            if not os.path.exists(p):
+                raise RuntimeError(
+                    f"CUDA library not built: {p} is missing "
+                    "(run `python -m linear_attention_11_b200.build`)")
+            _lib = _declare(ctypes.CDLL(p))
+    return _lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise LAError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dims(q, k):
+    B, Hq, N, d = q.shape
+    return B, Hq, k.shape[1], N, d
+
+
+def la_status_string(code: int) -> str:
+    return load_library().la_status_string(code).decode()
+
+
+def la_forward(q, k, v, o=None, chunk: int = 64, stream=None):
+    """O for q [B,Hq,N,d], k, v [B,Hkv,N,d] (bf16, CUDA); zero initial state."""
+    if o is None:
+        o = torch.empty_like(q)
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("la_forward", load_library().la_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, d, chunk, _stream(stream)))
+    return o
+
+
+def la_forward_state(q, k, v, S=None, o=None, chunk: int = 64, stream=None):
+    """As la_forward; S [B,Hkv,d,d] fp32 (in: initial state, out: final state)."""
+    if o is None:
+        o = torch.empty_like(q)
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("la_forward_state", load_library().la_forward_state(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, _stream(stream)))
+    return o
+
+
+def la_forward_workspace_bytes(B, Hq, Hkv, N, d, chunk) -> int:
+    return int(load_library().la_forward_workspace_bytes(B, Hq, Hkv, N, d, chunk))
+
+
+def la_forward_ws(q, k, v, o, S, workspace, chunk: int = 64, stream=None):
+    B, Hq, Hkv, N, d = _dims(q, k)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("la_forward_ws", load_library().la_forward_ws(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk,
+        _ptr(workspace), nbytes, _stream(stream)))
+    return o
+
+
+def la_prefill_plan(B, Hq, Hkv, N, d, chunk) -> la_plan:
+    plan = la_plan()
+    _check("la_prefill_plan", load_library().la_prefill_plan(B, Hq, Hkv, N, d, chunk,
+                                                             ctypes.byref(plan)))
+    return plan
+
+
+def la_prefill_span_states(k, v, plan: la_plan, ws, stream=None):
+    B, Hkv, N, d = k.shape
+    _check("la_prefill_span_states", load_library().la_prefill_span_states(
+        _ptr(k), _ptr(v), B, Hkv, N, d, ctypes.byref(plan), _ptr(ws), _stream(stream)))
+
+
+def la_prefill_scan(ws, S, plan: la_plan, B, Hkv, d, stream=None):
+    _check("la_prefill_scan", load_library().la_prefill_scan(
+        _ptr(ws), _ptr(S), B, Hkv, d, ctypes.byref(plan), _stream(stream)))
+
+
+def la_prefill_main(q, k, v, o, ws, plan: la_plan, stream=None):
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("la_prefill_main", load_library().la_prefill_main(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ws), B, Hq, Hkv, N, d, ctypes.byref(plan),
+        _stream(stream)))
+
+
+def la_forward_f32(q, k, v, o=None, S=None, chunk: int = 64, stream=None):
+    if o is None:
+        o = torch.empty_like(q)
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("la_forward_f32", load_library().la_forward_f32(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, _stream(stream)))
+    return o
+
+
+def la_decode_step(S, q, k, v, o=None, stream=None):
+    """One decode step: S [B,Hkv,d,d] fp32 updated in place; returns o [B,Hq,d]."""
+    if o is None:
+        o = torch.empty_like(q)
+    B, Hq, d = q.shape
+    _check("la_decode_step", load_library().la_decode_step(
+        _ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, k.shape[1], d, _stream(stream)))
+    return o
+
+
+def la_device_status(clear: bool = True):
+    """(status code, device flags).  Synchronises the current device."""
+    flags = ctypes.c_uint(0)
+    code = load_library().la_device_status(ctypes.byref(flags), 1 if clear else 0)
+    return code, flags.value
+
+
+def la_selftest_wait(timeout_ns: int, stream=None):
+    _check("la_selftest_wait", load_library().la_selftest_wait(timeout_ns, _stream(stream)))
+
+
+def la_shutdown():
+    load_library().la_shutdown()
