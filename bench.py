@@ -1,0 +1,379 @@
+"""Benchmark of the causal Lightning Attention prefill (and decode step) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa32k|mha8k|long1m] [--chunk 64|128]
+
+One JSON line on rank 0.  A step is one la_forward call over the whole
+workload (span states, state scan, chunk loop = every prefill stage).  The
+default workload is the grouped-query MiniMax-01-shaped layer: B=1, 128 query
+heads over 32 kv heads, N=32768, d=128, chunk 64, bf16 (q, k ~ N(0,1)/sqrt(d),
+v ~ N(0,1), seed 2).  Its inputs (2.7 GB) exceed L2, so no flush is needed.
+
+  value      Mtok/s with inputs resident in HBM (tokens = B*N positions, all heads)
+  e2e        the same metric through the public call with pinned host buffers,
+             host->device copies of q, k, v and the device->host copy of O
+             inside the timed region
+  roofline   the main chunk-loop kernel: algorithmic Q+K+V+O bytes / its
+             CUDA-event duration, against the measured HBM copy bandwidth
+  decode     the decode step on B=256, Hq=64/Hkv=16, d=128, 64 steps: GB/s
+  cpu_baseline  the fp64 CPU oracle (recurrent form) on a bounded sample
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (independent
+sequences, no collective on the data path): weak scaling; the reported time is
+the max over ranks.  ``--impl reference`` times the CPU oracle on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_11_b200 import synth  # noqa: E402
+
+WORKLOADS = {"gqa32k": synth.GQA_32K, "mha8k": synth.MHA_8K, "long1m": synth.LONG_1M}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa32k")
+    ap.add_argument("--chunk", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=None)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons while the GPU works."""
+
+    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001
+            self._nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def timed(fn, steps, stream):
+    """Device time of `steps` calls of fn on `stream`, with clock samples."""
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dev = torch.cuda.current_device()
+    with ClockSampler(dev) as clk:
+        start.record(stream)
+        for _ in range(steps):
+            fn()
+        end.record(stream)
+        while not end.query():
+            time.sleep(0.001)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / 1e3, clk.summary()
+
+
+def traffic_from_profile(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source is unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "linear_attention_11_b200", "csrc", "la_prefill.cu")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        e = t.get(kernel_key)
+        if e and e.get("source_sha256") == sha:
+            return e["dram_bytes_per_launch"]
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_baseline(w, sample_tokens=None, target_s=10.0):
+    """The fp64 oracle (recurrent form), as it stands, on a sequence of n tokens
+    drawn with the workload's recipe, all heads.  Without sample_tokens, n is
+    grown from a 256-token probe to about target_s seconds of work.
+    Returns (tokens/s, sample description, threads used, seconds)."""
+    import numpy as np
+
+    import oracle
+    cores = oracle.threads()
+    units = w.B * w.Hkv
+    if sample_tokens is None:
+        q, k, v = synth.prefill_inputs(w, N=256)
+        t0 = time.perf_counter()
+        oracle.recurrent(q, k, v, o_dtype=np.float32)
+        dt0 = time.perf_counter() - t0
+        n = int(min(w.N, max(256, 256 * target_s / max(dt0, 1e-3))))
+    else:
+        n = sample_tokens
+    q, k, v = synth.prefill_inputs(w, N=n)
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, o_dtype=np.float32)
+    dt = time.perf_counter() - t0
+    sample = (f"{n} of {w.N} tokens drawn with the workload recipe, B={w.B}, all {w.Hq} query "
+              f"heads; {units} independent (batch, kv head) units over {min(cores, units)} threads")
+    return w.B * n / dt, sample, min(cores, units), dt
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    steps, warm = args.steps, args.warmup
+    n = args.cpu_sample_tokens or 512
+    cores = min(oracle.threads(), w.B * w.Hkv)
+    q, k, v = synth.prefill_inputs(w, N=n)
+    per = []
+    for i in range(warm + steps):
+        t0 = time.perf_counter()
+        oracle.recurrent(q, k, v, o_dtype=np.float32)
+        if i >= warm:
+            per.append(time.perf_counter() - t0)
+    dt = sum(per)
+    value = w.B * n * steps / dt / 1e6
+    line = {"impl": "reference", "metric": "causal lightning-attn prefill throughput",
+            "value": value, "unit": "Mtok/s", "n_gpus": args.gpus, "steps": steps,
+            "warmup": warm, "ms_per_step": 1e3 * dt / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N,
+                       "chunk": args.chunk or w.chunks[0], "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: the first {n} tokens of the workload "
+                                       f"(B={w.B}, all {w.Hq} query heads), fp64 recurrent form"},
+            "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w):
+    import linear_attention_11_b200 as la
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    chunk = args.chunk or w.chunks[0]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    q, k, v = synth.prefill_inputs(w)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    o = torch.empty_like(qd)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+
+    def step():
+        la.la_forward(qd, kd, vd, o=o, chunk=chunk, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    barrier()
+    t, clocks = timed(step, args.steps, stream)
+    barrier()
+    if dist:
+        tt = torch.tensor([t], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    value = world * B * N * args.steps / t / 1e6
+
+    # --- per-kernel timing of the main chunk-loop pass (stages called apart)
+    plan = la.api.la_prefill_plan(B, Hq, Hkv, N, d, chunk)
+    ws = torch.empty(plan.workspace_bytes // 4, dtype=torch.float32, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(max(3, min(args.steps, 20)))]
+    for i in range(len(ev) + 2):
+        la.api.la_prefill_span_states(kd, vd, plan, ws, stream=stream)
+        la.api.la_prefill_scan(ws, None, plan, B, Hkv, d, stream=stream)
+        if i >= 2:
+            ev[i - 2][0].record(stream)
+        la.api.la_prefill_main(qd, kd, vd, o, ws, plan, stream=stream)
+        if i >= 2:
+            ev[i - 2][1].record(stream)
+    torch.cuda.synchronize()
+    t_main = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
+    elt = 2
+    alg_bytes = elt * (2 * B * Hq * N * d + 2 * B * Hkv * N * d)
+    flops_ns = B * Hq * N * (4 * chunk * d + 4 * d * d)
+    pk = peaks()
+    achieved = alg_bytes / t_main / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic_from_profile("prefill_main"),
+                "kernel": "prefill_main_kernel", "launch_ms": t_main * 1e3,
+                "algorithmic_bytes_per_launch": alg_bytes, "peak_source": pk["source"]}
+    step_frac = (alg_bytes / (t / args.steps) / 1e9) / pk["hbm_gbs"]
+
+    # --- end to end: pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = args.e2e_steps or max(3, min(args.steps, 10))
+        qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+        oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        qe, ke, ve = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+
+        def e2e_step():
+            qe.copy_(qh, non_blocking=True)
+            ke.copy_(kh, non_blocking=True)
+            ve.copy_(vh, non_blocking=True)
+            la.la_forward(qe, ke, ve, o=o, chunk=chunk, stream=stream)
+            oh.copy_(o, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        te, _ = timed(e2e_step, e2e_steps, stream)
+        barrier()
+        if dist:
+            tt = torch.tensor([te], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            te = float(tt.item())
+        e2e = {"value": world * B * N * e2e_steps / te / 1e6, "unit": "Mtok/s",
+               "h2d_bytes_per_step": elt * (q.numel() + k.numel() + v.numel()),
+               "d2h_bytes_per_step": elt * q.numel(), "steps": e2e_steps}
+        del qh, kh, vh, oh, qe, ke, ve
+
+    # --- decode step
+    decode = None
+    if not args.no_decode:
+        del qd, kd, vd, o, ws
+        torch.cuda.empty_cache()
+        dw = synth.DECODE_B256
+        S = synth.decode_state(dw).to(dev)
+        toks = [tuple(t.to(dev) for t in synth.decode_token(dw, i)) for i in range(dw.steps)]
+        od = torch.empty(dw.B, dw.Hq, dw.d, dtype=torch.bfloat16, device=dev)
+        for i in range(3):
+            la.la_decode_step(S, *toks[i], o=od, stream=stream)
+        it = iter(range(10**9))
+
+        def dstep():
+            i = next(it) % dw.steps
+            la.la_decode_step(S, *toks[i], o=od, stream=stream)
+
+        td, dclk = timed(dstep, dw.steps, stream)
+        per = td / dw.steps
+        dbytes = 4 * 2 * dw.B * dw.Hkv * dw.d * dw.d + 2 * (2 * dw.B * dw.Hq * dw.d +
+                                                             2 * dw.B * dw.Hkv * dw.d)
+        decode = {"metric": "decode-step HBM bandwidth", "value": dbytes / per / 1e9,
+                  "unit": "GB/s", "us_per_step": per * 1e6, "steps": dw.steps,
+                  "frac_of_hbm_peak": dbytes / per / 1e9 / pk["hbm_gbs"],
+                  "bytes_per_step": dbytes, "workload": dw.name, "clocks": dclk}
+
+    line = {
+        "metric": "causal lightning-attn prefill throughput (Mtok/s); decode-step GB/s",
+        "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": B * world, "seq_len": N, "chunk": chunk,
+                   "Hq": Hq, "Hkv": Hkv, "d": d, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "clocks": clocks,
+        "gpu_launches": 3 * args.steps,
+        "roofline": roofline,
+        "step_hbm_frac": step_frac,
+        "tflops_north_star": flops_ns / (t / args.steps) / 1e12,
+        "e2e": e2e,
+        "decode": decode,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok_s, sample, cores, dt = cpu_baseline(w, args.cpu_sample_tokens)
+        line["cpu_baseline"] = {"value": tok_s / 1e6, "unit": "Mtok/s", "cores": cores,
+                                "kind": "oracle", "sample": sample, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,429 @@
+// la_api.cu -- the C ABI declared in include/la.h: argument validation,
+// planning of the span-parallel prefill, tensor-map construction, launches,
+// and the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "la.h"
+#include "la_internal.h"
+#include "la_ptx.cuh"
+
+#define LA_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace la {
+
+// Device status word (LA_DEV_* bits) and a flag nothing ever sets (waited on by
+// the self-test).  One copy per device that loads the library.
+__device__ unsigned g_status;
+__device__ unsigned g_never_set;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned* g_status_ptr[kMaxDevices];
+int g_num_sms[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Per-device device address of g_status and SM count, looked up once.
+bool device_info(unsigned** status, int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return false;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return false;
+    g_num_sms[dev] = n;
+    g_status_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  if (status) *status = g_status_ptr[dev];
+  if (sms) *sms = g_num_sms[dev];
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Common shape checks of the prefill entry points.
+la_status check_shape(int B, int Hq, int Hkv, int64_t N, int d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return LA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return LA_ERR_INVALID_ARG;
+  // bulk tensor copies take int32 coordinates
+  if (N > (int64_t)0x7fff0000 || (int64_t)B * Hq > 0x7fffffff) return LA_ERR_INVALID_ARG;
+  return LA_OK;
+}
+
+la_status plan_impl(int B, int Hq, int Hkv, int64_t N, int d, int chunk, int sms, la_plan* out) {
+  la_status st = check_shape(B, Hq, Hkv, N, d);
+  if (st != LA_OK) return st;
+  if (d != kHeadDim || (chunk != 64 && chunk != 128)) return LA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  int T, HPT;
+  if (chunk == 64 && G % 2 == 0) {
+    T = 64;
+    HPT = 2;  // two query heads x 64 tokens
+  } else {
+    T = 128;  // one head x 128 tokens (two 64-token chunks stacked when chunk == 64)
+    HPT = 1;
+  }
+  const int64_t tiles = (N + T - 1) / T;
+  const int64_t units = (int64_t)B * Hkv * (G / HPT);
+  // Pick the span count: the main kernel runs units * nspan CTAs, one per SM
+  // at a time; estimated time ~ waves * (tiles per span + a fixed per-CTA cost
+  // of about three tiles).
+  const int64_t max_span = std::min<int64_t>(tiles, 4096);
+  int64_t best = 1;
+  double best_cost = 1e300;
+  for (int64_t ns = 1; ns <= max_span; ++ns) {
+    const int64_t ctas = units * ns;
+    if (ctas > 0x7fffffff) break;
+    const int64_t waves = (ctas + sms - 1) / sms;
+    const int64_t per = (tiles + ns - 1) / ns;
+    const double cost = (double)waves * (double)(per + 3);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = ns;
+    }
+  }
+  out->nspan = (int32_t)best;
+  out->tile = T;
+  out->heads_per_tile = HPT;
+  out->tiles_total = (int32_t)tiles;
+  out->workspace_bytes = (int64_t)B * Hkv * best * d * d * (int64_t)sizeof(float);
+  return LA_OK;
+}
+
+// A caller-supplied plan must describe this problem.
+la_status check_plan(const la_plan* p, int B, int Hq, int Hkv, int64_t N, int d) {
+  if (!p) return LA_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (!((p->tile == 64 && p->heads_per_tile == 2) || (p->tile == 128 && p->heads_per_tile == 1)))
+    return LA_ERR_INVALID_ARG;
+  if (G % p->heads_per_tile != 0) return LA_ERR_INVALID_ARG;
+  if ((int64_t)p->tiles_total != (N + p->tile - 1) / p->tile) return LA_ERR_INVALID_ARG;
+  if (p->nspan < 1 || p->nspan > p->tiles_total) return LA_ERR_INVALID_ARG;
+  if (p->workspace_bytes != (int64_t)B * Hkv * p->nspan * d * d * (int64_t)sizeof(float))
+    return LA_ERR_INVALID_ARG;
+  if ((int64_t)B * Hkv * p->nspan * (G / p->heads_per_tile) > 0x7fffffff) return LA_ERR_INVALID_ARG;
+  return LA_OK;
+}
+
+PrefillGeometry geometry(const la_plan* p, int B, int Hq, int Hkv, int64_t N) {
+  PrefillGeometry g;
+  g.B = B;
+  g.Hq = Hq;
+  g.Hkv = Hkv;
+  g.G = Hq / Hkv;
+  g.N = N;
+  g.tile = p->tile;
+  g.heads_per_tile = p->heads_per_tile;
+  g.tiles_total = p->tiles_total;
+  g.nspan = p->nspan;
+  return g;
+}
+
+la_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+// Pointer checks of a bf16 prefill call: present, 16-byte aligned, o (and S)
+// disjoint from everything else.
+la_status check_prefill_ptrs(const void* q, const void* k, const void* v, const void* o,
+                             const void* S, int B, int Hq, int Hkv, int64_t N, int d) {
+  if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LA_ERR_INVALID_ARG;
+  if (S && !aligned16(S)) return LA_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * N * d * 2, kbytes = (size_t)B * Hkv * N * d * 2,
+               sbytes = (size_t)B * Hkv * d * d * 4;
+  if (overlap(o, qbytes, q, qbytes) || overlap(o, qbytes, k, kbytes) ||
+      overlap(o, qbytes, v, kbytes) || overlap(o, qbytes, S, sbytes) ||
+      overlap(S, sbytes, q, qbytes) || overlap(S, sbytes, k, kbytes) ||
+      overlap(S, sbytes, v, kbytes))
+    return LA_ERR_INVALID_ARG;
+  return LA_OK;
+}
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, int64_t heads,
+                    int box_rows) {
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows_per_head, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2,
+                                 (cuuint64_t)rows_per_head * kHeadDim * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+__global__ void selftest_wait_kernel(unsigned* status, const unsigned* flag, int64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (*reinterpret_cast<const volatile unsigned*>(flag) == 0u) {
+    if (globaltimer_ns() - t0 > (uint64_t)limit_ns) {
+      if (threadIdx.x == 0) atomicOr(status, kDevTimeout);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_selftest_wait(unsigned* status, int64_t timeout_ns, cudaStream_t stream) {
+  void* flag = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&flag, g_never_set);
+  if (e != cudaSuccess) return e;
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(status, static_cast<const unsigned*>(flag),
+                                             timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace la
+
+using namespace la;
+
+// ---------------------------------------------------------------------------
+LA_EXPORT const char* la_status_string(la_status s) {
+  switch (s) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA";
+    case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE";
+  }
+  return "LA_ERR_UNKNOWN";
+}
+
+LA_EXPORT int la_version(void) { return 1; }
+
+LA_EXPORT la_status la_prefill_plan(int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                                    la_plan* plan) {
+  if (!plan) return LA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (!device_info(nullptr, &sms)) return LA_ERR_CUDA;
+  return plan_impl(B, Hq, Hkv, N, d, chunk, sms, plan);
+}
+
+LA_EXPORT size_t la_forward_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d, int chunk) {
+  la_plan p;
+  if (la_prefill_plan(B, Hq, Hkv, N, d, chunk, &p) != LA_OK) return 0;
+  return (size_t)p.workspace_bytes;
+}
+
+LA_EXPORT la_status la_prefill_span_states(const la_bf16* k, const la_bf16* v, int B, int Hkv,
+                                           int64_t N, int d, const la_plan* plan, float* ws,
+                                           la_stream stream) {
+  la_status st = check_shape(B, Hkv, Hkv, N, d);
+  if (st != LA_OK) return st;
+  if (d != kHeadDim) return LA_ERR_UNSUPPORTED;
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return LA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_ERR_WORKSPACE;
+  if (!plan || plan->nspan < 1 || plan->nspan > plan->tiles_total) return LA_ERR_INVALID_ARG;
+  if (!((plan->tile == 64 && plan->heads_per_tile == 2) ||
+        (plan->tile == 128 && plan->heads_per_tile == 1)) ||
+      (int64_t)plan->tiles_total != (N + plan->tile - 1) / plan->tile)
+    return LA_ERR_INVALID_ARG;
+  unsigned* status = nullptr;
+  if (!device_info(&status, nullptr)) return LA_ERR_CUDA;
+  PrefillMaps maps;
+  const int64_t heads = (int64_t)B * Hkv;
+  if (!make_tmap_bf16(&maps.k, k, N, heads, plan->tile) ||
+      !make_tmap_bf16(&maps.v, v, N, heads, plan->tile))
+    return LA_ERR_CUDA;
+  PrefillGeometry g = geometry(plan, B, Hkv, Hkv, N);
+  return from_cuda(
+      launch_span_states(g, maps.k, maps.v, ws, status, static_cast<cudaStream_t>(stream)));
+}
+
+LA_EXPORT la_status la_prefill_scan(float* ws, float* S, int B, int Hkv, int d,
+                                    const la_plan* plan, la_stream stream) {
+  if (B <= 0 || Hkv <= 0 || d != kHeadDim) return d != kHeadDim ? LA_ERR_UNSUPPORTED
+                                                                 : LA_ERR_INVALID_ARG;
+  if (!plan || plan->nspan < 1) return LA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_ERR_WORKSPACE;
+  if (S && !aligned16(S)) return LA_ERR_INVALID_ARG;
+  return from_cuda(
+      launch_state_scan(ws, S, B * Hkv, plan->nspan, d, static_cast<cudaStream_t>(stream)));
+}
+
+LA_EXPORT la_status la_prefill_main(const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                                    la_bf16* o, const float* ws, int B, int Hq, int Hkv,
+                                    int64_t N, int d, const la_plan* plan, la_stream stream) {
+  la_status st = check_shape(B, Hq, Hkv, N, d);
+  if (st != LA_OK) return st;
+  if (d != kHeadDim) return LA_ERR_UNSUPPORTED;
+  if ((st = check_prefill_ptrs(q, k, v, o, nullptr, B, Hq, Hkv, N, d)) != LA_OK) return st;
+  if ((st = check_plan(plan, B, Hq, Hkv, N, d)) != LA_OK) return st;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return LA_ERR_WORKSPACE;
+  unsigned* status = nullptr;
+  if (!device_info(&status, nullptr)) return LA_ERR_CUDA;
+  PrefillMaps maps;
+  if (!make_tmap_bf16(&maps.q, q, N, (int64_t)B * Hq, plan->tile) ||
+      !make_tmap_bf16(&maps.o, o, N, (int64_t)B * Hq, plan->tile) ||
+      !make_tmap_bf16(&maps.k, k, N, (int64_t)B * Hkv, plan->tile) ||
+      !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan->tile))
+    return LA_ERR_CUDA;
+  PrefillGeometry g = geometry(plan, B, Hq, Hkv, N);
+  return from_cuda(launch_prefill_main(g, maps, ws, status, static_cast<cudaStream_t>(stream)));
+}
+
+LA_EXPORT la_status la_forward_ws(const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                                  la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N, int d,
+                                  int chunk, void* workspace, size_t workspace_bytes,
+                                  la_stream stream) {
+  if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  la_plan plan;
+  la_status st = la_prefill_plan(B, Hq, Hkv, N, d, chunk, &plan);
+  if (st != LA_OK) return st;
+  if ((st = check_prefill_ptrs(q, k, v, o, S, B, Hq, Hkv, N, d)) != LA_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < (size_t)plan.workspace_bytes)
+    return LA_ERR_WORKSPACE;
+  float* ws = static_cast<float*>(workspace);
+  if ((st = la_prefill_span_states(k, v, B, Hkv, N, d, &plan, ws, stream)) != LA_OK) return st;
+  if ((st = la_prefill_scan(ws, S, B, Hkv, d, &plan, stream)) != LA_OK) return st;
+  return la_prefill_main(q, k, v, o, ws, B, Hq, Hkv, N, d, &plan, stream);
+}
+
+LA_EXPORT la_status la_forward_state(const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                                     la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N,
+                                     int d, int chunk, la_stream stream) {
+  if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  la_plan plan;
+  la_status st = la_prefill_plan(B, Hq, Hkv, N, d, chunk, &plan);
+  if (st != LA_OK) return st;
+  if ((st = check_prefill_ptrs(q, k, v, o, S, B, Hq, Hkv, N, d)) != LA_OK) return st;
+  // Stream-ordered workspace from the device's default memory pool, kept
+  // cached by the pool between calls (release threshold raised once).
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  {
+    static std::once_flag once[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LA_ERR_CUDA;
+    std::call_once(once[dev], [dev]() {
+      cudaMemPool_t pool;
+      if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+        uint64_t keep = ~0ull;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+      }
+    });
+  }
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, (size_t)plan.workspace_bytes, s) != cudaSuccess) return LA_ERR_CUDA;
+  st = la_forward_ws(q, k, v, o, S, B, Hq, Hkv, N, d, chunk, ws, (size_t)plan.workspace_bytes,
+                     stream);
+  if (cudaFreeAsync(ws, s) != cudaSuccess && st == LA_OK) st = LA_ERR_CUDA;
+  return st;
+}
+
+LA_EXPORT la_status la_forward(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
+                               int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                               la_stream stream) {
+  return la_forward_state(q, k, v, o, nullptr, B, Hq, Hkv, N, d, chunk, stream);
+}
+
+LA_EXPORT la_status la_forward_f32(const float* q, const float* k, const float* v, float* o,
+                                   float* S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                                   la_stream stream) {
+  la_status st = check_shape(B, Hq, Hkv, N, d);
+  if (st != LA_OK) return st;
+  if ((d != 64 && d != 128) || (chunk != 64 && chunk != 128)) return LA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (S && !aligned16(S)))
+    return LA_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * N * d * 4, kbytes = (size_t)B * Hkv * N * d * 4,
+               sbytes = (size_t)B * Hkv * d * d * 4;
+  if (overlap(o, qbytes, q, qbytes) || overlap(o, qbytes, k, kbytes) ||
+      overlap(o, qbytes, v, kbytes) || overlap(o, qbytes, S, sbytes))
+    return LA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* S_in = nullptr;
+  if (S) {  // the kernel reads the initial state from a copy and writes S
+    if (cudaMallocAsync(reinterpret_cast<void**>(&S_in), sbytes, s) != cudaSuccess)
+      return LA_ERR_CUDA;
+    if (cudaMemcpyAsync(S_in, S, sbytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+      cudaFreeAsync(S_in, s);
+      return LA_ERR_CUDA;
+    }
+  }
+  st = from_cuda(launch_forward_simt_f32(q, k, v, o, S_in, S, B, Hq, Hkv, N, d, chunk, s));
+  if (S_in) cudaFreeAsync(S_in, s);
+  return st;
+}
+
+LA_EXPORT la_status la_decode_step(float* S, const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                                   la_bf16* o, int B, int Hq, int Hkv, int d, la_stream stream) {
+  if (!S || !q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0) return LA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 32) return LA_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv > 0x7fffffff) return LA_ERR_INVALID_ARG;
+  if (!aligned16(S) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return LA_ERR_INVALID_ARG;
+  const size_t sbytes = (size_t)B * Hkv * d * d * 4, qbytes = (size_t)B * Hq * d * 2,
+               kbytes = (size_t)B * Hkv * d * 2;
+  if (overlap(o, qbytes, S, sbytes) || overlap(o, qbytes, q, qbytes) ||
+      overlap(o, qbytes, k, kbytes) || overlap(o, qbytes, v, kbytes) ||
+      overlap(S, sbytes, q, qbytes) || overlap(S, sbytes, k, kbytes) ||
+      overlap(S, sbytes, v, kbytes))
+    return LA_ERR_INVALID_ARG;
+  return from_cuda(
+      launch_decode(S, q, k, v, o, B, Hq, Hkv, d, static_cast<cudaStream_t>(stream)));
+}
+
+LA_EXPORT la_status la_device_status(unsigned int* flags, int clear) {
+  if (!flags) return LA_ERR_INVALID_ARG;
+  *flags = 0;
+  if (!device_info(nullptr, nullptr)) return LA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LA_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return LA_ERR_CUDA;
+  if (clear) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return LA_ERR_CUDA;
+  }
+  *flags = v;
+  return (v & LA_DEV_TIMEOUT) ? LA_ERR_TIMEOUT : LA_OK;
+}
+
+LA_EXPORT la_status la_selftest_wait(int64_t timeout_ns, la_stream stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return LA_ERR_INVALID_ARG;
+  unsigned* status = nullptr;
+  if (!device_info(&status, nullptr)) return LA_ERR_CUDA;
+  return from_cuda(launch_selftest_wait(status, timeout_ns, static_cast<cudaStream_t>(stream)));
+}
+
+LA_EXPORT void la_shutdown(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  cudaMemPool_t pool;
+  if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) cudaMemPoolTrimTo(pool, 0);
+}

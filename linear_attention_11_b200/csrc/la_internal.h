@@ -1,0 +1,47 @@
+// la_internal.h -- launch helpers shared by the translation units of the
+// library (host side only; not part of the public ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace la {
+
+constexpr int kHeadDim = 128;   // head dim of the tensor-core path
+constexpr int kTileRows = 128;  // rows of one tcgen05 M=128 tile
+
+struct PrefillGeometry {
+  int B, Hq, Hkv, G;
+  int64_t N;
+  int tile;            // tokens per tile (T)
+  int heads_per_tile;  // HPT, tile * HPT == 128
+  int tiles_total;     // ceil(N / T)
+  int nspan;           // spans per (b, kv head)
+};
+
+// Tensor maps for one call: q, o over [B*Hq, N, 128]; k, v over [B*Hkv, N, 128];
+// box {64, tile, 1}, 128-byte swizzle, bf16.
+struct PrefillMaps {
+  CUtensorMap q, k, v, o;
+};
+
+// Builds a 3-D bf16 tensor map; returns false on failure.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, int64_t heads,
+                    int box_rows);
+
+cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
+                               const CUtensorMap& v, float* ws, unsigned* status,
+                               cudaStream_t stream);
+cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
+                                const float* ws, unsigned* status, cudaStream_t stream);
+cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
+                              cudaStream_t stream);
+cudaError_t launch_decode(float* S, const void* q, const void* k, const void* v, void* o, int B,
+                          int Hq, int Hkv, int d, cudaStream_t stream);
+cudaError_t launch_forward_simt_f32(const float* q, const float* k, const float* v, float* o,
+                                    const float* S_in, float* S_out, int B, int Hq, int Hkv,
+                                    int64_t N, int d, int chunk, cudaStream_t stream);
+cudaError_t launch_selftest_wait(unsigned* status, int64_t timeout_ns, cudaStream_t stream);
+
+}  // namespace la

@@ -1,0 +1,59 @@
+// la_scan.cu -- exclusive prefix over span states (the second prefill stage).
+//
+// The state entering span j of a (batch, kv head) is S0 + sum_{i<j} K_i^T V_i,
+// where K_i^T V_i is span i's contribution; the state after the last span is
+// the final state S0 + K^T V ("MiniMax-01与Lightning Attention", section 2.2,
+// kv_sum over the whole sequence).  Elementwise fp32 adds, HBM/L2-bound: one
+// thread owns one float4 of the d x d matrix of one unit and walks the spans
+// in order, loading eight spans ahead to keep loads in flight.
+#include <cuda_runtime.h>
+
+#include "la_internal.h"
+
+namespace la {
+namespace {
+
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__global__ void __launch_bounds__(256)
+    state_scan_kernel(float4* __restrict__ ws, float4* __restrict__ S, int nspan, int n4,
+                      int blocks_per_unit) {
+  const size_t unit = blockIdx.x / blocks_per_unit;
+  const int p = (blockIdx.x % blocks_per_unit) * blockDim.x + threadIdx.x;
+  if (p >= n4) return;
+  float4* w = ws + unit * (size_t)nspan * n4 + p;
+  float4 carry = S ? S[unit * n4 + p] : make_float4(0.f, 0.f, 0.f, 0.f);
+  int j = 0;
+  for (; j + 8 <= nspan; j += 8) {
+    float4 x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = w[(size_t)(j + u) * n4];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      w[(size_t)(j + u) * n4] = carry;
+      carry = add4(carry, x[u]);
+    }
+  }
+  for (; j < nspan; ++j) {
+    const float4 x = w[(size_t)j * n4];
+    w[(size_t)j * n4] = carry;
+    carry = add4(carry, x);
+  }
+  if (S) S[unit * n4 + p] = carry;
+}
+
+}  // namespace
+
+cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
+                              cudaStream_t stream) {
+  const int n4 = d * d / 4;
+  const int bpu = (n4 + 255) / 256;
+  const dim3 grid((unsigned)(units * bpu));
+  state_scan_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<float4*>(ws),
+                                              reinterpret_cast<float4*>(S), nspan, n4, bpu);
+  return cudaGetLastError();
+}
+
+}  // namespace la

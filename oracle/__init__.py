@@ -15,7 +15,8 @@ Functions
 quadratic(q, k, v)        masked form, all rows:  O[t] = sum_{s<=t} (q_t.k_s) v_s
 rows(q, k, v, rows)       the same sum at selected (b, h, t) rows only
 recurrent(q, k, v, S0)    token recurrence S += k^T v; o = q S; returns (O, S)
-state(k, v)               S = K^T V
+state(k, v)               S = K^T V (scalar loops)
+state_gemm(k, v)          S = K^T V (one fp64 matmul per head, for long sequences)
 decode(S, q, k, v)        one decode step on a copy of S; returns (o, S_new)
 
 Inputs may be torch CPU tensors (float32 or bfloat16) or numpy arrays
@@ -53,7 +54,7 @@ def _bind(path: str):
     lib.la_oracle_rows.argtypes = [P, P, P, I, I, I, I, L, I, P, L, P, I]
     lib.la_oracle_recurrent.argtypes = [P, P, P, I, I, I, I, L, I, P, P, P, P, I]
     lib.la_oracle_state.argtypes = [P, P, I, I, I, L, I, P, I]
-    lib.la_oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, P]
+    lib.la_oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, P, I]
     for f in (lib.la_oracle_quadratic, lib.la_oracle_rows, lib.la_oracle_recurrent,
               lib.la_oracle_state, lib.la_oracle_decode):
         f.restype = ctypes.c_int
@@ -171,16 +172,49 @@ def state(k, v, nthreads: int | None = None) -> np.ndarray:
     return S
 
 
-def decode(S, q, k, v):
-    """One step on a float64 copy of S.  q [B,Hq,d]; k, v [B,Hkv,d].  Returns (o, S_new)."""
+def state_gemm(k, v) -> np.ndarray:
+    """S = K^T V for each (b, kv head) as one fp64 library GEMM per head.
+
+    The same definition as ``state`` ("MiniMax-01与Lightning Attention",
+    section 2.2: kv_sum over the sequence axis) with numpy's matmul as the
+    summation step; used for very long sequences where the scalar loop would
+    take minutes."""
+    (ka, kt), (va, vt) = _as_array(k), _as_array(v)
+    if kt != vt or ka.shape != va.shape:
+        raise ValueError("k, v must match")
+    B, Hkv, N, d = ka.shape
+    S = np.empty((B, Hkv, d, d), np.float64)
+    for b in range(B):
+        for g in range(Hkv):
+            kd, vd = _widen(ka[b, g], kt), _widen(va[b, g], vt)
+            S[b, g] = kd.T @ vd
+    return S
+
+
+def _widen(a, dt):
+    """Exact widening of fp32 values or bf16 bits to float64."""
+    if dt == BF16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def decode(S, q, k, v, nthreads: int | None = None, inplace: bool = False):
+    """One step.  q [B,Hq,d]; k, v [B,Hkv,d].  Returns (o, S_new).
+
+    S_new is a float64 copy of S after the update, or S itself when ``inplace``
+    and S is already a C-contiguous float64 array."""
     (qa, qt), (ka, kt), (va, vt) = _as_array(q), _as_array(k), _as_array(v)
     if not (qt == kt == vt):
         raise TypeError("q, k, v must share one dtype")
     B, Hq, d = qa.shape
     Hkv = ka.shape[1]
-    Sn = np.array(np.asarray(S, dtype=np.float64).reshape(B, Hkv, d, d), copy=True, order="C")
+    if inplace and isinstance(S, np.ndarray) and S.dtype == np.float64 and S.flags.c_contiguous:
+        Sn = S
+    else:
+        Sn = np.array(np.asarray(S, dtype=np.float64).reshape(B, Hkv, d, d), copy=True, order="C")
     o = np.empty((B, Hq, d), np.float64)
-    rc = load().la_oracle_decode(_ptr(Sn), _ptr(qa), _ptr(ka), _ptr(va), qt, B, Hq, Hkv, d, _ptr(o))
+    rc = load().la_oracle_decode(_ptr(Sn), _ptr(qa), _ptr(ka), _ptr(va), qt, B, Hq, Hkv, d, _ptr(o),
+                                 nthreads or threads())
     if rc:
         raise ValueError(f"la_oracle_decode rc={rc}")
     return o, Sn

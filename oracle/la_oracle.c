@@ -253,28 +253,39 @@ int la_oracle_state(const void *k, const void *v, int dtype, int B, int Hkv, int
 }
 
 /* ---- decode step: S (in/out, [B,Hkv,d,d]) += k^T v; o_h = q_h S -------- */
-/* q,o [B,Hq,d]; k,v [B,Hkv,d].                                              */
+/* q,o [B,Hq,d]; k,v [B,Hkv,d].  One unit = one (b, kv head).                */
+
+typedef struct {
+  double *S;
+  const void *q, *k, *v;
+  int dtype, Hq, Hkv, d;
+  double *o;
+} decode_job;
+
+static void decode_unit(void *ctx, int64_t unit) {
+  decode_job *J = (decode_job *)ctx;
+  const int G = J->Hq / J->Hkv;
+  const int64_t b = unit / J->Hkv, g = unit % J->Hkv, d = J->d;
+  double *Sg = J->S + unit * d * d;
+  const int64_t kv = unit * d;
+  for (int64_t i = 0; i < d; ++i) { /* S += k^T v */
+    const double ki = elem(J->k, kv + i, J->dtype);
+    for (int64_t j = 0; j < d; ++j) Sg[i * d + j] += ki * elem(J->v, kv + j, J->dtype);
+  }
+  for (int hh = 0; hh < G; ++hh) { /* o_h = q_h S */
+    const int64_t qo = (b * J->Hq + g * G + hh) * d;
+    for (int64_t j = 0; j < d; ++j) J->o[qo + j] = 0.0;
+    for (int64_t i = 0; i < d; ++i) {
+      const double qi = elem(J->q, qo + i, J->dtype);
+      for (int64_t j = 0; j < d; ++j) J->o[qo + j] += qi * Sg[i * d + j];
+    }
+  }
+}
 
 int la_oracle_decode(double *S, const void *q, const void *k, const void *v, int dtype, int B,
-                     int Hq, int Hkv, int d, double *o) {
+                     int Hq, int Hkv, int d, double *o, int nthreads) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv || !S || !o) return 1;
-  const int G = Hq / Hkv;
-  for (int64_t b = 0; b < B; ++b)
-    for (int64_t g = 0; g < Hkv; ++g) {
-      double *Sg = S + (b * Hkv + g) * d * d;
-      const int64_t kv = (b * Hkv + g) * d;
-      for (int64_t i = 0; i < d; ++i) {
-        const double ki = elem(k, kv + i, dtype);
-        for (int64_t j = 0; j < d; ++j) Sg[i * d + j] += ki * elem(v, kv + j, dtype);
-      }
-      for (int hh = 0; hh < G; ++hh) {
-        const int64_t qo = (b * Hq + g * G + hh) * d;
-        for (int64_t j = 0; j < d; ++j) o[qo + j] = 0.0;
-        for (int64_t i = 0; i < d; ++i) {
-          const double qi = elem(q, qo + i, dtype);
-          for (int64_t j = 0; j < d; ++j) o[qo + j] += qi * Sg[i * d + j];
-        }
-      }
-    }
+  decode_job J = {S, q, k, v, dtype, Hq, Hkv, d, o};
+  parallel_units(decode_unit, &J, (int64_t)B * Hkv, nthreads);
   return 0;
 }

@@ -1,0 +1,61 @@
+"""Decode step on the GPU against the fp64 oracle's decode step."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_11_b200 import synth
+
+from _compare import assert_bf16_close, assert_f32_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d", [(3, 4, 2, 128), (2, 6, 3, 64), (1, 32, 1, 128), (5, 1, 1, 64)])
+def test_decode_small(la, B, Hq, Hkv, d):
+    w = synth.Decode("t", B, Hq, Hkv, d, 5, 9)
+    S = synth.decode_state(w)
+    Sref = S.double().numpy().copy()
+    Sd = S.to(DEV)
+    for step in range(w.steps):
+        q, k, v = synth.decode_token(w, step)
+        o_ref, Sref = oracle.decode(Sref, q, k, v)
+        o = la.la_decode_step(Sd, q.to(DEV), k.to(DEV), v.to(DEV))
+        torch.cuda.synchronize()
+        assert_bf16_close(o.cpu(), o_ref, f"o step {step}")
+    assert_f32_close(Sd.cpu(), Sref, "state", tol=1e-6)
+
+
+def test_decode_continues_prefill(la):
+    """Prefill N tokens, then decode the next ones: rows equal one longer prefill."""
+    B, Hq, Hkv, N, extra = 1, 4, 2, 300, 6
+    q, k, v = synth.random_qkv(B, Hq, Hkv, N + extra, 128, torch.bfloat16, 77)
+    ref_o, ref_S = oracle.recurrent(q, k, v)
+    S = torch.zeros(B, Hkv, 128, 128, device=DEV)
+    qd, kd, vd = (t.to(DEV) for t in (q, k, v))
+    la.la_forward_state(*(t[:, :, :N].contiguous() for t in (qd, kd, vd)), S=S, chunk=64)
+    for t in range(N, N + extra):
+        o = la.la_decode_step(S, qd[:, :, t].contiguous(), kd[:, :, t].contiguous(),
+                              vd[:, :, t].contiguous())
+        torch.cuda.synchronize()
+        assert_bf16_close(o.cpu(), ref_o[:, :, t], f"decode row {t}")
+    assert_f32_close(S.cpu(), ref_S, "state after decode", tol=1e-6)
+
+
+def test_decode_full_b256_64_steps(la):
+    """The decode workload: B=256, Hq=64/Hkv=16, d=128, 64 consecutive steps."""
+    w = synth.DECODE_B256
+    S = synth.decode_state(w)
+    Sref = np.ascontiguousarray(S.double().numpy())
+    Sd = S.to(DEV)
+    worst = 0.0
+    for step in range(w.steps):
+        q, k, v = synth.decode_token(w, step)
+        o_ref, Sref = oracle.decode(Sref, q, k, v, inplace=True)
+        o = la.la_decode_step(Sd, q.to(DEV), k.to(DEV), v.to(DEV))
+        torch.cuda.synchronize()
+        rel, _ = assert_bf16_close(o.cpu(), o_ref, f"o step {step}")
+        worst = max(worst, rel)
+    assert_f32_close(Sd.cpu(), Sref, "state after 64 steps", tol=1e-6)

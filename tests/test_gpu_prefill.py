@@ -1,0 +1,215 @@
+"""bf16 prefill on the GPU (tcgen05 kernels, called through the C ABI) against
+the fp64 oracle.
+
+Stage by stage first (span states, scan, main pass), then whole calls on small
+ragged shapes that span several tiles, then the full-size workloads in the
+launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_11_b200 import synth
+
+from _compare import STATE_REL_L2, assert_bf16_close, assert_f32_close, errors
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _qkv(B, Hq, Hkv, N, seed, d=128):
+    return synth.random_qkv(B, Hq, Hkv, N, d, torch.bfloat16, seed)
+
+
+def _cuda(*ts):
+    return [t.to(DEV) for t in ts]
+
+
+def _span_bounds(plan, j):
+    b = (j * plan.tiles_total) // plan.nspan * plan.tile
+    e = ((j + 1) * plan.tiles_total) // plan.nspan * plan.tile
+    return b, e
+
+
+@pytest.mark.parametrize("Hq,Hkv,N,chunk", [(2, 2, 700, 64), (4, 2, 1000, 64), (4, 1, 520, 128)])
+def test_span_states_and_scan(la, Hq, Hkv, N, chunk):
+    B = 2
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=100 + N)
+    kd, vd = _cuda(k, v)
+    for nspan in (1, 3, None):
+        plan = la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk)
+        if nspan is not None:
+            plan.nspan = min(nspan, plan.tiles_total)
+            plan.workspace_bytes = B * Hkv * plan.nspan * 128 * 128 * 4
+        ws = torch.empty(B, Hkv, plan.nspan, 128, 128, dtype=torch.float32, device=DEV)
+        la.api.la_prefill_span_states(kd, vd, plan, ws)
+        torch.cuda.synchronize()
+        got = ws.cpu()
+        for j in range(plan.nspan):
+            b0, b1 = _span_bounds(plan, j)
+            ref = oracle.state_gemm(k[:, :, b0:min(b1, N)], v[:, :, b0:min(b1, N)])
+            assert_f32_close(got[:, :, j], ref, f"span state {j}/{plan.nspan}", tol=STATE_REL_L2)
+        # scan with an initial state
+        S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(5))
+        S = S0.to(DEV)
+        la.api.la_prefill_scan(ws, S, plan, B, Hkv, 128)
+        torch.cuda.synchronize()
+        got = ws.cpu()
+        for j in range(plan.nspan):
+            b0, _ = _span_bounds(plan, j)
+            ref = S0.double().numpy() + (oracle.state_gemm(k[:, :, :b0], v[:, :, :b0]) if b0 else 0)
+            assert_f32_close(got[:, :, j], ref, f"entering state {j}", tol=STATE_REL_L2)
+        ref = S0.double().numpy() + oracle.state_gemm(k, v)
+        assert_f32_close(S.cpu(), ref, "final state", tol=STATE_REL_L2)
+
+
+SMALL = [
+    # B, Hq, Hkv, N, chunk  -- tile = 64 needs an even group; other cases use 128-token tiles
+    (1, 1, 1, 1, 64),
+    (1, 2, 2, 63, 64),
+    (1, 2, 1, 64, 64),
+    (1, 2, 1, 65, 64),
+    (2, 2, 2, 300, 64),      # single-head groups at chunk 64: two chunks per tile
+    (2, 4, 2, 777, 64),      # two query heads per tile, ragged tail
+    (1, 8, 2, 1000, 64),     # GQA 4:1
+    (1, 8, 2, 1000, 128),
+    (1, 3, 1, 385, 64),      # odd group -> 128-token tiles
+    (3, 6, 3, 129, 128),
+    (1, 4, 4, 2048, 128),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,chunk", SMALL)
+def test_forward_small(la, B, Hq, Hkv, N, chunk):
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=N * 7 + Hq)
+    ref = oracle.quadratic(q, k, v)
+    qd, kd, vd = _cuda(q, k, v)
+    o = la.la_forward(qd, kd, vd, chunk=chunk)
+    torch.cuda.synchronize()
+    assert_bf16_close(o.cpu(), ref, f"O {B}x{Hq}/{Hkv}x{N} chunk {chunk}")
+    assert la.la_device_status()[1] == 0
+
+
+@pytest.mark.parametrize("nspan", [1, 2, 5, 16])
+def test_span_count_does_not_change_result(la, nspan):
+    B, Hq, Hkv, N, chunk = 1, 4, 2, 1024, 64
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=31)
+    ref = oracle.quadratic(q, k, v)
+    qd, kd, vd = _cuda(q, k, v)
+    plan = la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk)
+    plan.nspan = nspan
+    plan.workspace_bytes = B * Hkv * nspan * 128 * 128 * 4
+    ws = torch.empty(plan.workspace_bytes // 4, dtype=torch.float32, device=DEV)
+    o = torch.empty_like(qd)
+    la.api.la_prefill_span_states(kd, vd, plan, ws)
+    la.api.la_prefill_scan(ws, None, plan, B, Hkv, 128)
+    la.api.la_prefill_main(qd, kd, vd, o, ws, plan)
+    torch.cuda.synchronize()
+    assert_bf16_close(o.cpu(), ref, f"nspan={nspan}")
+
+
+def test_state_in_out_and_resume(la):
+    B, Hq, Hkv, N, chunk = 2, 4, 2, 900, 64
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=41)
+    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(42)) / 128
+    ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy())
+    qd, kd, vd = _cuda(q, k, v)
+    S = S0.to(DEV)
+    o = la.la_forward_state(qd, kd, vd, S=S, chunk=chunk)
+    torch.cuda.synchronize()
+    assert_bf16_close(o.cpu(), ref_o, "O with initial state")
+    assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
+    # the same sequence in two pieces, carrying the state
+    cut = 333
+    S2 = S0.to(DEV)
+    o1 = la.la_forward_state(*(t[:, :, :cut].contiguous() for t in (qd, kd, vd)), S=S2, chunk=chunk)
+    o2 = la.la_forward_state(*(t[:, :, cut:].contiguous() for t in (qd, kd, vd)), S=S2, chunk=chunk)
+    torch.cuda.synchronize()
+    assert_bf16_close(torch.cat([o1, o2], dim=2).cpu(), ref_o, "resumed O")
+    assert_f32_close(S2.cpu(), ref_S, "resumed final state", tol=STATE_REL_L2)
+
+
+def test_chunk_sizes_agree(la):
+    q, k, v = _cuda(*_qkv(1, 8, 2, 1500, seed=51))
+    a = la.la_forward(q, k, v, chunk=64)
+    b = la.la_forward(q, k, v, chunk=128)
+    torch.cuda.synchronize()
+    assert_bf16_close(a.cpu(), b.cpu(), "chunk 64 vs 128")
+
+
+def test_forward_ws_and_workspace_errors(la):
+    B, Hq, Hkv, N = 1, 4, 2, 500
+    q, k, v = _cuda(*_qkv(B, Hq, Hkv, N, seed=61))
+    nbytes = la.api.la_forward_workspace_bytes(B, Hq, Hkv, N, 128, 64)
+    assert nbytes > 0
+    ws = torch.empty(nbytes // 4, dtype=torch.float32, device=DEV)
+    o = torch.empty_like(q)
+    la.api.la_forward_ws(q, k, v, o, None, ws, chunk=64)
+    ref = la.la_forward(q, k, v, chunk=64)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref)
+    small = torch.empty(nbytes // 8, dtype=torch.float32, device=DEV)
+    with pytest.raises(la.LAError) as e:
+        la.api.la_forward_ws(q, k, v, o, None, small, chunk=64)
+    assert e.value.code == 5
+
+
+def test_argument_errors_on_device(la):
+    q, k, v = _cuda(*_qkv(1, 2, 2, 64, seed=71))
+    with pytest.raises(la.LAError) as e:
+        la.la_forward(q, k, v, o=q)  # output aliases an input
+    assert e.value.code == 1
+    with pytest.raises(la.LAError) as e:
+        la.la_forward(q, k, v, chunk=32)
+    assert e.value.code == 2
+    q64 = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(la.LAError) as e:
+        la.la_forward(q64, q64.clone(), q64.clone())
+    assert e.value.code == 2
+    raw = la.api.load_library()
+    base = torch.zeros(1 << 16, dtype=torch.bfloat16, device=DEV)
+    mis = base.data_ptr() + 2  # not 16-byte aligned
+    rc = raw.la_forward(mis, k.data_ptr(), v.data_ptr(), base.data_ptr() + 4096 * 2, 1, 2, 2, 64,
+                        128, 64, None)
+    assert rc == 1
+
+
+# ------------------------------------------------------------------ full size
+def _full(la, w, chunk, rows_only=False):
+    q, k, v = synth.prefill_inputs(w)
+    qd, kd, vd = _cuda(q, k, v)
+    S = torch.zeros(w.B, w.Hkv, 128, 128, dtype=torch.float32, device=DEV)
+    o = la.la_forward_state(qd, kd, vd, S=S, chunk=chunk)
+    torch.cuda.synchronize()
+    assert la.la_device_status()[1] == 0
+    oc = o.cpu()
+    del o, qd, kd, vd
+    if rows_only:
+        rng = np.random.default_rng(0)
+        N = w.N
+        ts = sorted({0, 1, 127, 128, 129, N // 2, N - 129, N - 128, N - 1,
+                     *rng.integers(0, N, 40).tolist()})
+        sel = [(int(rng.integers(0, w.B)), int(rng.integers(0, w.Hq)), t) for t in ts]
+        ref = oracle.rows(q, k, v, sel)
+        got = torch.stack([oc[b, h, t] for b, h, t in sel])
+        assert_bf16_close(got, ref, f"{w.name} sampled rows")
+        ref_S = oracle.state_gemm(k, v)
+    else:
+        ref_o, ref_S = oracle.recurrent(q, k, v, o_dtype=np.float32)
+        assert_bf16_close(oc, ref_o, f"{w.name} chunk {chunk}")
+    assert_f32_close(S.cpu(), ref_S, f"{w.name} final state", tol=STATE_REL_L2)
+
+
+def test_full_mha_8k(la):
+    _full(la, synth.MHA_8K, 64)
+
+
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_full_gqa_32k(la, chunk):
+    _full(la, synth.GQA_32K, chunk)
+
+
+def test_full_long_1m(la):
+    _full(la, synth.LONG_1M, 128, rows_only=True)

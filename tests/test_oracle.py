@@ -94,6 +94,10 @@ def pin_state_is_ktv():
     want = np.einsum("bgsi,bgsj->bgij", _f64(k), _f64(v))
     assert _rel(oracle.state(k, v), want) < 1e-13
     assert _rel(oracle.recurrent(q, k, v, want_o=False)[1], want) < 1e-13
+    kb, vb = k.bfloat16(), v.bfloat16()
+    wantb = np.einsum("bgsi,bgsj->bgij", _f64(kb), _f64(vb))
+    assert _rel(oracle.state_gemm(kb, vb), wantb) < 1e-13
+    assert _rel(oracle.state(kb, vb), wantb) < 1e-13
 
 
 def pin_last_row_noncausal():
@@ -303,8 +307,8 @@ MUTANTS = [
      "for (int64_t j = 0; j < d; ++j) ot[j] += qi * S[j * d + i];"),
     ("bf16-widening-shift", "((uint32_t)((const uint16_t *)p)[i]) << 16;",
      "((uint32_t)((const uint16_t *)p)[i]) << 15;"),
-    ("decode-transposed", "for (int64_t j = 0; j < d; ++j) Sg[i * d + j] += ki * elem(v, kv + j, dtype);",
-     "for (int64_t j = 0; j < d; ++j) Sg[j * d + i] += ki * elem(v, kv + j, dtype);"),
+    ("decode-transposed", "for (int64_t j = 0; j < d; ++j) Sg[i * d + j] += ki * elem(J->v, kv + j, J->dtype);",
+     "for (int64_t j = 0; j < d; ++j) Sg[j * d + i] += ki * elem(J->v, kv + j, J->dtype);"),
     ("state-q-for-k", "const double ki = elem(J->k, kbase + s * d + i, J->dtype);",
      "const double ki = elem(J->v, kbase + s * d + i, J->dtype);"),
     ("recurrent-read-before-update",
