@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=None)
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override N (smaller case of the same workload, for profiling)")
     return ap.parse_args()
 
 
@@ -369,6 +371,9 @@ def run_ours(args, w):
 def main():
     args = parse()
     w = WORKLOADS[args.workload]
+    if args.seq_len:
+        import dataclasses
+        w = dataclasses.replace(w, N=args.seq_len, name=f"{w.name.split(' N')[0]} N{args.seq_len} d{w.d}")
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -83,9 +83,10 @@ int la_version(void);
  * mask -- the same sum in exact arithmetic, since the chunked form is exact for
  * every block length.
  *
- * Uses a workspace for the per-span states; la_forward / la_forward_state
- * keep one cached per device (grown on demand with cudaMalloc, freed by
- * la_shutdown), la_forward_ws takes one from the caller.
+ * Uses a workspace for the per-span states: la_forward / la_forward_state take
+ * it from the device's default stream-ordered memory pool (cudaMallocAsync and
+ * cudaFreeAsync on `stream`; the pool keeps the memory cached between calls),
+ * la_forward_ws takes one from the caller.
  *
  * Errors: LA_ERR_INVALID_ARG (null or misaligned pointer, B/Hq/Hkv/N <= 0,
  * Hq % Hkv, o overlapping an input), LA_ERR_UNSUPPORTED (d != 128, chunk not
@@ -183,8 +184,8 @@ la_status la_decode_step(float *S, const la_bf16 *q, const la_bf16 *k, const la_
 la_status la_device_status(unsigned int *flags, int clear);
 la_status la_selftest_wait(int64_t timeout_ns, la_stream stream);
 
-/* Frees the cached per-device workspace of la_forward / la_forward_state.
- * Call only when no call of this library is in flight. */
+/* Returns the memory the device's default pool keeps cached for the
+ * workspaces of la_forward / la_forward_state (cudaMemPoolTrimTo). */
 void la_shutdown(void);
 
 #ifdef __cplusplus
