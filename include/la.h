@@ -115,6 +115,29 @@ la_status la_forward_ws(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la
                         void *workspace, size_t workspace_bytes, la_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Prefill without any device allocation.  The pages have no counterpart to
+ * this entry point: it exists for callers that cannot allocate device memory
+ * at call time (code inside an allocator or memory-pool callback, frameworks
+ * that own every device byte, paths that must not block in the driver's
+ * allocator).  Same arguments, results and errors as la_forward_state, with
+ * the span-state workspace taken from one 32 MiB file-scope device array
+ * instead of an allocation; every GPU that loads this part of the library
+ * keeps that array until the process exits.
+ *   - Limit: B * Hkv * d * d * 4 bytes (one span per (batch, kv head)) must
+ *     fit in 32 MiB, i.e. B * Hkv <= 512 at d = 128; beyond that the call
+ *     returns LA_ERR_WORKSPACE.  Within it, the span count is lowered when
+ *     the usual plan would not fit.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the array: calls whose work overlaps on the GPU race
+ *     and must be serialised by the caller.  Each call writes every entry it
+ *     reads, so nothing from an earlier call needs clearing.
+ * ---------------------------------------------------------------------- */
+la_status la_forward_noalloc(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
+                             float *S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                             la_stream stream);
+
+/* ------------------------------------------------------------------------
  * The prefill's three stages, for callers that schedule or time them apart.
  * la_forward_ws == plan, then span_states, scan, main on one stream.
  *

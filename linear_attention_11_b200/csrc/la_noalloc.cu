@@ -1,0 +1,86 @@
+// la_noalloc.cu -- la_forward_noalloc: the bf16 prefill without any device
+// allocation, for callers that cannot call cudaMalloc or any allocator:
+// code running where allocation is forbidden or unsafe (inside a custom
+// allocator or memory-pool callback, a framework that owns all device memory
+// and rejects foreign allocations, or a hard-real-time path that must not
+// block on the driver's allocator).
+//
+// The span-state workspace that la_forward takes from the stream-ordered pool
+// lives instead in one file-scope device array of fixed size.  Every GPU that
+// loads this part of the library holds the array until the process exits.
+// Every call uses the same array, so calls whose work overlaps on the GPU
+// (other streams, other host threads) race on it and must be serialised by
+// the caller.  Each call writes every workspace entry before reading it, so
+// nothing left by an earlier call needs clearing.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "la.h"
+
+#define LA_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+// 32 MiB of span states: B * Hkv * nspan * d * d * 4 bytes must fit.
+constexpr size_t kScratchBytes = (size_t)32 << 20;
+static __device__ __align__(256) float g_noalloc_scratch[kScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the array's name as a device address).
+void* scratch_on_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+LA_EXPORT la_status la_forward_noalloc(const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                                       la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N,
+                                       int d, int chunk, la_stream stream) {
+  if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  la_plan plan;
+  la_status st = la_prefill_plan(B, Hq, Hkv, N, d, chunk, &plan);
+  if (st != LA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (S && !aligned16(S)))
+    return LA_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * N * d * 2, kbytes = (size_t)B * Hkv * N * d * 2,
+               sbytes = (size_t)B * Hkv * d * d * 4;
+  if (overlap(o, qbytes, q, qbytes) || overlap(o, qbytes, k, kbytes) ||
+      overlap(o, qbytes, v, kbytes) || overlap(o, qbytes, S, sbytes) ||
+      overlap(S, sbytes, q, qbytes) || overlap(S, sbytes, k, kbytes) ||
+      overlap(S, sbytes, v, kbytes))
+    return LA_ERR_INVALID_ARG;
+  // Fewer spans if the planned workspace exceeds the array; reject when even
+  // one span per (batch, kv head) does not fit.
+  const int64_t per_span = (int64_t)B * Hkv * d * d * (int64_t)sizeof(float);
+  if (per_span > (int64_t)kScratchBytes) return LA_ERR_WORKSPACE;
+  if (plan.workspace_bytes > (int64_t)kScratchBytes) {
+    plan.nspan = (int32_t)((int64_t)kScratchBytes / per_span);
+    plan.workspace_bytes = per_span * plan.nspan;
+  }
+  float* ws = static_cast<float*>(scratch_on_current_device());
+  if (!ws) return LA_ERR_CUDA;
+  if ((st = la_prefill_span_states(k, v, B, Hkv, N, d, &plan, ws, stream)) != LA_OK) return st;
+  if ((st = la_prefill_scan(ws, S, B, Hkv, d, &plan, stream)) != LA_OK) return st;
+  return la_prefill_main(q, k, v, o, ws, B, Hq, Hkv, N, d, &plan, stream);
+}
