@@ -123,6 +123,20 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def max_over_ranks(t: float, dist=None, device=None) -> float:
+    """The largest of every rank's value (a scalar all-reduce; no data path)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return t
+    tt = torch.tensor([t], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def throughput_mtok(world: int, B: int, N: int, steps: int, seconds: float) -> float:
+    """Whole-job Mtok/s: every rank processes its own B x N tokens per step."""
+    return world * B * N * steps / seconds / 1e6
+
+
 def timed(fn, steps, stream):
     """Device time of `steps` calls of fn on `stream`, with clock samples."""
     torch.cuda.synchronize()
@@ -139,18 +153,20 @@ def timed(fn, steps, stream):
     return start.elapsed_time(end) / 1e3, clk.summary()
 
 
-def traffic_from_profile(kernel_key: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    source is unchanged since the capture; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def traffic_from_profile():
+    """DRAM bytes per launch of the main kernel from the committed ncu summary,
+    if the kernel source is unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "prefill_main_traffic_gqa_b1_h128kv32.md")
     src = os.path.join(ROOT, "linear_attention_11_b200", "csrc", "la_prefill.cu")
     try:
-        with open(path) as f:
-            t = json.load(f)
+        fields = {}
+        for line in open(path):
+            if ":" in line:
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        e = t.get(kernel_key)
-        if e and e.get("source_sha256") == sha:
-            return e["dram_bytes_per_launch"]
+        if fields.get("kernel-source-sha256") == sha:
+            return int(fields["traffic-bytes-per-launch"])
     except (OSError, ValueError, KeyError):
         pass
     return None
@@ -255,11 +271,8 @@ def run_ours(args, w):
     barrier()
     t, clocks = timed(step, args.steps, stream)
     barrier()
-    if dist:
-        tt = torch.tensor([t], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
-    value = world * B * N * args.steps / t / 1e6
+    t = max_over_ranks(t, dist, dev)
+    value = throughput_mtok(world, B, N, args.steps, t)
 
     # --- per-kernel timing of the main chunk-loop pass (stages called apart)
     plan = la.api.la_prefill_plan(B, Hq, Hkv, N, d, chunk)
@@ -282,7 +295,7 @@ def run_ours(args, w):
     pk = peaks()
     achieved = alg_bytes / t_main / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": traffic_from_profile("prefill_main"),
+                "frac": achieved / pk["hbm_gbs"], "traffic": (traffic_from_profile() if (w is synth.GQA_32K and chunk == 64) else None),
                 "kernel": "prefill_main_kernel", "launch_ms": t_main * 1e3,
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": pk["source"]}
     step_frac = (alg_bytes / (t / args.steps) / 1e9) / pk["hbm_gbs"]
@@ -306,11 +319,8 @@ def run_ours(args, w):
         barrier()
         te, _ = timed(e2e_step, e2e_steps, stream)
         barrier()
-        if dist:
-            tt = torch.tensor([te], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            te = float(tt.item())
-        e2e = {"value": world * B * N * e2e_steps / te / 1e6, "unit": "Mtok/s",
+        te = max_over_ranks(te, dist, dev)
+        e2e = {"value": throughput_mtok(world, B, N, e2e_steps, te), "unit": "Mtok/s",
                "h2d_bytes_per_step": elt * (q.numel() + k.numel() + v.numel()),
                "d2h_bytes_per_step": elt * q.numel(), "steps": e2e_steps}
         del qh, kh, vh, oh, qe, ke, ve
