@@ -115,6 +115,28 @@ la_status la_forward_ws(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la
                         void *workspace, size_t workspace_bytes, la_stream stream);
 
 /* ------------------------------------------------------------------------
+ * The prefill as one persistent kernel (an alternative schedule of the same
+ * arithmetic; la_forward runs the three-kernel scheme below).  Every (batch, kv head) sequence is cut into `nspan`
+ * spans; span-state items (K^T V of a span, then the chained prefix: the state
+ * entering the next span) and chunk-loop items (the chunk loop of one span for
+ * a group of query heads, from its entering state) are taken in rounds, one
+ * round per span index, so the chunk loops of a span re-read its K and V from
+ * L2 right after the span-state item has read them from HBM.  The entering
+ * states are published through GPU-scope flags; every wait is bounded.
+ *   nspan <= 0 picks the span count for the problem and device; otherwise
+ *   1 <= nspan <= ceil(N / tile) (tile = la_plan.tile).
+ *   workspace: device memory, 256-byte aligned, at least
+ *   la_prefill_fused_workspace_bytes(..., nspan) bytes (entering states and
+ *   flags); the call clears the flags on `stream` first (cudaMemsetAsync).
+ * Errors as la_forward_ws.
+ * ---------------------------------------------------------------------- */
+size_t la_prefill_fused_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                                        int nspan);
+la_status la_prefill_fused(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
+                           float *S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                           int nspan, void *workspace, size_t workspace_bytes, la_stream stream);
+
+/* ------------------------------------------------------------------------
  * Prefill without any device allocation.  The pages have no counterpart to
  * this entry point: it exists for callers that cannot allocate device memory
  * at call time (code inside an allocator or memory-pool callback, frameworks
@@ -138,8 +160,9 @@ la_status la_forward_noalloc(const la_bf16 *q, const la_bf16 *k, const la_bf16 *
                              la_stream stream);
 
 /* ------------------------------------------------------------------------
- * The prefill's three stages, for callers that schedule or time them apart.
- * la_forward_ws == plan, then span_states, scan, main on one stream.
+ * The prefill's three stages -- the scheme la_forward, la_forward_state,
+ * la_forward_ws and la_forward_noalloc run -- for callers that schedule or time
+ * them apart: plan, then span_states, scan, main on one stream.
  *
  * The sequence of every (batch, kv head) is cut into `nspan` spans of whole
  * chunks.  span_states writes each span's K^T V into the workspace; scan turns

@@ -23,7 +23,8 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_E
 
 # Every symbol include/la.h declares.
 EXPORTS = ("la_status_string", "la_version", "la_forward", "la_forward_state",
-           "la_forward_workspace_bytes", "la_forward_ws", "la_forward_noalloc", "la_prefill_plan",
+           "la_forward_workspace_bytes", "la_forward_ws", "la_forward_noalloc",
+           "la_prefill_fused_workspace_bytes", "la_prefill_fused", "la_prefill_plan",
            "la_prefill_span_states", "la_prefill_scan", "la_prefill_main", "la_forward_f32",
            "la_decode_step", "la_device_status", "la_selftest_wait", "la_shutdown")
 
@@ -55,6 +56,8 @@ def _declare(lib):
         "la_forward_workspace_bytes": ([I, I, I, L, I, I], S),
         "la_forward_ws": ([P, P, P, P, P, I, I, I, L, I, I, P, S, P], I),
         "la_forward_noalloc": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
+        "la_prefill_fused_workspace_bytes": ([I, I, I, L, I, I, I], S),
+        "la_prefill_fused": ([P, P, P, P, P, I, I, I, L, I, I, I, P, S, P], I),
         "la_prefill_plan": ([I, I, I, L, I, I, PP], I),
         "la_prefill_span_states": ([P, P, I, I, L, I, PP, P, P], I),
         "la_prefill_scan": ([P, P, I, I, I, PP, P], I),
@@ -151,6 +154,20 @@ def la_forward_noalloc(q, k, v, S=None, o=None, chunk: int = 64, stream=None):
     B, Hq, Hkv, N, d = _dims(q, k)
     _check("la_forward_noalloc", load_library().la_forward_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, _stream(stream)))
+    return o
+
+
+def la_prefill_fused_workspace_bytes(B, Hq, Hkv, N, d, chunk, nspan=0) -> int:
+    return int(load_library().la_prefill_fused_workspace_bytes(B, Hq, Hkv, N, d, chunk, nspan))
+
+
+def la_prefill_fused(q, k, v, o, S, workspace, chunk: int = 64, nspan: int = 0, stream=None):
+    """The single-pass prefill with an explicit span count (0 = automatic)."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("la_prefill_fused", load_library().la_prefill_fused(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, nspan,
+        _ptr(workspace), nbytes, _stream(stream)))
     return o
 
 

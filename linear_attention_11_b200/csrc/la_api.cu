@@ -105,6 +105,23 @@ la_status plan_impl(int B, int Hq, int Hkv, int64_t N, int d, int chunk, int sms
   return LA_OK;
 }
 
+// Span count of the fused single-pass kernel.  Each round (one span index
+// over every kv head) re-reads its K and V from L2, so a round's K+V should
+// stay well inside the 126 MB L2 next to the streaming Q and O: about 24 MB.
+// Enough chunk-loop items for the dynamic scheduler to balance (two per SM),
+// and at least four tiles per item so per-item costs stay small.
+int fused_nspan(int B, int Hkv, int G, int HPT, int64_t N, int T, int sms) {
+  const int64_t tiles = (N + T - 1) / T;
+  const double kv_bytes = 2.0 * 2.0 * (double)B * Hkv * (double)N * kHeadDim;
+  const double round_budget = 24.0 * 1024 * 1024;
+  int64_t ns = (int64_t)(kv_bytes / round_budget) + 1;
+  const int64_t units_m = (int64_t)B * Hkv * (G / HPT);
+  ns = std::max<int64_t>(ns, (2 * sms + units_m - 1) / units_m);
+  ns = std::min<int64_t>(ns, std::max<int64_t>(1, tiles / 4));
+  ns = std::min<int64_t>(ns, tiles);
+  return (int)std::max<int64_t>(1, ns);
+}
+
 // A caller-supplied plan must describe this problem.
 la_status check_plan(const la_plan* p, int B, int Hq, int Hkv, int64_t N, int d) {
   if (!p) return LA_ERR_INVALID_ARG;
@@ -295,6 +312,50 @@ LA_EXPORT la_status la_prefill_main(const la_bf16* q, const la_bf16* k, const la
   return from_cuda(launch_prefill_main(g, maps, ws, status, static_cast<cudaStream_t>(stream)));
 }
 
+LA_EXPORT size_t la_prefill_fused_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d,
+                                                 int chunk, int nspan) {
+  la_plan plan;
+  if (la_prefill_plan(B, Hq, Hkv, N, d, chunk, &plan) != LA_OK) return 0;
+  int sms = 0;
+  if (!device_info(nullptr, &sms)) return 0;
+  if (nspan <= 0)
+    nspan = fused_nspan(B, Hkv, Hq / Hkv, plan.heads_per_tile, N, plan.tile, sms);
+  if (nspan > plan.tiles_total) return 0;
+  return fused_workspace_bytes(B, Hkv, nspan);
+}
+
+LA_EXPORT la_status la_prefill_fused(const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                                     la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N,
+                                     int d, int chunk, int nspan, void* workspace,
+                                     size_t workspace_bytes, la_stream stream) {
+  if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  la_plan plan;
+  la_status st = la_prefill_plan(B, Hq, Hkv, N, d, chunk, &plan);
+  if (st != LA_OK) return st;
+  if ((st = check_prefill_ptrs(q, k, v, o, S, B, Hq, Hkv, N, d)) != LA_OK) return st;
+  unsigned* status = nullptr;
+  int sms = 0;
+  if (!device_info(&status, &sms)) return LA_ERR_CUDA;
+  if (nspan <= 0) nspan = fused_nspan(B, Hkv, Hq / Hkv, plan.heads_per_tile, N, plan.tile, sms);
+  if (nspan > plan.tiles_total) return LA_ERR_INVALID_ARG;
+  if ((int64_t)nspan * ((int64_t)B * Hkv + (int64_t)B * Hkv * (Hq / Hkv / plan.heads_per_tile)) >
+      0x7fffffff)
+    return LA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < fused_workspace_bytes(B, Hkv, nspan))
+    return LA_ERR_WORKSPACE;
+  plan.nspan = nspan;
+  PrefillMaps maps;
+  if (!make_tmap_bf16(&maps.q, q, N, (int64_t)B * Hq, plan.tile) ||
+      !make_tmap_bf16(&maps.o, o, N, (int64_t)B * Hq, plan.tile) ||
+      !make_tmap_bf16(&maps.k, k, N, (int64_t)B * Hkv, plan.tile) ||
+      !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
+    return LA_ERR_CUDA;
+  PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
+  return from_cuda(launch_prefill_fused(g, maps, S, workspace, status, sms,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 LA_EXPORT la_status la_forward_ws(const la_bf16* q, const la_bf16* k, const la_bf16* v,
                                   la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N, int d,
                                   int chunk, void* workspace, size_t workspace_bytes,
@@ -336,10 +397,11 @@ LA_EXPORT la_status la_forward_state(const la_bf16* q, const la_bf16* k, const l
       }
     });
   }
+  const size_t bytes = la_forward_workspace_bytes(B, Hq, Hkv, N, d, chunk);
+  if (bytes == 0) return LA_ERR_CUDA;
   void* ws = nullptr;
-  if (cudaMallocAsync(&ws, (size_t)plan.workspace_bytes, s) != cudaSuccess) return LA_ERR_CUDA;
-  st = la_forward_ws(q, k, v, o, S, B, Hq, Hkv, N, d, chunk, ws, (size_t)plan.workspace_bytes,
-                     stream);
+  if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return LA_ERR_CUDA;
+  st = la_forward_ws(q, k, v, o, S, B, Hq, Hkv, N, d, chunk, ws, bytes, stream);
   if (cudaFreeAsync(ws, s) != cudaSuccess && st == LA_OK) st = LA_ERR_CUDA;
   return st;
 }

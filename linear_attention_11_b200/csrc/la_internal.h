@@ -35,6 +35,10 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                cudaStream_t stream);
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
                                 const float* ws, unsigned* status, cudaStream_t stream);
+size_t fused_workspace_bytes(int B, int Hkv, int nspan);
+cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
+                                 void* workspace, unsigned* status, int num_sms,
+                                 cudaStream_t stream);
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
                               cudaStream_t stream);
 cudaError_t launch_decode(float* S, const void* q, const void* k, const void* v, void* o, int B,

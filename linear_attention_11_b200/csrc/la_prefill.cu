@@ -28,9 +28,11 @@
 // swizzle; rows beyond N read as zero and stores beyond N are clipped, which
 // handles the short last chunk.
 //
-// Warp roles (192 threads): warp 0 issues the copies, warp 1 owns the tensor
-// memory and issues the MMAs, warps 2-5 (128 threads, one per TMEM lane) do
-// the mask, the state conversion and the output epilogue.
+// Warp roles of the main kernel (320 threads): warp 0 issues the copies, warp 1
+// owns the tensor memory and issues the MMAs, warps 2-5 (one thread per TMEM
+// lane) mask the score tiles, warps 6-9 write the output tiles; both
+// warpgroups convert half of the state.  The span-state kernel uses 192
+// threads (one epilogue warpgroup).
 //
 // Tensor memory (512 columns, fp32 unless noted):
 //   [  0,128)  O buffer 0     (the score tile A of even tiles lives here first)
@@ -42,32 +44,10 @@
 
 #include "la_internal.h"
 #include "la_ptx.cuh"
+#include "la_tile.cuh"
 
 namespace la {
 namespace {
-
-constexpr int kQBytes = kTileRows * kHeadDim * 2;  // 32 KB: 128 rows x 128 bf16
-constexpr int kHalf = kTileRows * 128;             // one 64-column block of a 128-row tile
-constexpr int kSBytes = kHeadDim * kHeadDim * 2;   // bf16 copy of the state
-constexpr uint32_t kColS = 384;
-
-// Store 32 fp32 values (bits) of row r, columns [32*blk, 32*blk+32), as bf16
-// into a 128-row tile laid out as two 64-column blocks of 128-byte swizzled
-// rows (the layout the bulk tensor copies and the MMA descriptors both use).
-__device__ __forceinline__ void store_row32_sw128(uint32_t base, int r, int blk,
-                                                  const uint32_t (&v)[32]) {
-  const uint32_t row = base + (uint32_t)((blk >> 1) * kHalf + r * 128);
-  const int c0 = (blk & 1) * 4;
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const uint32_t chunk = (uint32_t)((c0 + m) ^ (r & 7));
-    st_shared_v4(row + chunk * 16,
-                 pack_bf16x2(__uint_as_float(v[8 * m + 0]), __uint_as_float(v[8 * m + 1])),
-                 pack_bf16x2(__uint_as_float(v[8 * m + 2]), __uint_as_float(v[8 * m + 3])),
-                 pack_bf16x2(__uint_as_float(v[8 * m + 4]), __uint_as_float(v[8 * m + 5])),
-                 pack_bf16x2(__uint_as_float(v[8 * m + 6]), __uint_as_float(v[8 * m + 7])));
-  }
-}
 
 struct MainParams {
   const float* ws;
@@ -75,54 +55,70 @@ struct MainParams {
   int Hq, Hkv, G, nsub, nspan, tiles_total;
 };
 
-template <int T, int STAGES>
+// Shared memory of the main kernel: a ring of Q tiles, a separate ring of K/V
+// tiles, the bf16 state copy, and (at T = 64) a dedicated output staging tile.
+// Q(i) is released once Q(i) S has been issued and completed; K/V(i) once the
+// state update of tile i has; so copies of later tiles start early and more
+// bytes stay in flight.  At T = 128 there is no room for a separate staging
+// tile and the output goes through the Q slot (released after its store has
+// read it).
+template <int T, int QST, int KVST>
 struct MainLayout {
+  static constexpr bool kDedicatedO = (T == 64);
   static constexpr int kKBytes = T * kHeadDim * 2;
-  static constexpr int kStageBytes = kQBytes + 2 * kKBytes;
-  static constexpr int kSOff = STAGES * kStageBytes;
-  static constexpr int kBarOff = kSOff + kSBytes;
-  static constexpr int kNumBars = 2 * STAGES + 9;
+  static constexpr int kKVBytes = 2 * kKBytes;
+  static constexpr int kKVOff = QST * kQBytes;
+  static constexpr int kSOff = kKVOff + KVST * kKVBytes;
+  static constexpr int kOOff = kSOff + kSBytes;
+  static constexpr int kBarOff = kOOff + (kDedicatedO ? kQBytes : 0);
+  // q_full[QST], q_empty[QST], kv_full[KVST], kv_empty[KVST], a_full, p_full,
+  // o_full[2], o_empty[2], s_full, sb_full, mma_done, store_ready, ostage_free
+  static constexpr int kNumBars = 2 * QST + 2 * KVST + 11;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
 };
 
-template <int T, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+template <int T, int QST, int KVST>
+__global__ void __launch_bounds__(320, 1)
     prefill_main_kernel(const __grid_constant__ CUtensorMap map_q,
                         const __grid_constant__ CUtensorMap map_k,
                         const __grid_constant__ CUtensorMap map_v,
                         const __grid_constant__ CUtensorMap map_o, const MainParams p) {
-  using L = MainLayout<T, STAGES>;
+  using L = MainLayout<T, QST, KVST>;
   constexpr int HPT = kTileRows / T;
-  constexpr uint32_t kStageTx = L::kStageBytes;
+  constexpr bool kDedicatedO = L::kDedicatedO;
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, T, 0, 0);
   constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, 0, 1);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
   constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, 1, 1);
+  constexpr bool kLookahead = KVST >= 3;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sm = smem_raw + (base - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBarOff);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* a_full = bars + 2 * STAGES + 0;
-  uint64_t* p_full = bars + 2 * STAGES + 1;
-  uint64_t* o_full = bars + 2 * STAGES + 2;
-  uint64_t* o_empty = bars + 2 * STAGES + 3;  // two barriers
-  uint64_t* s_full = bars + 2 * STAGES + 5;
-  uint64_t* sb_full = bars + 2 * STAGES + 6;
-  uint64_t* mma_done = bars + 2 * STAGES + 7;
-  uint64_t* store_ready = bars + 2 * STAGES + 8;
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = q_full + QST;
+  uint64_t* kv_full = q_empty + QST;
+  uint64_t* kv_empty = kv_full + KVST;
+  uint64_t* a_full = kv_empty + KVST;
+  uint64_t* p_full = a_full + 1;
+  uint64_t* o_full = p_full + 1;    // two: tile i completes o_full[i & 1]
+  uint64_t* o_empty = o_full + 2;   // two
+  uint64_t* s_full = o_empty + 2;
+  uint64_t* sb_full = s_full + 1;
+  uint64_t* mma_done = sb_full + 1;
+  uint64_t* store_ready = mma_done + 1;
+  uint64_t* ostage_free = store_ready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
 
-  const uint32_t sQ0 = base;
   const uint32_t sS = base + L::kSOff;
-  auto sQ = [&](int s) { return sQ0 + (uint32_t)(s * L::kStageBytes); };
-  auto sK = [&](int s) { return sQ(s) + (uint32_t)kQBytes; };
-  auto sV = [&](int s) { return sQ(s) + (uint32_t)(kQBytes + L::kKBytes); };
+  auto sQ = [&](int i) { return base + (uint32_t)((i % QST) * kQBytes); };
+  auto sK = [&](int i) { return base + (uint32_t)(L::kKVOff + (i % KVST) * L::kKVBytes); };
+  auto sV = [&](int i) { return sK(i) + (uint32_t)L::kKBytes; };
+  auto sO = [&](int i) { return kDedicatedO ? base + (uint32_t)L::kOOff : sQ(i); };
 
   // ---- work item
   int idx = blockIdx.x;
@@ -140,19 +136,25 @@ __global__ void __launch_bounds__(192, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 2);  // MMA commit + output-store release
+    for (int i = 0; i < QST; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], kDedicatedO ? 1 : 2);  // MMA commit (+ output-store release)
+    }
+    for (int i = 0; i < KVST; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
     mbar_init(a_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
-    mbar_init(&o_empty[0], 128);
+    mbar_init(p_full, 128);       // mask warpgroup
+    mbar_init(&o_full[0], 1);
+    mbar_init(&o_full[1], 1);
+    mbar_init(&o_empty[0], 128);  // epilogue warpgroup
     mbar_init(&o_empty[1], 128);
     mbar_init(s_full, 1);
-    mbar_init(sb_full, 128);
+    mbar_init(sb_full, 256);      // both warpgroups convert half of the state
     mbar_init(mma_done, 1);
     mbar_init(store_ready, 128);
+    mbar_init(ostage_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -166,110 +168,146 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (elect_one()) {
+    // ------------------------------------------------------------ copies
+    // Lane 0 streams the Q tiles, lane 1 the K/V tiles, each through its own
+    // ring, so a K/V copy never waits behind a Q slot (and vice versa).
+    if (lane == 0) {
       prefetch_tmap(&map_q);
-      prefetch_tmap(&map_k);
-      prefetch_tmap(&map_v);
       prefetch_tmap(&map_o);
       const uint64_t pol_q = policy_evict_first();
-      const uint64_t pol_kv = policy_evict_last();  // re-read by the other head subsets
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % STAGES;
-        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, p.status, abort_flag))
-          break;
-        mbar_arrive_expect_tx(&full[s], kStageTx);
+        const int s = i % QST;
+        if (i >= QST && !mbar_wait(&q_empty[s], ((i / QST) - 1) & 1, p.status, abort_flag)) break;
+        mbar_arrive_expect_tx(&q_full[s], kQBytes);
         const int c1 = (tile_begin + i) * T;
-        uint8_t* q_dst = sm + (sQ(s) - base);
+        uint8_t* q_dst = sm + (sQ(i) - base);
 #pragma unroll
         for (int hh = 0; hh < HPT; ++hh) {
-          tma_load_3d(q_dst + hh * T * 128, &map_q, &full[s], 0, c1, b * p.Hq + head0 + hh, pol_q);
-          tma_load_3d(q_dst + kHalf + hh * T * 128, &map_q, &full[s], 64, c1,
+          tma_load_3d(q_dst + hh * T * 128, &map_q, &q_full[s], 0, c1, b * p.Hq + head0 + hh,
+                      pol_q);
+          tma_load_3d(q_dst + kHalf + hh * T * 128, &map_q, &q_full[s], 64, c1,
                       b * p.Hq + head0 + hh, pol_q);
         }
-        uint8_t* k_dst = sm + (sK(s) - base);
-        uint8_t* v_dst = sm + (sV(s) - base);
-        tma_load_3d(k_dst, &map_k, &full[s], 0, c1, bg, pol_kv);
-        tma_load_3d(k_dst + T * 128, &map_k, &full[s], 64, c1, bg, pol_kv);
-        tma_load_3d(v_dst, &map_v, &full[s], 0, c1, bg, pol_kv);
-        tma_load_3d(v_dst + T * 128, &map_v, &full[s], 64, c1, bg, pol_kv);
         issued = i + 1;
       }
       if (*abort_flag) {  // let copies already issued land before the block exits
-        for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-          mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1);
+        for (int i = (issued > QST ? issued - QST : 0); i < issued; ++i)
+          mbar_wait_drain(&q_full[i % QST], (i / QST) & 1);
+      }
+    } else if (lane == 1) {
+      prefetch_tmap(&map_k);
+      prefetch_tmap(&map_v);
+      const uint64_t pol_kv = policy_evict_last();  // re-read by the other head subsets
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % KVST;
+        if (i >= KVST && !mbar_wait(&kv_empty[s], ((i / KVST) - 1) & 1, p.status, abort_flag))
+          break;
+        mbar_arrive_expect_tx(&kv_full[s], L::kKVBytes);
+        const int c1 = (tile_begin + i) * T;
+        uint8_t* k_dst = sm + (sK(i) - base);
+        uint8_t* v_dst = sm + (sV(i) - base);
+        tma_load_3d(k_dst, &map_k, &kv_full[s], 0, c1, bg, pol_kv);
+        tma_load_3d(k_dst + T * 128, &map_k, &kv_full[s], 64, c1, bg, pol_kv);
+        tma_load_3d(v_dst, &map_v, &kv_full[s], 0, c1, bg, pol_kv);
+        tma_load_3d(v_dst + T * 128, &map_v, &kv_full[s], 64, c1, bg, pol_kv);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        for (int i = (issued > KVST ? issued - KVST : 0); i < issued; ++i)
+          mbar_wait_drain(&kv_full[i % KVST], (i / KVST) & 1);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Order per tile i:  QS(i) PV(i) | QK(i+1) | KV(i) with a 3-deep K/V ring:
+    // the next tile's scores go before this tile's state update, so its causal
+    // mask overlaps the update.  With 2 K/V slots the next tile's copy is
+    // usually still in flight, so the update goes first: QS(i) PV(i) KV(i) |
+    // QK(i+1).
     if (elect_one()) {
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % STAGES;
+      auto issue_qk = [&](int i) -> bool {
         const uint32_t ob = (uint32_t)(i & 1);
-        const uint32_t ocol = ob * 128;
-        const uint32_t pcol = 256 + ob * (T / 2);
-        if (!mbar_wait(&full[s], (i / STAGES) & 1, p.status, abort_flag)) break;
-        if (i >= 2 && !mbar_wait(&o_empty[ob], ((i >> 1) - 1) & 1, p.status, abort_flag)) break;
+        if (!mbar_wait(&q_full[i % QST], (i / QST) & 1, p.status, abort_flag)) return false;
+        if (!mbar_wait(&kv_full[i % KVST], (i / KVST) & 1, p.status, abort_flag)) return false;
+        if (i >= 2 && !mbar_wait(&o_empty[ob], ((i >> 1) - 1) & 1, p.status, abort_flag))
+          return false;
         tc_fence_after();
-        const uint32_t q_addr = sQ(s), k_addr = sK(s), v_addr = sV(s);
-        // A = Q K^T  (both K-major; 16-element k-steps inside 128-byte rows)
+        const uint32_t q_addr = sQ(i), k_addr = sK(i);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 8; ++kk) {  // A = Q K^T, both K-major
           const uint32_t koff = (uint32_t)((kk & 3) * 32);
           const uint64_t da = smem_desc_sw128(q_addr + (kk >> 2) * kHalf + koff, 16, 1024);
           const uint64_t db = smem_desc_sw128(k_addr + (kk >> 2) * (T * 128) + koff, 16, 1024);
-          mma_ss(tmem + ocol, da, db, IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + ob * 128, da, db, IDESC_QK, kk > 0 ? 1u : 0u);
         }
         mma_commit(a_full);
+        return true;
+      };
+      bool ok = ntiles > 0 && issue_qk(0);
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const uint32_t ob = (uint32_t)(i & 1);
+        const uint32_t ocol = ob * 128;
+        const uint32_t pcol = 256 + ob * (T / 2);
         if (!mbar_wait(p_full, i & 1, p.status, abort_flag)) break;
         if (!mbar_wait(sb_full, i & 1, p.status, abort_flag)) break;
         tc_fence_after();
-        // O = Q S   (S: MN-major, 16 key rows of 128 B per k-step)
+        const uint32_t q_addr = sQ(i), k_addr = sK(i), v_addr = sV(i);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 8; ++kk) {  // O = Q S (S: MN-major, 16 key rows per k-step)
           const uint64_t da =
               smem_desc_sw128(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t db = smem_desc_sw128(sS + kk * 2048, kHalf, 1024);
           mma_ss(tmem + ocol, da, db, IDESC_QS, kk > 0 ? 1u : 0u);
         }
-        // O += P V  (P from TMEM, 8 columns = 16 bf16 per k-step; V MN-major)
 #pragma unroll
-        for (int kk = 0; kk < T / 16; ++kk) {
+        for (int kk = 0; kk < T / 16; ++kk) {  // O += P V (P from TMEM)
           const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
           mma_ts(tmem + ocol, tmem + pcol + kk * 8, db, IDESC_PV, 1u);
         }
-        mma_commit(o_full);
-        // S += K^T V  (K as MN-major A, V as MN-major B)
+        mma_commit(&o_full[ob]);
+        mma_commit(&q_empty[i % QST]);  // Q(i) read by QK(i) and QS(i), both done then
+        if (i + 1 < ntiles) {
+          if (kLookahead && !issue_qk(i + 1)) break;
 #pragma unroll
-        for (int kk = 0; kk < T / 16; ++kk) {
-          const uint64_t da = smem_desc_sw128(k_addr + kk * 2048, T * 128, 1024);
-          const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
-          mma_ss(tmem + kColS, da, db, IDESC_KV, 1u);
+          for (int kk = 0; kk < T / 16; ++kk) {  // S += K^T V (both MN-major)
+            const uint64_t da = smem_desc_sw128(k_addr + kk * 2048, T * 128, 1024);
+            const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
+            mma_ss(tmem + kColS, da, db, IDESC_KV, 1u);
+          }
+          mma_commit(s_full);
+          mma_commit(&kv_empty[i % KVST]);
+          if (!kLookahead && !issue_qk(i + 1)) break;
+        } else {
+          mma_commit(&kv_empty[i % KVST]);
         }
-        mma_commit(s_full);
-        mma_commit(&empty[s]);
       }
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ math warps
+    // ------------------------------------------------------------ math warpgroups
+    // WG1 (warps 2-5): causal mask; WG2 (warps 6-9): output epilogue and stores.
+    // Both convert half of the state (WG1 columns 0-63, WG2 columns 64-127).
+    const bool wg1 = warp < 6;
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // TMEM lane = tile row
+    const int r = quarter * 32 + lane;  // TMEM lane = tile row = state row
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int t_in = r % T;
-    const int mt = threadIdx.x - 64;
+    const int blk0 = wg1 ? 0 : 2;  // state column blocks this warpgroup converts
+    const bool store_thread = (warp == 6 && lane == 0);
     bool ok = true;
 
-    // Entering state of this span: fp32 rows -> TMEM S, bf16 copy -> smem.
+    // Entering state of this span (this warpgroup's half of the row).
     {
       const float4* src = reinterpret_cast<const float4*>(
           p.ws + ((size_t)bg * p.nspan + j) * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim);
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
+      for (int bb = 0; bb < 2; ++bb) {
+        const int blk = blk0 + bb;
         uint32_t v[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -288,87 +326,108 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(sb_full);
     }
 
-    for (int i = 0; i < ntiles && ok; ++i) {
-      const int s = i % STAGES;
-      const uint32_t ob = (uint32_t)(i & 1);
-      const uint32_t ocol = ob * 128;
-      const uint32_t pcol = 256 + ob * (T / 2);
-
-      // ---- causal mask of the score tile -> P (bf16 in TMEM)
-      if (!warp_wait(a_full, i & 1, p.status, abort_flag)) { ok = false; break; }
+    // half of the bf16 state copy for the next tile's Q S
+    auto convert_state = [&](int i) -> bool {
+      if (!warp_wait(s_full, i & 1, p.status, abort_flag)) return false;
       tc_fence_after();
-#pragma unroll
-      for (int blk = 0; blk < T / 32; ++blk) {
-        uint32_t a[32];
-        tmem_ld32(tmem + lane_base + ocol + blk * 32, a);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const int s0 = blk * 32 + 2 * m;
-          const float f0 = (s0 <= t_in) ? __uint_as_float(a[2 * m]) : 0.0f;
-          const float f1 = (s0 + 1 <= t_in) ? __uint_as_float(a[2 * m + 1]) : 0.0f;
-          pk[m] = pack_bf16x2(f0, f1);
-        }
-        tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
-
-      // ---- the previous tile's output store has read its smem: free that stage
-      if (mt == 0 && i > 0) {
-        bulk_wait_group_read<0>();
-        mbar_arrive(&empty[(i - 1) % STAGES]);
-      }
-
-      // ---- bf16 copy of the updated state for the next tile's Q S
-      if (i + 1 < ntiles) {
-        if (!warp_wait(s_full, i & 1, p.status, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + kColS + blk * 32, v);
-          tmem_wait_ld();
-          store_row32_sw128(sS, r, blk, v);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(sb_full);
-      }
-
-      // ---- output epilogue: TMEM -> bf16 -> this stage's Q buffer -> store
-      if (!warp_wait(o_full, i & 1, p.status, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t stage_q = sQ(s);
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + ocol + blk * 32, v);
-        tmem_wait_ld();
-        store_row32_sw128(stage_q, r, blk, v);
-      }
-      tc_fence_before();
-      mbar_arrive(&o_empty[ob]);
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
+      tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
+      tmem_wait_ld();
+      store_row32_sw128(sS, r, blk0, v0);
+      store_row32_sw128(sS, r, blk0 + 1, v1);
       fence_proxy_async_smem();
-      mbar_arrive(store_ready);
-      if (warp == 2) {
-        // every math thread has written its row of the staging tile
-        if (!warp_wait(store_ready, i & 1, p.status, abort_flag)) { ok = false; break; }
-      }
-      if (mt == 0) {
-        const int c1 = (tile_begin + i) * T;
-        const uint8_t* src = sm + (stage_q - base);
+      tc_fence_before();
+      mbar_arrive(sb_full);
+      return true;
+    };
+
+    if (wg1) {
+      auto mask_tile = [&](int i) -> bool {
+        const uint32_t ob = (uint32_t)(i & 1);
+        const uint32_t ocol = ob * 128;
+        const uint32_t pcol = 256 + ob * (T / 2);
+        if (!warp_wait(a_full, i & 1, p.status, abort_flag)) return false;
+        tc_fence_after();
+        uint32_t a[T / 32][32];
 #pragma unroll
-        for (int hh = 0; hh < HPT; ++hh) {
-          tma_store_3d(&map_o, src + hh * T * 128, 0, c1, b * p.Hq + head0 + hh);
-          tma_store_3d(&map_o, src + kHalf + hh * T * 128, 64, c1, b * p.Hq + head0 + hh);
+        for (int blk = 0; blk < T / 32; ++blk) tmem_ld32(tmem + lane_base + ocol + blk * 32, a[blk]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int blk = 0; blk < T / 32; ++blk) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const int s0 = blk * 32 + 2 * m;
+            const float f0 = (s0 <= t_in) ? __uint_as_float(a[blk][2 * m]) : 0.0f;
+            const float f1 = (s0 + 1 <= t_in) ? __uint_as_float(a[blk][2 * m + 1]) : 0.0f;
+            pk[m] = pack_bf16x2(f0, f1);
+          }
+          tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
         }
-        bulk_commit_group();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        return true;
+      };
+      ok = ntiles > 0 && mask_tile(0);
+      for (int i = 0; i < ntiles && ok; ++i) {
+        if (i + 1 < ntiles) {
+          // the MMA order decides which of the two is ready first
+          if (kLookahead) {
+            if (!mask_tile(i + 1) || !convert_state(i)) { ok = false; break; }
+          } else {
+            if (!convert_state(i) || !mask_tile(i + 1)) { ok = false; break; }
+          }
+        }
       }
+    } else {
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const uint32_t ob = (uint32_t)(i & 1);
+        const uint32_t ocol = ob * 128;
+        if (i + 1 < ntiles && !convert_state(i)) { ok = false; break; }
+        // output epilogue: TMEM -> bf16 -> staging tile -> bulk store
+        if (!warp_wait(&o_full[ob], (i >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+        if (kDedicatedO && i > 0 && !warp_wait(ostage_free, (i - 1) & 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t stage_o = sO(i);
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_base + ocol + (2 * bb) * 32, v0);
+          tmem_ld32(tmem + lane_base + ocol + (2 * bb + 1) * 32, v1);
+          tmem_wait_ld();
+          store_row32_sw128(stage_o, r, 2 * bb, v0);
+          store_row32_sw128(stage_o, r, 2 * bb + 1, v1);
+        }
+        tc_fence_before();
+        mbar_arrive(&o_empty[ob]);
+        fence_proxy_async_smem();
+        mbar_arrive(store_ready);
+        if (warp == 6) {
+          if (!warp_wait(store_ready, i & 1, p.status, abort_flag)) { ok = false; break; }
+        }
+        if (store_thread) {
+          const int c1 = (tile_begin + i) * T;
+          const uint8_t* src = sm + (stage_o - base);
+#pragma unroll
+          for (int hh = 0; hh < HPT; ++hh) {
+            tma_store_3d(&map_o, src + hh * T * 128, 0, c1, b * p.Hq + head0 + hh);
+            tma_store_3d(&map_o, src + kHalf + hh * T * 128, 64, c1, b * p.Hq + head0 + hh);
+          }
+          bulk_commit_group();
+          bulk_wait_group_read<0>();  // the store has read the staging tile
+          if (kDedicatedO)
+            mbar_arrive(ostage_free);
+          else
+            mbar_arrive(&q_empty[i % QST]);
+        }
+      }
+      if (store_thread) bulk_wait_group<0>();
     }
-    if (mt == 0) bulk_wait_group<0>();
   }
 
   tc_fence_before();
@@ -550,14 +609,17 @@ cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& map
   const dim3 grid((unsigned)(g.B * g.Hkv * g.nspan * nsub));
   cudaError_t e;
   if (g.tile == 64) {
-    using L = MainLayout<64, 3>;
-    if ((e = set_smem(prefill_main_kernel<64, 3>, L::kBytes)) != cudaSuccess) return e;
-    prefill_main_kernel<64, 3><<<grid, 192, L::kBytes, stream>>>(maps.q, maps.k, maps.v, maps.o, p);
+    using L = MainLayout<64, 2, 3>;
+    static_assert(L::kBytes <= 232448, "shared memory");
+    if ((e = set_smem(prefill_main_kernel<64, 2, 3>, L::kBytes)) != cudaSuccess) return e;
+    prefill_main_kernel<64, 2, 3><<<grid, 320, L::kBytes, stream>>>(maps.q, maps.k, maps.v, maps.o,
+                                                                    p);
   } else {
-    using L = MainLayout<128, 2>;
-    if ((e = set_smem(prefill_main_kernel<128, 2>, L::kBytes)) != cudaSuccess) return e;
-    prefill_main_kernel<128, 2><<<grid, 192, L::kBytes, stream>>>(maps.q, maps.k, maps.v, maps.o,
-                                                                  p);
+    using L = MainLayout<128, 2, 2>;
+    static_assert(L::kBytes <= 232448, "shared memory");
+    if ((e = set_smem(prefill_main_kernel<128, 2, 2>, L::kBytes)) != cudaSuccess) return e;
+    prefill_main_kernel<128, 2, 2><<<grid, 320, L::kBytes, stream>>>(maps.q, maps.k, maps.v,
+                                                                     maps.o, p);
   }
   return cudaGetLastError();
 }

@@ -111,6 +111,38 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
+// ---------------------------------------------------------------- global flags
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until *flag != 0 (acquire, GPU scope), bounded like mbar_wait; every
+// lane of the warp takes the same outcome.
+__device__ __forceinline__ bool warp_wait_flag(const unsigned* flag, unsigned* status,
+                                               volatile int* abort) {
+  bool ok = ld_acquire_gpu(flag) != 0u;
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      if (ld_acquire_gpu(flag) != 0u) { ok = true; break; }
+      if (*abort) break;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kDevTimeout);
+        *abort = 1;
+        break;
+      }
+      __nanosleep(100);
+    }
+  }
+  return __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -145,6 +177,16 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, 
       "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(tmap)),
       "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// The same store with an L2 eviction-priority hint.
+__device__ __forceinline__ void tma_store_3d_hint(const void* tmap, const void* src, int c0, int c1,
+                                                  int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3, %4}], [%1], %5;" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
 }
 

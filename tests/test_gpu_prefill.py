@@ -213,3 +213,42 @@ def test_full_gqa_32k(la, chunk):
 
 def test_full_long_1m(la):
     _full(la, synth.LONG_1M, 128, rows_only=True)
+
+
+# ------------------------------------------------------------------ fused kernel
+@pytest.mark.parametrize("Hq,Hkv,chunk", [(4, 2, 64), (2, 2, 64), (4, 1, 128), (6, 3, 64)])
+@pytest.mark.parametrize("nspan", [1, 2, 3, 7, 0, -1])
+def test_fused_span_counts(la, Hq, Hkv, chunk, nspan):
+    """The single-pass kernel for span counts 1, 2, 3, 7, automatic (0) and
+    one span per tile (-1), with an initial state; two calls on one workspace."""
+    B, N = 2, 1100
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=300 + Hq * 10 + Hkv + chunk)
+    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(7)) / 128
+    ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy())
+    qd, kd, vd = _cuda(q, k, v)
+    if nspan == -1:
+        nspan = la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).tiles_total
+    nbytes = la.api.la_prefill_fused_workspace_bytes(B, Hq, Hkv, N, 128, chunk, nspan)
+    assert nbytes > 0
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    for call in range(2):
+        S = S0.to(DEV)
+        o = torch.full_like(qd, float("nan"))
+        la.api.la_prefill_fused(qd, kd, vd, o, S, ws, chunk=chunk, nspan=nspan)
+        torch.cuda.synchronize()
+        assert_bf16_close(o.cpu(), ref_o, f"O nspan={nspan} call {call}")
+        assert_f32_close(S.cpu(), ref_S, f"final state nspan={nspan} call {call}", tol=STATE_REL_L2)
+    assert la.la_device_status()[1] == 0
+
+
+def test_fused_rejects_bad_span_count(la):
+    q, k, v = _cuda(*_qkv(1, 2, 2, 256, seed=9))
+    tiles = la.api.la_prefill_plan(1, 2, 2, 256, 128, 64).tiles_total
+    assert la.api.la_prefill_fused_workspace_bytes(1, 2, 2, 256, 128, 64, tiles + 1) == 0
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
+    with pytest.raises(la.LAError) as e:
+        la.api.la_prefill_fused(q, k, v, torch.empty_like(q), None, ws, chunk=64, nspan=tiles + 1)
+    assert e.value.code == 1
+    with pytest.raises(la.LAError) as e:
+        la.api.la_prefill_fused(q, k, v, torch.empty_like(q), None, ws[:64], chunk=64, nspan=1)
+    assert e.value.code == 5
