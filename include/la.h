@@ -125,6 +125,8 @@ la_status la_forward_ws(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la
  * states are published through GPU-scope flags; every wait is bounded.
  *   nspan <= 0 picks the span count for the problem and device; otherwise
  *   1 <= nspan <= ceil(N / tile) (tile = la_plan.tile).
+ *   lookahead: how many rounds the span-state items run ahead of the chunk
+ *   loops that need them (<= 0: 1; capped at nspan).
  *   workspace: device memory, 256-byte aligned, at least
  *   la_prefill_fused_workspace_bytes(..., nspan) bytes (entering states and
  *   flags); the call clears the flags on `stream` first (cudaMemsetAsync).
@@ -134,7 +136,8 @@ size_t la_prefill_fused_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d
                                         int nspan);
 la_status la_prefill_fused(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
                            float *S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
-                           int nspan, void *workspace, size_t workspace_bytes, la_stream stream);
+                           int nspan, int lookahead, void *workspace, size_t workspace_bytes,
+                           la_stream stream);
 
 /* ------------------------------------------------------------------------
  * Prefill without any device allocation.  The pages have no counterpart to

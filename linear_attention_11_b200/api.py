@@ -57,7 +57,7 @@ def _declare(lib):
         "la_forward_ws": ([P, P, P, P, P, I, I, I, L, I, I, P, S, P], I),
         "la_forward_noalloc": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
         "la_prefill_fused_workspace_bytes": ([I, I, I, L, I, I, I], S),
-        "la_prefill_fused": ([P, P, P, P, P, I, I, I, L, I, I, I, P, S, P], I),
+        "la_prefill_fused": ([P, P, P, P, P, I, I, I, L, I, I, I, I, P, S, P], I),
         "la_prefill_plan": ([I, I, I, L, I, I, PP], I),
         "la_prefill_span_states": ([P, P, I, I, L, I, PP, P, P], I),
         "la_prefill_scan": ([P, P, I, I, I, PP, P], I),
@@ -161,12 +161,13 @@ def la_prefill_fused_workspace_bytes(B, Hq, Hkv, N, d, chunk, nspan=0) -> int:
     return int(load_library().la_prefill_fused_workspace_bytes(B, Hq, Hkv, N, d, chunk, nspan))
 
 
-def la_prefill_fused(q, k, v, o, S, workspace, chunk: int = 64, nspan: int = 0, stream=None):
-    """The single-pass prefill with an explicit span count (0 = automatic)."""
+def la_prefill_fused(q, k, v, o, S, workspace, chunk: int = 64, nspan: int = 0,
+                     lookahead: int = 0, stream=None):
+    """The single-pass prefill with an explicit span count and lookahead (0 = automatic)."""
     B, Hq, Hkv, N, d = _dims(q, k)
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("la_prefill_fused", load_library().la_prefill_fused(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, nspan,
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, nspan, lookahead,
         _ptr(workspace), nbytes, _stream(stream)))
     return o
 

@@ -326,7 +326,7 @@ LA_EXPORT size_t la_prefill_fused_workspace_bytes(int B, int Hq, int Hkv, int64_
 
 LA_EXPORT la_status la_prefill_fused(const la_bf16* q, const la_bf16* k, const la_bf16* v,
                                      la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N,
-                                     int d, int chunk, int nspan, void* workspace,
+                                     int d, int chunk, int nspan, int lookahead, void* workspace,
                                      size_t workspace_bytes, la_stream stream) {
   if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
   la_plan plan;
@@ -352,7 +352,8 @@ LA_EXPORT la_status la_prefill_fused(const la_bf16* q, const la_bf16* k, const l
       !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
     return LA_ERR_CUDA;
   PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
-  return from_cuda(launch_prefill_fused(g, maps, S, workspace, status, sms,
+  if (lookahead <= 0) lookahead = 1;
+  return from_cuda(launch_prefill_fused(g, maps, S, workspace, status, sms, lookahead,
                                         static_cast<cudaStream_t>(stream)));
 }
 

@@ -37,7 +37,7 @@ cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& map
                                 const float* ws, unsigned* status, cudaStream_t stream);
 size_t fused_workspace_bytes(int B, int Hkv, int nspan);
 cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
-                                 void* workspace, unsigned* status, int num_sms,
+                                 void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
                               cudaStream_t stream);

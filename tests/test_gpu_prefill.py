@@ -217,10 +217,12 @@ def test_full_long_1m(la):
 
 # ------------------------------------------------------------------ fused kernel
 @pytest.mark.parametrize("Hq,Hkv,chunk", [(4, 2, 64), (2, 2, 64), (4, 1, 128), (6, 3, 64)])
-@pytest.mark.parametrize("nspan", [1, 2, 3, 7, 0, -1])
-def test_fused_span_counts(la, Hq, Hkv, chunk, nspan):
+@pytest.mark.parametrize("nspan,lookahead", [(1, 0), (2, 1), (3, 2), (7, 1), (7, 3), (7, 99),
+                                             (0, 0), (-1, 1), (-1, 4)])
+def test_fused_span_counts(la, Hq, Hkv, chunk, nspan, lookahead):
     """The single-pass kernel for span counts 1, 2, 3, 7, automatic (0) and
-    one span per tile (-1), with an initial state; two calls on one workspace."""
+    one span per tile (-1), state items 1 to all rounds ahead, with an
+    initial state; two calls on one workspace."""
     B, N = 2, 1100
     q, k, v = _qkv(B, Hq, Hkv, N, seed=300 + Hq * 10 + Hkv + chunk)
     S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(7)) / 128
@@ -234,7 +236,7 @@ def test_fused_span_counts(la, Hq, Hkv, chunk, nspan):
     for call in range(2):
         S = S0.to(DEV)
         o = torch.full_like(qd, float("nan"))
-        la.api.la_prefill_fused(qd, kd, vd, o, S, ws, chunk=chunk, nspan=nspan)
+        la.api.la_prefill_fused(qd, kd, vd, o, S, ws, chunk=chunk, nspan=nspan, lookahead=lookahead)
         torch.cuda.synchronize()
         assert_bf16_close(o.cpu(), ref_o, f"O nspan={nspan} call {call}")
         assert_f32_close(S.cpu(), ref_S, f"final state nspan={nspan} call {call}", tol=STATE_REL_L2)
