@@ -218,6 +218,16 @@ la_status la_forward_f32(const float *q, const float *k, const float *v, float *
 la_status la_decode_step(float *S, const la_bf16 *q, const la_bf16 *k, const la_bf16 *v,
                          la_bf16 *o, int B, int Hq, int Hkv, int d, la_stream stream);
 
+/* Several decode steps per launch for tokens that are all known in advance
+ * (speculative or draft tokens, short appended segments): for t = 0..steps-1,
+ *     S[b,g] += k[b,g,t]^T v[b,g,t];   o[b,h,t] = q[b,h,t] S[b,g]
+ * -- la_decode_step applied `steps` times, in fp32, with each state held in
+ * registers across the steps so it is read and written once per call.
+ * q, o [B,Hq,steps,d] and k, v [B,Hkv,steps,d] bf16 (the prefill layout with
+ * N = steps); S as la_decode_step.  Errors as la_decode_step. */
+la_status la_decode_steps(float *S, const la_bf16 *q, const la_bf16 *k, const la_bf16 *v,
+                          la_bf16 *o, int B, int Hq, int Hkv, int d, int steps, la_stream stream);
+
 /* ------------------------------------------------------------------------
  * Failure detection.
  * la_device_status: synchronises the current device, then stores the device

@@ -9,6 +9,7 @@ the library has not been built.
 from .api import (  # noqa: F401
     LAError,
     la_decode_step,
+    la_decode_steps,
     la_device_status,
     la_forward,
     la_forward_f32,

@@ -26,7 +26,8 @@ EXPORTS = ("la_status_string", "la_version", "la_forward", "la_forward_state",
            "la_forward_workspace_bytes", "la_forward_ws", "la_forward_noalloc",
            "la_prefill_fused_workspace_bytes", "la_prefill_fused", "la_prefill_plan",
            "la_prefill_span_states", "la_prefill_scan", "la_prefill_main", "la_forward_f32",
-           "la_decode_step", "la_device_status", "la_selftest_wait", "la_shutdown")
+           "la_decode_step", "la_decode_steps", "la_device_status", "la_selftest_wait",
+           "la_shutdown")
 
 
 class LAError(RuntimeError):
@@ -64,6 +65,7 @@ def _declare(lib):
         "la_prefill_main": ([P, P, P, P, P, I, I, I, L, I, PP, P], I),
         "la_forward_f32": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
         "la_decode_step": ([P, P, P, P, P, I, I, I, I, P], I),
+        "la_decode_steps": ([P, P, P, P, P, I, I, I, I, I, P], I),
         "la_device_status": ([ctypes.POINTER(ctypes.c_uint), I], I),
         "la_selftest_wait": ([L, P], I),
         "la_shutdown": ([], None),
@@ -213,6 +215,16 @@ def la_decode_step(S, q, k, v, o=None, stream=None):
     B, Hq, d = q.shape
     _check("la_decode_step", load_library().la_decode_step(
         _ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, k.shape[1], d, _stream(stream)))
+    return o
+
+
+def la_decode_steps(S, q, k, v, o=None, stream=None):
+    """Several decode steps: q [B,Hq,steps,d], k, v [B,Hkv,steps,d]; S updated in place."""
+    if o is None:
+        o = torch.empty_like(q)
+    B, Hq, steps, d = q.shape
+    _check("la_decode_steps", load_library().la_decode_steps(
+        _ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, k.shape[1], d, steps, _stream(stream)))
     return o
 
 

@@ -462,6 +462,28 @@ LA_EXPORT la_status la_decode_step(float* S, const la_bf16* q, const la_bf16* k,
       launch_decode(S, q, k, v, o, B, Hq, Hkv, d, static_cast<cudaStream_t>(stream)));
 }
 
+LA_EXPORT la_status la_decode_steps(float* S, const la_bf16* q, const la_bf16* k,
+                                    const la_bf16* v, la_bf16* o, int B, int Hq, int Hkv, int d,
+                                    int steps, la_stream stream) {
+  if (!S || !q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || steps <= 0 || Hq % Hkv != 0)
+    return LA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 32) return LA_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv > 0x7fffffff) return LA_ERR_INVALID_ARG;
+  if (!aligned16(S) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return LA_ERR_INVALID_ARG;
+  const size_t sbytes = (size_t)B * Hkv * d * d * 4, qbytes = (size_t)B * Hq * steps * d * 2,
+               kbytes = (size_t)B * Hkv * steps * d * 2;
+  if (overlap(o, qbytes, S, sbytes) || overlap(o, qbytes, q, qbytes) ||
+      overlap(o, qbytes, k, kbytes) || overlap(o, qbytes, v, kbytes) ||
+      overlap(S, sbytes, q, qbytes) || overlap(S, sbytes, k, kbytes) ||
+      overlap(S, sbytes, v, kbytes))
+    return LA_ERR_INVALID_ARG;
+  return from_cuda(launch_decode_steps(S, q, k, v, o, B, Hq, Hkv, d, steps,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 LA_EXPORT la_status la_device_status(unsigned int* flags, int clear) {
   if (!flags) return LA_ERR_INVALID_ARG;
   *flags = 0;

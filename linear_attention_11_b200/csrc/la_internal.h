@@ -43,6 +43,8 @@ cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
                               cudaStream_t stream);
 cudaError_t launch_decode(float* S, const void* q, const void* k, const void* v, void* o, int B,
                           int Hq, int Hkv, int d, cudaStream_t stream);
+cudaError_t launch_decode_steps(float* S, const void* q, const void* k, const void* v, void* o,
+                                int B, int Hq, int Hkv, int d, int steps, cudaStream_t stream);
 cudaError_t launch_forward_simt_f32(const float* q, const float* k, const float* v, float* o,
                                     const float* S_in, float* S_out, int B, int Hq, int Hkv,
                                     int64_t N, int d, int chunk, cudaStream_t stream);

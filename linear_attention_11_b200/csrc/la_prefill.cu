@@ -301,7 +301,10 @@ __global__ void __launch_bounds__(320, 1)
     const bool store_thread = (warp == 6 && lane == 0);
     bool ok = true;
 
-    // Entering state of this span (this warpgroup's half of the row).
+    // Entering state of this span (this warpgroup's half of the row).  The
+    // kernel may start before the scan has finished (programmatic dependent
+    // launch); only the workspace read waits for it.
+    griddep_wait();
     {
       const float4* src = reinterpret_cast<const float4*>(
           p.ws + ((size_t)bg * p.nspan + j) * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim);
@@ -471,6 +474,7 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
 
+  griddep_launch_dependents();  // the scan may be scheduled; it waits for this grid
   const int j = blockIdx.x % p.nspan;
   const int bg = blockIdx.x / p.nspan;
   const int tile_begin = (int)(((int64_t)j * p.tiles_total) / p.nspan);
@@ -602,6 +606,22 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
   return cudaGetLastError();
 }
 
+template <typename K>
+cudaError_t launch_dependent(K kernel, dim3 grid, int threads, int smem, cudaStream_t stream,
+                             const PrefillMaps& maps, const MainParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, maps.q, maps.k, maps.v, maps.o, p);
+}
+
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
                                 const float* ws, unsigned* status, cudaStream_t stream) {
   const int nsub = g.G / g.heads_per_tile;
@@ -612,16 +632,12 @@ cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& map
     using L = MainLayout<64, 2, 3>;
     static_assert(L::kBytes <= 232448, "shared memory");
     if ((e = set_smem(prefill_main_kernel<64, 2, 3>, L::kBytes)) != cudaSuccess) return e;
-    prefill_main_kernel<64, 2, 3><<<grid, 320, L::kBytes, stream>>>(maps.q, maps.k, maps.v, maps.o,
-                                                                    p);
-  } else {
-    using L = MainLayout<128, 2, 2>;
-    static_assert(L::kBytes <= 232448, "shared memory");
-    if ((e = set_smem(prefill_main_kernel<128, 2, 2>, L::kBytes)) != cudaSuccess) return e;
-    prefill_main_kernel<128, 2, 2><<<grid, 320, L::kBytes, stream>>>(maps.q, maps.k, maps.v,
-                                                                     maps.o, p);
+    return launch_dependent(prefill_main_kernel<64, 2, 3>, grid, 320, L::kBytes, stream, maps, p);
   }
-  return cudaGetLastError();
+  using L = MainLayout<128, 2, 2>;
+  static_assert(L::kBytes <= 232448, "shared memory");
+  if ((e = set_smem(prefill_main_kernel<128, 2, 2>, L::kBytes)) != cudaSuccess) return e;
+  return launch_dependent(prefill_main_kernel<128, 2, 2>, grid, 320, L::kBytes, stream, maps, p);
 }
 
 }  // namespace la

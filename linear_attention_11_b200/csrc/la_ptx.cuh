@@ -143,6 +143,18 @@ __device__ __forceinline__ bool warp_wait_flag(const unsigned* flag, unsigned* s
   return __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start before the previous kernel in the
+// stream has finished; griddep_wait() blocks until that kernel has completed
+// and its memory is visible.  griddep_launch_dependents() lets the next kernel
+// start early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

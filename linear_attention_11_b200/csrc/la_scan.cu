@@ -5,10 +5,13 @@
 // the final state S0 + K^T V ("MiniMax-01与Lightning Attention", section 2.2,
 // kv_sum over the whole sequence).  Elementwise fp32 adds, HBM/L2-bound: one
 // thread owns one float4 of the d x d matrix of one unit and walks the spans
-// in order, loading eight spans ahead to keep loads in flight.
+// in order, loading eight spans ahead to keep loads in flight.  Launched as a
+// programmatic dependent of the span-state kernel: it lets the chunk-loop
+// kernel start its copies, then waits for the span states.
 #include <cuda_runtime.h>
 
 #include "la_internal.h"
+#include "la_ptx.cuh"
 
 namespace la {
 namespace {
@@ -20,6 +23,8 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
 __global__ void __launch_bounds__(256)
     state_scan_kernel(float4* __restrict__ ws, float4* __restrict__ S, int nspan, int n4,
                       int blocks_per_unit) {
+  griddep_launch_dependents();  // the chunk-loop kernel may start its copies
+  griddep_wait();               // the span states are complete
   const size_t unit = blockIdx.x / blocks_per_unit;
   const int p = (blockIdx.x % blocks_per_unit) * blockDim.x + threadIdx.x;
   if (p >= n4) return;
@@ -50,10 +55,18 @@ cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
                               cudaStream_t stream) {
   const int n4 = d * d / 4;
   const int bpu = (n4 + 255) / 256;
-  const dim3 grid((unsigned)(units * bpu));
-  state_scan_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<float4*>(ws),
-                                              reinterpret_cast<float4*>(S), nspan, n4, bpu);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(units * bpu));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, state_scan_kernel, reinterpret_cast<float4*>(ws),
+                            reinterpret_cast<float4*>(S), nspan, n4, bpu);
 }
 
 }  // namespace la

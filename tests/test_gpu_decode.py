@@ -59,3 +59,43 @@ def test_decode_full_b256_64_steps(la):
         rel, _ = assert_bf16_close(o.cpu(), o_ref, f"o step {step}")
         worst = max(worst, rel)
     assert_f32_close(Sd.cpu(), Sref, "state after 64 steps", tol=1e-6)
+
+
+# ------------------------------------------------------------------ several steps per launch
+def _stack_steps(w, steps, B=None):
+    toks = [synth.decode_token(w, t, B=B) for t in range(steps)]
+    q = torch.stack([t[0] for t in toks], dim=2).contiguous()  # [B, Hq, steps, d]
+    k = torch.stack([t[1] for t in toks], dim=2).contiguous()  # [B, Hkv, steps, d]
+    v = torch.stack([t[2] for t in toks], dim=2).contiguous()
+    return q, k, v
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,steps", [(3, 4, 2, 128, 5), (2, 6, 3, 64, 17), (1, 32, 1, 128, 3),
+                                               (4, 8, 8, 128, 1), (2, 2, 1, 64, 40)])
+def test_decode_steps_matches_recurrence(la, B, Hq, Hkv, d, steps):
+    w = synth.Decode("t", B, Hq, Hkv, d, steps, 13)
+    S0 = synth.decode_state(w)
+    q, k, v = _stack_steps(w, steps)
+    ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy())
+    S = S0.to(DEV)
+    o = la.la_decode_steps(S, q.to(DEV), k.to(DEV), v.to(DEV))
+    torch.cuda.synchronize()
+    assert_bf16_close(o.cpu(), ref_o, "o")
+    assert_f32_close(S.cpu(), ref_S, "state", tol=1e-6)
+
+
+def test_decode_steps_equals_single_steps_bitwise(la):
+    """64 steps of the decode workload in one launch give exactly the outputs
+    and state of 64 single-step launches (same fp32 operations, same order)."""
+    w = synth.DECODE_B256
+    S0 = synth.decode_state(w)
+    q, k, v = _stack_steps(w, w.steps)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    S_multi = S0.to(DEV)
+    o_multi = la.la_decode_steps(S_multi, qd, kd, vd)
+    S_single = S0.to(DEV)
+    outs = [la.la_decode_step(S_single, qd[:, :, t].contiguous(), kd[:, :, t].contiguous(),
+                              vd[:, :, t].contiguous()) for t in range(w.steps)]
+    torch.cuda.synchronize()
+    assert torch.equal(S_multi, S_single)
+    assert torch.equal(o_multi, torch.stack(outs, dim=2))
