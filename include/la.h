@@ -115,6 +115,26 @@ la_status la_forward_ws(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la
                         void *workspace, size_t workspace_bytes, la_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Prefill from and to HOST memory, transfers pipelined against the compute.
+ * q, k, v, o are host pointers, page-locked (cudaHostAlloc / cudaHostRegister)
+ * so the copies run asynchronously, in the layouts above; S (nullable) is a
+ * DEVICE state as in la_forward_state.  The sequence is processed in pieces of
+ * `piece` tokens (0: about N/8; rounded up to whole tiles): piece p is copied
+ * in on a copy-in stream, computed on `stream` with the state carried from
+ * piece p-1 ([MX01] section 4.1: the state is the whole resume point), and
+ * copied out on a copy-out stream, so the two copy directions and the compute
+ * of neighbouring pieces overlap.  Same result as la_forward_state on the
+ * whole sequence (up to the rounding of the bf16 state copy at piece ends).
+ * Asynchronous: returns once the work is queued; the host buffers must stay
+ * valid and unmodified until `stream` has reached the end of the call.  Device
+ * buffers for two pieces come from the stream-ordered pool and go back to it.
+ * Errors as la_forward_state; piece < 0 is LA_ERR_INVALID_ARG.
+ * ---------------------------------------------------------------------- */
+la_status la_forward_host(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
+                          float *S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                          int64_t piece, la_stream stream);
+
+/* ------------------------------------------------------------------------
  * The prefill as one persistent kernel (an alternative schedule of the same
  * arithmetic; la_forward runs the three-kernel scheme below).  Every (batch, kv head) sequence is cut into `nspan`
  * spans; span-state items (K^T V of a span, then the chained prefix: the state

@@ -13,6 +13,7 @@ from .api import (  # noqa: F401
     la_device_status,
     la_forward,
     la_forward_f32,
+    la_forward_host,
     la_forward_state,
     la_status_string,
     library_path,

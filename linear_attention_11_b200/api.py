@@ -24,7 +24,8 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_E
 # Every symbol include/la.h declares.
 EXPORTS = ("la_status_string", "la_version", "la_forward", "la_forward_state",
            "la_forward_workspace_bytes", "la_forward_ws", "la_forward_noalloc",
-           "la_prefill_fused_workspace_bytes", "la_prefill_fused", "la_prefill_plan",
+           "la_forward_host", "la_prefill_fused_workspace_bytes", "la_prefill_fused",
+           "la_prefill_plan",
            "la_prefill_span_states", "la_prefill_scan", "la_prefill_main", "la_forward_f32",
            "la_decode_step", "la_decode_steps", "la_device_status", "la_selftest_wait",
            "la_shutdown")
@@ -57,6 +58,7 @@ def _declare(lib):
         "la_forward_workspace_bytes": ([I, I, I, L, I, I], S),
         "la_forward_ws": ([P, P, P, P, P, I, I, I, L, I, I, P, S, P], I),
         "la_forward_noalloc": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
+        "la_forward_host": ([P, P, P, P, P, I, I, I, L, I, I, L, P], I),
         "la_prefill_fused_workspace_bytes": ([I, I, I, L, I, I, I], S),
         "la_prefill_fused": ([P, P, P, P, P, I, I, I, L, I, I, I, I, P, S, P], I),
         "la_prefill_plan": ([I, I, I, L, I, I, PP], I),
@@ -156,6 +158,18 @@ def la_forward_noalloc(q, k, v, S=None, o=None, chunk: int = 64, stream=None):
     B, Hq, Hkv, N, d = _dims(q, k)
     _check("la_forward_noalloc", load_library().la_forward_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, _stream(stream)))
+    return o
+
+
+def la_forward_host(q, k, v, o=None, S=None, chunk: int = 64, piece: int = 0, stream=None):
+    """Prefill from and to pinned host tensors (q, k, v, o on the CPU, pinned);
+    S, if given, is a CUDA tensor.  Asynchronous on `stream`."""
+    if o is None:
+        o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("la_forward_host", load_library().la_forward_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, piece,
+        _stream(stream)))
     return o
 
 

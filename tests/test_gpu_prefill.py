@@ -254,3 +254,22 @@ def test_fused_rejects_bad_span_count(la):
     with pytest.raises(la.LAError) as e:
         la.api.la_prefill_fused(q, k, v, torch.empty_like(q), None, ws[:64], chunk=64, nspan=1)
     assert e.value.code == 5
+
+
+# ------------------------------------------------------------------ host buffers
+@pytest.mark.parametrize("N,piece,with_state", [(1000, 0, False), (1000, 128, True), (777, 300, True),
+                                                (64, 0, False)])
+def test_forward_host_pipelined(la, N, piece, with_state):
+    """Pinned host inputs and output, pieces pipelined against the compute:
+    the same result as the oracle, and the carried state as the final state."""
+    B, Hq, Hkv = 2, 4, 2
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=500 + N + piece)
+    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(8)) / 128
+    ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy() if with_state else None)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    S = S0.to(DEV) if with_state else None
+    o = la.la_forward_host(qh, kh, vh, S=S, chunk=64, piece=piece)
+    torch.cuda.synchronize()
+    assert_bf16_close(o, ref_o, f"O N={N} piece={piece}")
+    if with_state:
+        assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
