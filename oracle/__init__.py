@@ -18,6 +18,8 @@ recurrent(q, k, v, S0)    token recurrence S += k^T v; o = q S; returns (O, S)
 state(k, v)               S = K^T V (scalar loops)
 state_gemm(k, v)          S = K^T V (one fp64 matmul per head, for long sequences)
 decode(S, q, k, v)        one decode step on a copy of S; returns (o, S_new)
+backward(q, k, v, dO, S0, dSf, form)   gradients (dq, dk, dv, dS0) of the prefill
+                          for output gradient dO and final-state gradient dSf
 
 Inputs may be torch CPU tensors (float32 or bfloat16) or numpy arrays
 (float32, or uint16 holding bfloat16 bits).  Outputs are float64 numpy arrays.
@@ -55,8 +57,11 @@ def _bind(path: str):
     lib.la_oracle_recurrent.argtypes = [P, P, P, I, I, I, I, L, I, P, P, P, P, I]
     lib.la_oracle_state.argtypes = [P, P, I, I, I, L, I, P, I]
     lib.la_oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, P, I]
+    for f in (lib.la_oracle_backward_quadratic, lib.la_oracle_backward_recurrent):
+        f.argtypes = [P, P, P, P, I, I, I, I, L, I, P, P, P, P, P, P, I]
     for f in (lib.la_oracle_quadratic, lib.la_oracle_rows, lib.la_oracle_recurrent,
-              lib.la_oracle_state, lib.la_oracle_decode):
+              lib.la_oracle_state, lib.la_oracle_decode, lib.la_oracle_backward_quadratic,
+              lib.la_oracle_backward_recurrent):
         f.restype = ctypes.c_int
     return lib
 
@@ -218,3 +223,28 @@ def decode(S, q, k, v, nthreads: int | None = None, inplace: bool = False):
     if rc:
         raise ValueError(f"la_oracle_decode rc={rc}")
     return o, Sn
+
+
+def backward(q, k, v, dO, S0=None, dSf=None, form: str = "recurrent", nthreads: int | None = None):
+    """Gradients of the prefill: returns (dq, dk, dv, dS0) as float64 arrays.
+
+    form "quadratic" writes the sums out; "recurrent" runs a forward sweep for
+    dq and a reverse sweep for dk, dv (see la_oracle.c)."""
+    qa, ka, va, dt, (B, Hq, Hkv, N, d) = _prep(q, k, v)
+    (da, ddt) = _as_array(dO)
+    if ddt != dt or da.shape != qa.shape:
+        raise ValueError("dO must match q in dtype and shape")
+    f = {"quadratic": load().la_oracle_backward_quadratic,
+         "recurrent": load().la_oracle_backward_recurrent}[form]
+    s0 = None if S0 is None else np.ascontiguousarray(np.asarray(S0, np.float64).reshape(B, Hkv, d, d))
+    dsf = None if dSf is None else np.ascontiguousarray(np.asarray(dSf, np.float64).reshape(B, Hkv, d, d))
+    dq = np.empty((B, Hq, N, d), np.float64)
+    dk = np.empty((B, Hkv, N, d), np.float64)
+    dv = np.empty((B, Hkv, N, d), np.float64)
+    dS0 = np.empty((B, Hkv, d, d), np.float64)
+    rc = f(_ptr(qa), _ptr(ka), _ptr(va), _ptr(da), dt, B, Hq, Hkv, N, d,
+           _ptr(s0) if s0 is not None else None, _ptr(dsf) if dsf is not None else None,
+           _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dS0), nthreads or threads())
+    if rc:
+        raise ValueError(f"la_oracle_backward rc={rc}")
+    return dq, dk, dv, dS0

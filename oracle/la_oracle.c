@@ -289,3 +289,179 @@ int la_oracle_decode(double *S, const void *q, const void *k, const void *v, int
   parallel_units(decode_unit, &J, (int64_t)B * Hkv, nthreads);
   return 0;
 }
+
+/* ---- backward ----------------------------------------------------------
+ * Gradients of the prefill (fp64) for a loss whose gradient with respect to
+ * O is dO and with respect to the final state is dSf (nullable = 0).  From
+ * o_t = q_t S_t and S_t = S0 + sum_{s<=t} k_s^T v_s:
+ *   dq_t  = do_t S0^T + sum_{s<=t} (do_t . v_s) k_s
+ *   dk_s  = sum_{h in g} sum_{t>=s} (v_s . do_{t,h}) q_{t,h} + v_s dSf^T
+ *   dv_s  = sum_{h in g} sum_{t>=s} (k_s . q_{t,h}) do_{t,h} + k_s dSf
+ *   dS0   = dSf + sum_{h in g} sum_t q_{t,h}^T do_{t,h}
+ * Quadratic form: these sums written out.  Recurrent form: a forward sweep for
+ * dq (S_t as in the forward recurrence) and a reverse sweep for dk, dv with
+ * G_s = dSf + sum_{h} sum_{t>=s} q_{t,h}^T do_{t,h} (update, then read).
+ * Layouts as the forward; do, dq [B,Hq,N,d]; dk, dv [B,Hkv,N,d]; S0, dSf,
+ * dS0 [B,Hkv,d,d].  Outputs are double.  One unit = one (b, kv head). */
+
+typedef struct {
+  const void *q, *k, *v, *dO;
+  int dtype, B, Hq, Hkv, d;
+  int64_t N;
+  const double *S0, *dSf;
+  double *dq, *dk, *dv, *dS0;
+} bwd_job;
+
+static void backward_quadratic_unit(void *ctx, int64_t unit) {
+  bwd_job *J = (bwd_job *)ctx;
+  const int G = J->Hq / J->Hkv;
+  const int64_t b = unit / J->Hkv, g = unit % J->Hkv, N = J->N, d = J->d;
+  const int64_t kb = (b * J->Hkv + g) * N * d;
+  const double *S0 = J->S0 ? J->S0 + unit * d * d : NULL;
+  const double *dSf = J->dSf ? J->dSf + unit * d * d : NULL;
+  for (int hh = 0; hh < G; ++hh) { /* dq of every query head of the group */
+    const int64_t qb = (b * J->Hq + g * G + hh) * N * d;
+    for (int64_t t = 0; t < N; ++t) {
+      double *out = J->dq + qb + t * d;
+      for (int64_t i = 0; i < d; ++i) {
+        double a = 0.0;
+        if (S0)
+          for (int64_t j = 0; j < d; ++j) a += elem(J->dO, qb + t * d + j, J->dtype) * S0[i * d + j];
+        out[i] = a;
+      }
+      for (int64_t s = 0; s <= t; ++s) {
+        double a = 0.0;
+        for (int64_t j = 0; j < d; ++j)
+          a += elem(J->dO, qb + t * d + j, J->dtype) * elem(J->v, kb + s * d + j, J->dtype);
+        for (int64_t i = 0; i < d; ++i) out[i] += a * elem(J->k, kb + s * d + i, J->dtype);
+      }
+    }
+  }
+  for (int64_t s = 0; s < N; ++s) { /* dk, dv */
+    double *dk = J->dk + kb + s * d, *dv = J->dv + kb + s * d;
+    for (int64_t i = 0; i < d; ++i) {
+      double a = 0.0, c = 0.0;
+      if (dSf)
+        for (int64_t j = 0; j < d; ++j) {
+          a += elem(J->v, kb + s * d + j, J->dtype) * dSf[i * d + j]; /* (v dSf^T)_i */
+          c += elem(J->k, kb + s * d + j, J->dtype) * dSf[j * d + i]; /* (k dSf)_i */
+        }
+      dk[i] = a;
+      dv[i] = c;
+    }
+    for (int hh = 0; hh < G; ++hh) {
+      const int64_t qb = (b * J->Hq + g * G + hh) * N * d;
+      for (int64_t t = s; t < N; ++t) {
+        double vd = 0.0, kq = 0.0;
+        for (int64_t j = 0; j < d; ++j) {
+          vd += elem(J->v, kb + s * d + j, J->dtype) * elem(J->dO, qb + t * d + j, J->dtype);
+          kq += elem(J->k, kb + s * d + j, J->dtype) * elem(J->q, qb + t * d + j, J->dtype);
+        }
+        for (int64_t i = 0; i < d; ++i) {
+          dk[i] += vd * elem(J->q, qb + t * d + i, J->dtype);
+          dv[i] += kq * elem(J->dO, qb + t * d + i, J->dtype);
+        }
+      }
+    }
+  }
+  if (J->dS0) {
+    double *o = J->dS0 + unit * d * d;
+    for (int64_t e = 0; e < d * d; ++e) o[e] = dSf ? dSf[e] : 0.0;
+    for (int hh = 0; hh < G; ++hh) {
+      const int64_t qb = (b * J->Hq + g * G + hh) * N * d;
+      for (int64_t t = 0; t < N; ++t)
+        for (int64_t i = 0; i < d; ++i) {
+          const double qi = elem(J->q, qb + t * d + i, J->dtype);
+          for (int64_t j = 0; j < d; ++j) o[i * d + j] += qi * elem(J->dO, qb + t * d + j, J->dtype);
+        }
+    }
+  }
+}
+
+static void backward_recurrent_unit(void *ctx, int64_t unit) {
+  bwd_job *J = (bwd_job *)ctx;
+  const int G = J->Hq / J->Hkv;
+  const int64_t b = unit / J->Hkv, g = unit % J->Hkv, N = J->N, d = J->d;
+  const int64_t kb = (b * J->Hkv + g) * N * d;
+  double *St = (double *)malloc(sizeof(double) * d * d);
+  double *kt = (double *)malloc(sizeof(double) * d);
+  double *vt = (double *)malloc(sizeof(double) * d);
+  /* forward sweep: S_t, dq_t = do_t S_t^T */
+  if (J->S0)
+    memcpy(St, J->S0 + unit * d * d, sizeof(double) * d * d);
+  else
+    memset(St, 0, sizeof(double) * d * d);
+  for (int64_t t = 0; t < N; ++t) {
+    for (int64_t i = 0; i < d; ++i) {
+      kt[i] = elem(J->k, kb + t * d + i, J->dtype);
+      vt[i] = elem(J->v, kb + t * d + i, J->dtype);
+    }
+    for (int64_t i = 0; i < d; ++i)
+      for (int64_t j = 0; j < d; ++j) St[i * d + j] += kt[i] * vt[j];
+    for (int hh = 0; hh < G; ++hh) {
+      const int64_t qo = (b * J->Hq + g * G + hh) * N * d + t * d;
+      for (int64_t i = 0; i < d; ++i) {
+        double a = 0.0;
+        for (int64_t j = 0; j < d; ++j) a += elem(J->dO, qo + j, J->dtype) * St[i * d + j];
+        J->dq[qo + i] = a;
+      }
+    }
+  }
+  /* reverse sweep: G_s += sum_h q_{s,h}^T do_{s,h}; dk_s = v_s G_s^T; dv_s = k_s G_s */
+  if (J->dSf)
+    memcpy(St, J->dSf + unit * d * d, sizeof(double) * d * d);
+  else
+    memset(St, 0, sizeof(double) * d * d);
+  for (int64_t s = N - 1; s >= 0; --s) {
+    for (int hh = 0; hh < G; ++hh) {
+      const int64_t qo = (b * J->Hq + g * G + hh) * N * d + s * d;
+      for (int64_t i = 0; i < d; ++i) {
+        const double qi = elem(J->q, qo + i, J->dtype);
+        for (int64_t j = 0; j < d; ++j) St[i * d + j] += qi * elem(J->dO, qo + j, J->dtype);
+      }
+    }
+    for (int64_t i = 0; i < d; ++i) {
+      kt[i] = elem(J->k, kb + s * d + i, J->dtype);
+      vt[i] = elem(J->v, kb + s * d + i, J->dtype);
+    }
+    for (int64_t i = 0; i < d; ++i) {
+      double a = 0.0, c = 0.0;
+      for (int64_t j = 0; j < d; ++j) {
+        a += vt[j] * St[i * d + j]; /* (v G^T)_i */
+        c += kt[j] * St[j * d + i]; /* (k G)_i */
+      }
+      J->dk[kb + s * d + i] = a;
+      J->dv[kb + s * d + i] = c;
+    }
+  }
+  if (J->dS0) memcpy(J->dS0 + unit * d * d, St, sizeof(double) * d * d);
+  free(St);
+  free(kt);
+  free(vt);
+}
+
+static int backward(unit_fn fn, const void *q, const void *k, const void *v, const void *dO,
+                    int dtype, int B, int Hq, int Hkv, int64_t N, int d, const double *S0,
+                    const double *dSf, double *dq, double *dk, double *dv, double *dS0,
+                    int nthreads) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N < 0 || d <= 0 || Hq % Hkv || !dq || !dk || !dv) return 1;
+  bwd_job J = {q, k, v, dO, dtype, B, Hq, Hkv, d, N, S0, dSf, dq, dk, dv, dS0};
+  parallel_units(fn, &J, (int64_t)B * Hkv, nthreads);
+  return 0;
+}
+
+int la_oracle_backward_quadratic(const void *q, const void *k, const void *v, const void *dO,
+                                 int dtype, int B, int Hq, int Hkv, int64_t N, int d,
+                                 const double *S0, const double *dSf, double *dq, double *dk,
+                                 double *dv, double *dS0, int nthreads) {
+  return backward(backward_quadratic_unit, q, k, v, dO, dtype, B, Hq, Hkv, N, d, S0, dSf, dq, dk,
+                  dv, dS0, nthreads);
+}
+
+int la_oracle_backward_recurrent(const void *q, const void *k, const void *v, const void *dO,
+                                 int dtype, int B, int Hq, int Hkv, int64_t N, int d,
+                                 const double *S0, const double *dSf, double *dq, double *dk,
+                                 double *dv, double *dS0, int nthreads) {
+  return backward(backward_recurrent_unit, q, k, v, dO, dtype, B, Hq, Hkv, N, d, S0, dSf, dq, dk,
+                  dv, dS0, nthreads);
+}
