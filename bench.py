@@ -56,6 +56,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=None)
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override N (smaller case of the same workload, for profiling)")
@@ -330,6 +331,24 @@ def run_ours(args, w):
     }
     del ws1, wsf
 
+    # --- backward of the same workload (training): dq, dk, dv from dO
+    backward = None
+    if not args.no_backward:
+        dOd = synth.random_qkv(B, Hq, Hq, N, d, torch.bfloat16, 77)[0].to(dev)
+        for _ in range(2):
+            la.la_backward(qd, kd, vd, dOd, chunk=chunk, stream=stream)
+        reps = max(3, min(args.steps, 10))
+        tb, bclk = timed(lambda: la.la_backward(qd, kd, vd, dOd, chunk=chunk, stream=stream), reps,
+                         stream)
+        tb /= reps
+        bbytes = elt * (3 * B * Hq * N * d + 4 * B * Hkv * N * d)  # q, dO, dq + k, v, dk, dv
+        backward = {"ms_per_step": tb * 1e3, "mtok_s": world * B * N / tb / 1e6,
+                    "algorithmic_gb_s": bbytes / tb / 1e9,
+                    "frac_of_hbm_roofline": bbytes / tb / 1e9 / pk["hbm_gbs"],
+                    "bytes": bbytes, "clocks": bclk,
+                    "passes": "dq causal (grouped) + dv, dk anti-causal per query head + group sums"}
+        del dOd
+
     # --- end to end: pinned host buffers, copies inside the timed region.
     # The public host-buffer call pipelines the copies against the compute;
     # copies around the device call (serial) are reported beside it.
@@ -426,6 +445,7 @@ def run_ours(args, w):
         "alternatives": alternatives,
         "tflops_north_star": flops_ns / (t / args.steps) / 1e12,
         "e2e": e2e,
+        "backward": backward,
         "decode": decode,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

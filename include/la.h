@@ -220,6 +220,26 @@ la_status la_prefill_main(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, 
                           const la_plan *plan, la_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Backward of the bf16 prefill (training).  For a loss with gradient dO
+ * [B,Hq,N,d] on the output and dSf [B,Hkv,d,d] (nullable = 0) on the final
+ * state, with S0 (nullable = 0) the initial state of the forward call:
+ *   dq_t = do_t S0^T + sum_{s<=t} (do_t . v_s) k_s
+ *   dk_s = sum_{h in group} sum_{t>=s} (v_s . do_{t,h}) q_{t,h} + v_s dSf^T
+ *   dv_s = sum_{h in group} sum_{t>=s} (k_s . q_{t,h}) do_{t,h} + k_s dSf
+ *   dS0  = dSf + sum_{h in group} sum_t q_{t,h}^T do_{t,h}    (dS0 nullable)
+ * (the chain rule through o_t = q_t S_t, S_t = S0 + sum_{s<=t} k_s^T v_s of
+ * [VGX]).  dq is the forward pass itself on (dO, V, K, S0^T); dk and dv are
+ * anti-causal passes of the same tensor-core kernels, one per query head,
+ * summed over each group.  dq [B,Hq,N,d], dk, dv [B,Hkv,N,d] bf16 outputs
+ * (no overlap with the inputs).  Scratch comes from the stream-ordered pool.
+ * d = 128, chunk in {64, 128} (the chunk of the dq pass; the others use 128).
+ * Errors as la_forward_state. */
+la_status la_backward(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, const la_bf16 *dO,
+                      const float *S0, const float *dSf, la_bf16 *dq, la_bf16 *dk, la_bf16 *dv,
+                      float *dS0, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
+                      la_stream stream);
+
+/* ------------------------------------------------------------------------
  * Prefill in fp32 (inputs, output and state fp32; SIMT fp32 arithmetic).
  * Same definition and arguments as la_forward_state; d in {64, 128}, chunk in
  * {64, 128}.  For checking at fp32 precision, not tuned for speed.

@@ -8,6 +8,7 @@ the library has not been built.
 """
 from .api import (  # noqa: F401
     LAError,
+    la_backward,
     la_decode_step,
     la_decode_steps,
     la_device_status,

@@ -25,7 +25,7 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_E
 EXPORTS = ("la_status_string", "la_version", "la_forward", "la_forward_state",
            "la_forward_workspace_bytes", "la_forward_ws", "la_forward_noalloc",
            "la_forward_host", "la_prefill_fused_workspace_bytes", "la_prefill_fused",
-           "la_prefill_plan",
+           "la_prefill_plan", "la_backward",
            "la_prefill_span_states", "la_prefill_scan", "la_prefill_main", "la_forward_f32",
            "la_decode_step", "la_decode_steps", "la_device_status", "la_selftest_wait",
            "la_shutdown")
@@ -66,6 +66,7 @@ def _declare(lib):
         "la_prefill_scan": ([P, P, I, I, I, PP, P], I),
         "la_prefill_main": ([P, P, P, P, P, I, I, I, L, I, PP, P], I),
         "la_forward_f32": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
+        "la_backward": ([P, P, P, P, P, P, P, P, P, P, I, I, I, L, I, I, P], I),
         "la_decode_step": ([P, P, P, P, P, I, I, I, I, P], I),
         "la_decode_steps": ([P, P, P, P, P, I, I, I, I, I, P], I),
         "la_device_status": ([ctypes.POINTER(ctypes.c_uint), I], I),
@@ -211,6 +212,19 @@ def la_prefill_main(q, k, v, o, ws, plan: la_plan, stream=None):
     _check("la_prefill_main", load_library().la_prefill_main(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ws), B, Hq, Hkv, N, d, ctypes.byref(plan),
         _stream(stream)))
+
+
+def la_backward(q, k, v, dO, S0=None, dSf=None, want_dS0: bool = False, chunk: int = 64,
+                stream=None):
+    """Gradients (dq, dk, dv, dS0 or None) of the prefill for output gradient dO
+    and final-state gradient dSf (CUDA tensors; S0 the forward's initial state)."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dS0 = torch.empty(B, Hkv, d, d, dtype=torch.float32, device=q.device) if want_dS0 else None
+    _check("la_backward", load_library().la_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(S0), _ptr(dSf), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(dS0), B, Hq, Hkv, N, d, chunk, _stream(stream)))
+    return dq, dk, dv, dS0
 
 
 def la_forward_f32(q, k, v, o=None, S=None, chunk: int = 64, stream=None):

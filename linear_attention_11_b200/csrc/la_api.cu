@@ -172,6 +172,11 @@ la_status check_prefill_ptrs(const void* q, const void* k, const void* v, const 
 
 }  // namespace
 
+unsigned* device_status_ptr() {
+  unsigned* st = nullptr;
+  return device_info(&st, nullptr) ? st : nullptr;
+}
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, int64_t heads,
                     int box_rows) {
   {

@@ -26,6 +26,9 @@ struct PrefillMaps {
   CUtensorMap q, k, v, o;
 };
 
+// Device address of the status word on the current device (nullptr on failure).
+unsigned* device_status_ptr();
+
 // Builds a 3-D bf16 tensor map; returns false on failure.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, int64_t heads,
                     int box_rows);
@@ -33,14 +36,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, i
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
                                cudaStream_t stream);
+// qdiv: query rows of head h come from head h / qdiv of the query tensor map;
+// reverse: anti-causal pass (sum over s >= t), the tiles of every span walked
+// from the end.  The forward pass is qdiv = 1, reverse = 0.
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
-                                const float* ws, unsigned* status, cudaStream_t stream);
+                                const float* ws, unsigned* status, cudaStream_t stream,
+                                int qdiv = 1, int reverse = 0);
 size_t fused_workspace_bytes(int B, int Hkv, int nspan);
 cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
                                  void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);
+// reverse: ws[j] <- S0 + sum_{i>j} ws[i] (the state entering span j of a
+// backwards walk); S receives S0 + sum_i ws[i] either way.
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int reverse = 0);
 cudaError_t launch_decode(float* S, const void* q, const void* k, const void* v, void* o, int B,
                           int Hq, int Hkv, int d, cudaStream_t stream);
 cudaError_t launch_decode_steps(float* S, const void* q, const void* k, const void* v, void* o,

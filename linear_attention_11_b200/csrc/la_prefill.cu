@@ -53,6 +53,8 @@ struct MainParams {
   const float* ws;
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total;
+  int qdiv;     // query rows of head h come from head h / qdiv of the query tensor
+  int reverse;  // 1: anti-causal (s >= t), tiles of a span walked from the end
 };
 
 // Shared memory of the main kernel: a ring of Q tiles, a separate ring of K/V
@@ -131,6 +133,8 @@ __global__ void __launch_bounds__(320, 1)
   const int tile_end = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
   const int ntiles = tile_end - tile_begin;
   const int head0 = g * p.G + hs * HPT;
+  // i-th tile this CTA processes (the span is walked backwards in reverse mode)
+  auto tile_at = [&](int i) { return p.reverse ? tile_end - 1 - i : tile_begin + i; };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -180,14 +184,13 @@ __global__ void __launch_bounds__(320, 1)
         const int s = i % QST;
         if (i >= QST && !mbar_wait(&q_empty[s], ((i / QST) - 1) & 1, p.status, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[s], kQBytes);
-        const int c1 = (tile_begin + i) * T;
+        const int c1 = tile_at(i) * T;
         uint8_t* q_dst = sm + (sQ(i) - base);
 #pragma unroll
         for (int hh = 0; hh < HPT; ++hh) {
-          tma_load_3d(q_dst + hh * T * 128, &map_q, &q_full[s], 0, c1, b * p.Hq + head0 + hh,
-                      pol_q);
-          tma_load_3d(q_dst + kHalf + hh * T * 128, &map_q, &q_full[s], 64, c1,
-                      b * p.Hq + head0 + hh, pol_q);
+          const int qh = (b * p.Hq + head0 + hh) / p.qdiv;
+          tma_load_3d(q_dst + hh * T * 128, &map_q, &q_full[s], 0, c1, qh, pol_q);
+          tma_load_3d(q_dst + kHalf + hh * T * 128, &map_q, &q_full[s], 64, c1, qh, pol_q);
         }
         issued = i + 1;
       }
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(320, 1)
         if (i >= KVST && !mbar_wait(&kv_empty[s], ((i / KVST) - 1) & 1, p.status, abort_flag))
           break;
         mbar_arrive_expect_tx(&kv_full[s], L::kKVBytes);
-        const int c1 = (tile_begin + i) * T;
+        const int c1 = tile_at(i) * T;
         uint8_t* k_dst = sm + (sK(i) - base);
         uint8_t* v_dst = sm + (sV(i) - base);
         tma_load_3d(k_dst, &map_k, &kv_full[s], 0, c1, bg, pol_kv);
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(320, 1)
     const int t_in = r % T;
     const int blk0 = wg1 ? 0 : 2;  // state column blocks this warpgroup converts
     const bool store_thread = (warp == 6 && lane == 0);
+    const bool reverse = p.reverse != 0;
     bool ok = true;
 
     // Entering state of this span (this warpgroup's half of the row).  The
@@ -362,8 +366,10 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
             const int s0 = blk * 32 + 2 * m;
-            const float f0 = (s0 <= t_in) ? __uint_as_float(a[blk][2 * m]) : 0.0f;
-            const float f1 = (s0 + 1 <= t_in) ? __uint_as_float(a[blk][2 * m + 1]) : 0.0f;
+            const bool keep0 = reverse ? (s0 >= t_in) : (s0 <= t_in);
+            const bool keep1 = reverse ? (s0 + 1 >= t_in) : (s0 + 1 <= t_in);
+            const float f0 = keep0 ? __uint_as_float(a[blk][2 * m]) : 0.0f;
+            const float f1 = keep1 ? __uint_as_float(a[blk][2 * m + 1]) : 0.0f;
             pk[m] = pack_bf16x2(f0, f1);
           }
           tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
@@ -414,7 +420,7 @@ __global__ void __launch_bounds__(320, 1)
           if (!warp_wait(store_ready, i & 1, p.status, abort_flag)) { ok = false; break; }
         }
         if (store_thread) {
-          const int c1 = (tile_begin + i) * T;
+          const int c1 = tile_at(i) * T;
           const uint8_t* src = sm + (stage_o - base);
 #pragma unroll
           for (int hh = 0; hh < HPT; ++hh) {
@@ -623,9 +629,10 @@ cudaError_t launch_dependent(K kernel, dim3 grid, int threads, int smem, cudaStr
 }
 
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
-                                const float* ws, unsigned* status, cudaStream_t stream) {
+                                const float* ws, unsigned* status, cudaStream_t stream, int qdiv,
+                                int reverse) {
   const int nsub = g.G / g.heads_per_tile;
-  MainParams p{ws, status, g.Hq, g.Hkv, g.G, nsub, g.nspan, g.tiles_total};
+  MainParams p{ws, status, g.Hq, g.Hkv, g.G, nsub, g.nspan, g.tiles_total, qdiv, reverse};
   const dim3 grid((unsigned)(g.B * g.Hkv * g.nspan * nsub));
   cudaError_t e;
   if (g.tile == 64) {

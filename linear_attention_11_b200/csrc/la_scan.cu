@@ -22,7 +22,7 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
 
 __global__ void __launch_bounds__(256)
     state_scan_kernel(float4* __restrict__ ws, float4* __restrict__ S, int nspan, int n4,
-                      int blocks_per_unit) {
+                      int blocks_per_unit, int reverse) {
   griddep_launch_dependents();  // the chunk-loop kernel may start its copies
   griddep_wait();               // the span states are complete
   const size_t unit = blockIdx.x / blocks_per_unit;
@@ -30,6 +30,15 @@ __global__ void __launch_bounds__(256)
   if (p >= n4) return;
   float4* w = ws + unit * (size_t)nspan * n4 + p;
   float4 carry = S ? S[unit * n4 + p] : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (reverse) {  // spans from the last to the first
+    for (int j = nspan - 1; j >= 0; --j) {
+      const float4 x = w[(size_t)j * n4];
+      w[(size_t)j * n4] = carry;
+      carry = add4(carry, x);
+    }
+    if (S) S[unit * n4 + p] = carry;
+    return;
+  }
   int j = 0;
   for (; j + 8 <= nspan; j += 8) {
     float4 x[8];
@@ -52,7 +61,7 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int reverse) {
   const int n4 = d * d / 4;
   const int bpu = (n4 + 255) / 256;
   cudaLaunchConfig_t cfg = {};
@@ -66,7 +75,7 @@ cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, state_scan_kernel, reinterpret_cast<float4*>(ws),
-                            reinterpret_cast<float4*>(S), nspan, n4, bpu);
+                            reinterpret_cast<float4*>(S), nspan, n4, bpu, reverse);
 }
 
 }  // namespace la
