@@ -429,6 +429,23 @@ def run_ours(args, w):
             "speedup_vs_single_steps": per * dw.steps / tm,
             "gb_s": mbytes / tm / 1e9, "fp32_tflop_s": flops / tm / 1e12,
             "note": "fp32 FMA recurrence, state in registers; bound by fp32 ALU throughput"}
+        # the same tokens through the chunked tensor-core form: one span per
+        # (sequence, kv head), so la_forward_state is a single chunk-loop
+        # launch reading S and writing the final S (plus a counter reset)
+        for _ in range(3):
+            la.la_forward_state(qs, ks, vs, S=S, o=os_, chunk=64, stream=stream)
+        tc, tclk = timed(lambda: la.la_forward_state(qs, ks, vs, S=S, o=os_, chunk=64,
+                                                     stream=stream), reps, stream)
+        tc /= reps
+        decode["multi_step_tensor_core"] = {
+            "us_per_call": tc * 1e6, "tokens_per_call": dw.steps,
+            "us_per_token_step": tc * 1e6 / dw.steps,
+            "speedup_vs_single_steps": per * dw.steps / tc,
+            "gb_s": mbytes / tc / 1e9, "frac_of_hbm_peak": mbytes / tc / 1e9 / pk["hbm_gbs"],
+            "bytes_per_call": mbytes, "clocks": tclk,
+            "api": "la_forward_state on [B,H,64,d] with S in/out (chunk 64)",
+            "note": "bf16 operands, fp32 state in tensor memory; outputs within the bf16 "
+                    "tolerance of the oracle, not bitwise equal to single steps"}
 
     line = {
         "metric": "causal lightning-attn prefill throughput (Mtok/s); decode-step GB/s",

@@ -86,7 +86,10 @@ int la_version(void);
  * Uses a workspace for the per-span states: la_forward / la_forward_state take
  * it from the device's default stream-ordered memory pool (cudaMallocAsync and
  * cudaFreeAsync on `stream`; the pool keeps the memory cached between calls),
- * la_forward_ws takes one from the caller.
+ * la_forward_ws takes one from the caller.  When the plan has one span per
+ * (batch, kv head) -- many sequences or heads, short N -- the call is a single
+ * chunk-loop launch that reads the initial state and writes the final one
+ * itself, and the workspace holds only B * Hkv counters.
  *
  * Errors: LA_ERR_INVALID_ARG (null or misaligned pointer, B/Hq/Hkv/N <= 0,
  * Hq % Hkv, o overlapping an input), LA_ERR_UNSUPPORTED (d != 128, chunk not
@@ -168,10 +171,10 @@ la_status la_prefill_fused(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v,
  * the span-state workspace taken from one 32 MiB file-scope device array
  * instead of an allocation; every GPU that loads this part of the library
  * keeps that array until the process exits.
- *   - Limit: B * Hkv * d * d * 4 bytes (one span per (batch, kv head)) must
- *     fit in 32 MiB, i.e. B * Hkv <= 512 at d = 128; beyond that the call
- *     returns LA_ERR_WORKSPACE.  Within it, the span count is lowered when
- *     the usual plan would not fit.
+ *   - Limit: the span states (B * Hkv * nspan * d * d * 4 bytes) must fit in
+ *     32 MiB; the span count is lowered until they do, down to one span per
+ *     (batch, kv head), which runs as the single chunk-loop launch and needs
+ *     only B * Hkv * 4 bytes (LA_ERR_WORKSPACE beyond 8M kv heads).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls share the array: calls whose work overlaps on the GPU race

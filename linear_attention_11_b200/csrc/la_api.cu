@@ -218,6 +218,34 @@ __global__ void selftest_wait_kernel(unsigned* status, const unsigned* flag, int
 
 }  // namespace
 
+size_t forward_workspace_bytes(const la_plan& plan, int B, int Hkv) {
+  if (plan.nspan == 1) return (((size_t)B * Hkv * sizeof(unsigned)) + 255) & ~(size_t)255;
+  return (size_t)plan.workspace_bytes;
+}
+
+la_status forward_single_span(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
+                              float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
+                              unsigned* tickets, cudaStream_t stream) {
+  if (plan.nspan != 1) return LA_ERR_INVALID_ARG;
+  unsigned* status = nullptr;
+  if (!device_info(&status, nullptr)) return LA_ERR_CUDA;
+  PrefillMaps maps;
+  if (!make_tmap_bf16(&maps.q, q, N, (int64_t)B * Hq, plan.tile) ||
+      !make_tmap_bf16(&maps.o, o, N, (int64_t)B * Hq, plan.tile) ||
+      !make_tmap_bf16(&maps.k, k, N, (int64_t)B * Hkv, plan.tile) ||
+      !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
+    return LA_ERR_CUDA;
+  PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
+  const bool need_tickets = S && g.G / g.heads_per_tile > 1;
+  if (need_tickets) {
+    if (!tickets) return LA_ERR_WORKSPACE;
+    if (cudaMemsetAsync(tickets, 0, (size_t)B * Hkv * sizeof(unsigned), stream) != cudaSuccess)
+      return LA_ERR_CUDA;
+  }
+  return from_cuda(launch_prefill_main(g, maps, S, status, stream, 1, 0, S,
+                                       need_tickets ? tickets : nullptr));
+}
+
 cudaError_t launch_selftest_wait(unsigned* status, int64_t timeout_ns, cudaStream_t stream) {
   void* flag = nullptr;
   cudaError_t e = cudaGetSymbolAddress(&flag, g_never_set);
@@ -257,7 +285,7 @@ LA_EXPORT la_status la_prefill_plan(int B, int Hq, int Hkv, int64_t N, int d, in
 LA_EXPORT size_t la_forward_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d, int chunk) {
   la_plan p;
   if (la_prefill_plan(B, Hq, Hkv, N, d, chunk, &p) != LA_OK) return 0;
-  return (size_t)p.workspace_bytes;
+  return forward_workspace_bytes(p, B, Hkv);
 }
 
 LA_EXPORT la_status la_prefill_span_states(const la_bf16* k, const la_bf16* v, int B, int Hkv,
@@ -372,8 +400,11 @@ LA_EXPORT la_status la_forward_ws(const la_bf16* q, const la_bf16* k, const la_b
   if (st != LA_OK) return st;
   if ((st = check_prefill_ptrs(q, k, v, o, S, B, Hq, Hkv, N, d)) != LA_OK) return st;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      workspace_bytes < (size_t)plan.workspace_bytes)
+      workspace_bytes < forward_workspace_bytes(plan, B, Hkv))
     return LA_ERR_WORKSPACE;
+  if (plan.nspan == 1)  // one span per (batch, kv head): the chunk loop alone
+    return forward_single_span(q, k, v, o, S, B, Hq, Hkv, N, plan,
+                               static_cast<unsigned*>(workspace), static_cast<cudaStream_t>(stream));
   float* ws = static_cast<float*>(workspace);
   if ((st = la_prefill_span_states(k, v, B, Hkv, N, d, &plan, ws, stream)) != LA_OK) return st;
   if ((st = la_prefill_scan(ws, S, B, Hkv, d, &plan, stream)) != LA_OK) return st;

@@ -74,7 +74,10 @@ LA_EXPORT la_status la_forward_host(const la_bf16* q, const la_bf16* k, const la
 
   const size_t qrows = (size_t)B * Hq, krows = (size_t)B * Hkv;
   const size_t qbytes = qrows * piece * d * 2, kbytes = krows * piece * d * 2;
-  const size_t ws_bytes = la_forward_workspace_bytes(B, Hq, Hkv, piece, d, chunk);
+  // one workspace for every piece: the full pieces' or the shorter last one's
+  const int64_t last = N - (npieces - 1) * piece;
+  const size_t ws_bytes = std::max(la_forward_workspace_bytes(B, Hq, Hkv, piece, d, chunk),
+                                   la_forward_workspace_bytes(B, Hq, Hkv, last, d, chunk));
   const size_t sbytes = (size_t)B * Hkv * d * d * 4;
   if (ws_bytes == 0) return LA_ERR_CUDA;
   // two piece buffers (q, k, v, o), a carried state when the caller gives none,

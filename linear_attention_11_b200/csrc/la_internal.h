@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "la.h"
+
 namespace la {
 
 constexpr int kHeadDim = 128;   // head dim of the tensor-core path
@@ -38,11 +40,26 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                cudaStream_t stream);
 // qdiv: query rows of head h come from head h / qdiv of the query tensor map;
 // reverse: anti-causal pass (sum over s >= t), the tiles of every span walked
-// from the end.  The forward pass is qdiv = 1, reverse = 0.
+// from the end.  The forward pass is qdiv = 1, reverse = 0.  ws == nullptr
+// starts every span from a zero state.  s_out (nspan == 1 only; else
+// cudaErrorInvalidValue): the final state [B*Hkv, d, d] is written there; when
+// s_out is ws itself (in place) and G / heads_per_tile > 1, tickets must point
+// to B*Hkv zeroed counters.
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
                                 const float* ws, unsigned* status, cudaStream_t stream,
-                                int qdiv = 1, int reverse = 0);
+                                int qdiv = 1, int reverse = 0, float* s_out = nullptr,
+                                unsigned* tickets = nullptr);
 size_t fused_workspace_bytes(int B, int Hkv, int nspan);
+// The whole bf16 prefill of a plan with nspan == 1 as one chunk-loop launch
+// that reads S (nullable: zero) and writes the final state back into it.
+// `tickets`: device memory for B*Hkv counters (zeroed here), needed when S is
+// given and a kv group spans several CTAs.  Arguments already validated.
+la_status forward_single_span(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
+                              float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
+                              unsigned* tickets, cudaStream_t stream);
+// Workspace bytes la_forward_ws needs for `plan`: the span states, or only
+// the tickets of the single-span launch.
+size_t forward_workspace_bytes(const la_plan& plan, int B, int Hkv);
 cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
                                  void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);

@@ -5,8 +5,9 @@
 // and rejects foreign allocations, or a hard-real-time path that must not
 // block on the driver's allocator).
 //
-// The span-state workspace that la_forward takes from the stream-ordered pool
-// lives instead in one file-scope device array of fixed size.  Every GPU that
+// The workspace that la_forward takes from the stream-ordered pool (span
+// states, or the counters of the single-span launch) lives instead in one
+// file-scope device array of fixed size.  Every GPU that
 // loads this part of the library holds the array until the process exits.
 // Every call uses the same array, so calls whose work overlaps on the GPU
 // (other streams, other host threads) race on it and must be serialised by
@@ -14,9 +15,11 @@
 // nothing left by an earlier call needs clearing.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "la.h"
+#include "la_internal.h"
 
 #define LA_EXPORT extern "C" __attribute__((visibility("default")))
 
@@ -70,16 +73,21 @@ LA_EXPORT la_status la_forward_noalloc(const la_bf16* q, const la_bf16* k, const
       overlap(S, sbytes, q, qbytes) || overlap(S, sbytes, k, kbytes) ||
       overlap(S, sbytes, v, kbytes))
     return LA_ERR_INVALID_ARG;
-  // Fewer spans if the planned workspace exceeds the array; reject when even
-  // one span per (batch, kv head) does not fit.
+  // Fewer spans if the planned span states exceed the array; a single span
+  // needs only the counters of the one-launch path (B * Hkv * 4 bytes).
   const int64_t per_span = (int64_t)B * Hkv * d * d * (int64_t)sizeof(float);
-  if (per_span > (int64_t)kScratchBytes) return LA_ERR_WORKSPACE;
-  if (plan.workspace_bytes > (int64_t)kScratchBytes) {
-    plan.nspan = (int32_t)((int64_t)kScratchBytes / per_span);
+  if (plan.nspan > 1 && plan.workspace_bytes > (int64_t)kScratchBytes) {
+    plan.nspan = (int32_t)std::max<int64_t>(1, (int64_t)kScratchBytes / per_span);
     plan.workspace_bytes = per_span * plan.nspan;
   }
   float* ws = static_cast<float*>(scratch_on_current_device());
   if (!ws) return LA_ERR_CUDA;
+  if (plan.nspan == 1) {
+    if (la::forward_workspace_bytes(plan, B, Hkv) > kScratchBytes) return LA_ERR_WORKSPACE;
+    return la::forward_single_span(q, k, v, o, S, B, Hq, Hkv, N, plan,
+                                   reinterpret_cast<unsigned*>(ws),
+                                   static_cast<cudaStream_t>(stream));
+  }
   if ((st = la_prefill_span_states(k, v, B, Hkv, N, d, &plan, ws, stream)) != LA_OK) return st;
   if ((st = la_prefill_scan(ws, S, B, Hkv, d, &plan, stream)) != LA_OK) return st;
   return la_prefill_main(q, k, v, o, ws, B, Hq, Hkv, N, d, &plan, stream);

@@ -14,6 +14,10 @@
 //   prefill_main_kernel  one CTA per (batch, kv head, head subset, span): the
 //                        chunk loop of [VGX] over the span, starting from the
 //                        state that enters it (prepared by the scan kernel).
+//                        With one span per (batch, kv head) it can also run
+//                        alone: it reads the initial state itself and writes
+//                        the final one from tensor memory after the last
+//                        chunk's update (no span-state or scan kernel).
 //
 // Main-kernel tile: 128 rows = HPT query heads of one kv group x T tokens
 // (T = 64, HPT = 2 or T = 128, HPT = 1); d = 128.  Per tile c:
@@ -50,11 +54,20 @@ namespace la {
 namespace {
 
 struct MainParams {
-  const float* ws;
+  const float* ws;  // state entering span j of unit bg at ws[bg * nspan + j]; nullptr: zero
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total;
   int qdiv;     // query rows of head h come from head h / qdiv of the query tensor
   int reverse;  // 1: anti-causal (s >= t), tiles of a span walked from the end
+  // Final state (nspan == 1 only): after the last tile the state in tensor
+  // memory is entering state + K^T V of the whole sequence, and one CTA of
+  // each (batch, kv head) writes it to s_out[bg].  s_out may be the ws array
+  // itself (in place): then `tickets` (nsub > 1) holds one zeroed counter per
+  // bg; every CTA takes a ticket after reading its entering state, and the
+  // one that draws the last ticket -- all its siblings have read by then --
+  // writes.  Without tickets the head subset 0 writes.
+  float* s_out;
+  unsigned* tickets;
 };
 
 // Shared memory of the main kernel: a ring of Q tiles, a separate ring of K/V
@@ -80,7 +93,9 @@ struct MainLayout {
   static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
 };
 
-template <int T, int QST, int KVST>
+// kFinal: the final state is written (MainParams::s_out); a separate
+// instantiation, so the staged kernel carries none of that code.
+template <int T, int QST, int KVST, bool kFinal>
 __global__ void __launch_bounds__(320, 1)
     prefill_main_kernel(const __grid_constant__ CUtensorMap map_q,
                         const __grid_constant__ CUtensorMap map_k,
@@ -284,6 +299,15 @@ __global__ void __launch_bounds__(320, 1)
           mma_commit(&kv_empty[i % KVST]);
           if (!kLookahead && !issue_qk(i + 1)) break;
         } else {
+          if constexpr (kFinal) {  // the last chunk's update completes the final state
+#pragma unroll
+            for (int kk = 0; kk < T / 16; ++kk) {
+              const uint64_t da = smem_desc_sw128(k_addr + kk * 2048, T * 128, 1024);
+              const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
+              mma_ss(tmem + kColS, da, db, IDESC_KV, 1u);
+            }
+            mma_commit(s_full);
+          }
           mma_commit(&kv_empty[i % KVST]);
         }
       }
@@ -300,6 +324,7 @@ __global__ void __launch_bounds__(320, 1)
     const int r = quarter * 32 + lane;  // TMEM lane = tile row = state row
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int t_in = r % T;
+    const int diag_blk = t_in / 32;  // the 32-column score block holding this warp's diagonal
     const int blk0 = wg1 ? 0 : 2;  // state column blocks this warpgroup converts
     const bool store_thread = (warp == 6 && lane == 0);
     const bool reverse = p.reverse != 0;
@@ -310,15 +335,21 @@ __global__ void __launch_bounds__(320, 1)
     // launch); only the workspace read waits for it.
     griddep_wait();
     {
-      const float4* src = reinterpret_cast<const float4*>(
-          p.ws + ((size_t)bg * p.nspan + j) * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim);
+      // with an in-place final state another CTA of this kernel may write these
+      // addresses later, so no read-only-path loads then
+      const float4* src =
+          p.ws ? reinterpret_cast<const float4*>(p.ws +
+                                                 ((size_t)bg * p.nspan + j) * (kHeadDim * kHeadDim) +
+                                                 (size_t)r * kHeadDim)
+               : nullptr;
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb) {
         const int blk = blk0 + bb;
         uint32_t v[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float4 f = __ldg(src + blk * 8 + i);
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (src) f = kFinal ? src[blk * 8 + i] : __ldg(src + blk * 8 + i);
           v[4 * i + 0] = __float_as_uint(f.x);
           v[4 * i + 1] = __float_as_uint(f.y);
           v[4 * i + 2] = __float_as_uint(f.z);
@@ -331,6 +362,20 @@ __global__ void __launch_bounds__(320, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(sb_full);
+    }
+    // Which CTA of this (batch, kv head) writes the final state.  All 256 math
+    // threads reach these barriers unconditionally.
+    bool writer = false;
+    if constexpr (kFinal) {
+      writer = p.tickets ? false : hs == 0;
+      if (p.tickets) {
+        volatile int* writer_flag = abort_flag + 1;
+        named_barrier_sync(1, 256);  // every entering-state load of this CTA has returned
+        if (warp == 2 && lane == 0)
+          *writer_flag = atom_add_acq_rel_gpu(&p.tickets[bg], 1u) == (unsigned)(p.nsub - 1);
+        named_barrier_sync(1, 256);
+        writer = *writer_flag != 0;
+      }
     }
 
     // half of the bf16 state copy for the next tile's Q S
@@ -356,23 +401,37 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t pcol = 256 + ob * (T / 2);
         if (!warp_wait(a_full, i & 1, p.status, abort_flag)) return false;
         tc_fence_after();
-        uint32_t a[T / 32][32];
+        // 64 score columns per round (a whole 128-column row would take 128
+        // registers and spill).  At T = 128 a 32-column block that lies
+        // entirely on the masked side of this warp's 32 rows is not read at
+        // all (at T = 64 skipping measured slower).  Rounds are not unrolled:
+        // overlapping them would bring the 128 registers back.
+#pragma unroll 1
+        for (int h = 0; h < T / 64; ++h) {
+          uint32_t a[2][32];
+          bool need[2];
 #pragma unroll
-        for (int blk = 0; blk < T / 32; ++blk) tmem_ld32(tmem + lane_base + ocol + blk * 32, a[blk]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int blk = 0; blk < T / 32; ++blk) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const int s0 = blk * 32 + 2 * m;
-            const bool keep0 = reverse ? (s0 >= t_in) : (s0 <= t_in);
-            const bool keep1 = reverse ? (s0 + 1 >= t_in) : (s0 + 1 <= t_in);
-            const float f0 = keep0 ? __uint_as_float(a[blk][2 * m]) : 0.0f;
-            const float f1 = keep1 ? __uint_as_float(a[blk][2 * m + 1]) : 0.0f;
-            pk[m] = pack_bf16x2(f0, f1);
+          for (int bb = 0; bb < 2; ++bb) {
+            const int blk = 2 * h + bb;
+            need[bb] = T == 64 || (reverse ? (blk >= diag_blk) : (blk <= diag_blk));
+            if (need[bb]) tmem_ld32(tmem + lane_base + ocol + blk * 32, a[bb]);
           }
-          tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
+          tmem_wait_ld();
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            const int blk = 2 * h + bb;
+            uint32_t pk[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              const int s0 = blk * 32 + 2 * m;
+              const bool keep0 = need[bb] && (reverse ? (s0 >= t_in) : (s0 <= t_in));
+              const bool keep1 = need[bb] && (reverse ? (s0 + 1 >= t_in) : (s0 + 1 <= t_in));
+              const float f0 = keep0 ? __uint_as_float(a[bb][2 * m]) : 0.0f;
+              const float f1 = keep1 ? __uint_as_float(a[bb][2 * m + 1]) : 0.0f;
+              pk[m] = pack_bf16x2(f0, f1);
+            }
+            tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -436,6 +495,27 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (store_thread) bulk_wait_group<0>();
+    }
+    // final state: entering state + K^T V of every tile, completed by the last
+    // update (s_full completion number ntiles - 1)
+    if (kFinal && ok && ntiles > 0) {
+      if (warp_wait(s_full, (ntiles - 1) & 1, p.status, abort_flag) && writer) {
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
+        tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(p.s_out + (size_t)bg * (kHeadDim * kHeadDim) +
+                                                (size_t)r * kHeadDim + blk0 * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(v0[4 * i]), __uint_as_float(v0[4 * i + 1]),
+                               __uint_as_float(v0[4 * i + 2]), __uint_as_float(v0[4 * i + 3]));
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[8 + i] = make_float4(__uint_as_float(v1[4 * i]), __uint_as_float(v1[4 * i + 1]),
+                                   __uint_as_float(v1[4 * i + 2]), __uint_as_float(v1[4 * i + 3]));
+      }
     }
   }
 
@@ -612,9 +692,12 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
   return cudaGetLastError();
 }
 
+// Launch with programmatic stream serialization when `dependent` (the kernel
+// may start while the previous kernel of the stream finishes; it waits for it
+// before its first dependent read), plainly otherwise.
 template <typename K>
 cudaError_t launch_dependent(K kernel, dim3 grid, int threads, int smem, cudaStream_t stream,
-                             const PrefillMaps& maps, const MainParams& p) {
+                             const PrefillMaps& maps, const MainParams& p, bool dependent) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(threads);
@@ -624,27 +707,37 @@ cudaError_t launch_dependent(K kernel, dim3 grid, int threads, int smem, cudaStr
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = dependent ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, maps.q, maps.k, maps.v, maps.o, p);
+}
+
+template <int T, int QST, int KVST, bool kFinal>
+cudaError_t launch_main(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
+                        const MainParams& p, bool dependent) {
+  using L = MainLayout<T, QST, KVST>;
+  static_assert(L::kBytes <= 232448, "shared memory");
+  cudaError_t e = set_smem(prefill_main_kernel<T, QST, KVST, kFinal>, L::kBytes);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(prefill_main_kernel<T, QST, KVST, kFinal>, grid, 320, L::kBytes, stream,
+                          maps, p, dependent);
 }
 
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
                                 const float* ws, unsigned* status, cudaStream_t stream, int qdiv,
-                                int reverse) {
+                                int reverse, float* s_out, unsigned* tickets) {
   const int nsub = g.G / g.heads_per_tile;
-  MainParams p{ws, status, g.Hq, g.Hkv, g.G, nsub, g.nspan, g.tiles_total, qdiv, reverse};
+  if (s_out && g.nspan != 1) return cudaErrorInvalidValue;
+  if (s_out && s_out == ws && nsub > 1 && !tickets) return cudaErrorInvalidValue;
+  MainParams p{ws,         status,  g.Hq,  g.Hkv, g.G,     nsub,
+               g.nspan,    g.tiles_total, qdiv, reverse, s_out, nsub > 1 ? tickets : nullptr};
   const dim3 grid((unsigned)(g.B * g.Hkv * g.nspan * nsub));
-  cudaError_t e;
-  if (g.tile == 64) {
-    using L = MainLayout<64, 2, 3>;
-    static_assert(L::kBytes <= 232448, "shared memory");
-    if ((e = set_smem(prefill_main_kernel<64, 2, 3>, L::kBytes)) != cudaSuccess) return e;
-    return launch_dependent(prefill_main_kernel<64, 2, 3>, grid, 320, L::kBytes, stream, maps, p);
+  // a standalone launch (final state out) follows no kernel it depends on
+  if (s_out) {
+    if (g.tile == 64) return launch_main<64, 2, 3, true>(grid, stream, maps, p, false);
+    return launch_main<128, 2, 2, true>(grid, stream, maps, p, false);
   }
-  using L = MainLayout<128, 2, 2>;
-  static_assert(L::kBytes <= 232448, "shared memory");
-  if ((e = set_smem(prefill_main_kernel<128, 2, 2>, L::kBytes)) != cudaSuccess) return e;
-  return launch_dependent(prefill_main_kernel<128, 2, 2>, grid, 320, L::kBytes, stream, maps, p);
+  if (g.tile == 64) return launch_main<64, 2, 3, false>(grid, stream, maps, p, true);
+  return launch_main<128, 2, 2, false>(grid, stream, maps, p, true);
 }
 
 }  // namespace la

@@ -122,6 +122,16 @@ __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// *p += v with acquire-release ordering at GPU scope; returns the old value.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
 // Wait until *flag != 0 (acquire, GPU scope), bounded like mbar_wait; every
 // lane of the warp takes the same outcome.
 __device__ __forceinline__ bool warp_wait_flag(const unsigned* flag, unsigned* status,

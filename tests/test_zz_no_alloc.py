@@ -1,7 +1,8 @@
 """la_forward_noalloc: the prefill for callers that cannot allocate device
 memory (allocator callbacks, frameworks that own all device memory, paths that
-must not block in the driver's allocator).  It takes its span-state workspace
-from a fixed device array inside the library.
+must not block in the driver's allocator).  It takes its workspace (span
+states, or the counters of the single-span launch) from a fixed device array
+inside the library.
 
 Checked through the C ABI against la_forward_state, the entry point that
 allocates its workspace, on two calls in a row with different inputs (the
@@ -48,9 +49,20 @@ def test_noalloc_matches_allocating_entry_point(la, B, Hq, Hkv, N, chunk):
     assert la.la_device_status()[0] == 0
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch(la):
+def test_noalloc_one_span_beyond_span_state_limit(la):
+    """1024 kv heads would need 64 MiB of span states (over the 32 MiB
+    array) even at one span each; with one span the call runs as the single
+    chunk-loop launch, which needs only 4 KiB of counters, in place on S."""
     lib = la.api.load_library()
-    # B * Hkv = 1024 kv heads need 64 MiB for a single span each: over the 32 MiB limit.
-    q = torch.zeros(1, 1024, 1, 128, dtype=torch.bfloat16, device=DEV)
-    k, v, o = torch.zeros_like(q), torch.zeros_like(q), torch.empty_like(q)
-    assert _call_noalloc(lib, q, k, v, o, None, 64) == 5  # LA_ERR_WORKSPACE
+    B, Hq, Hkv, N, chunk = 256, 16, 4, 80, 64
+    assert la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).nspan == 1
+    q, k, v = (t.to(DEV) for t in synth.random_qkv(B, Hq, Hkv, N, 128, torch.bfloat16, 203))
+    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(204)) / 128
+    S_ref, S_new = S0.to(DEV), S0.to(DEV)
+    o_ref = la.la_forward_state(q, k, v, S=S_ref, chunk=chunk)
+    o_new = torch.empty_like(q)
+    assert _call_noalloc(lib, q, k, v, o_new, S_new, chunk) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o_new, o_ref)
+    assert torch.equal(S_new, S_ref)
+    assert la.la_device_status()[0] == 0
