@@ -154,18 +154,27 @@ def timed(fn, steps, stream):
     return start.elapsed_time(end) / 1e3, clk.summary()
 
 
+def kernel_source_sha256():
+    """Hash of the chunk-loop kernel's source (its file and the device headers
+    it includes), the key under which ncu figures of it are committed."""
+    csrc = os.path.join(ROOT, "linear_attention_11_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("la_prefill_persist.cu", "la_tile.cuh", "la_ptx.cuh"):
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
 def traffic_from_profile():
-    """DRAM bytes per launch of the main kernel from the committed ncu summary,
-    if the kernel source is unchanged since the capture; else None."""
-    path = os.path.join(ROOT, "profiles", "prefill_main_traffic_gqa_b1_h128kv32.md")
-    src = os.path.join(ROOT, "linear_attention_11_b200", "csrc", "la_prefill.cu")
+    """DRAM bytes per launch of the chunk-loop kernel from the committed ncu
+    summary, if the kernel source is unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "prefill_persist_traffic_gqa_b1_h128kv32.md")
     try:
         fields = {}
         for line in open(path):
             if ":" in line:
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        sha = kernel_source_sha256()
         if fields.get("kernel-source-sha256") == sha:
             return int(fields["traffic-bytes-per-launch"])
     except (OSError, ValueError, KeyError):
@@ -297,7 +306,7 @@ def run_ours(args, w):
     achieved = alg_bytes / t_main / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": (traffic_from_profile() if (w is synth.GQA_32K and chunk == 64) else None),
-                "kernel": "prefill_main_kernel", "launch_ms": t_main * 1e3,
+                "kernel": "prefill_persist_kernel", "launch_ms": t_main * 1e3,
                 "algorithmic_bytes_per_launch": alg_bytes, "peak_source": pk["source"]}
     step_frac = (alg_bytes / (t / args.steps) / 1e9) / pk["hbm_gbs"]
 
@@ -326,7 +335,8 @@ def run_ours(args, w):
         "two_pass_span_parallel_ms": 1e3 * t / args.steps,
         "sequential_chunk_loop_ms": 1e3 * t_seq,
         "single_pass_fused_ms": 1e3 * t_fused,
-        "note": "sequential = one CTA per (batch, kv head, head pair) walking every chunk; "
+        "note": "sequential = one span per (batch, kv head): one CTA walks every chunk of "
+                "the kv group; "
                 "fused = span states and chunk loops in one persistent kernel",
     }
     del ws1, wsf

@@ -86,10 +86,12 @@ int la_version(void);
  * Uses a workspace for the per-span states: la_forward / la_forward_state take
  * it from the device's default stream-ordered memory pool (cudaMallocAsync and
  * cudaFreeAsync on `stream`; the pool keeps the memory cached between calls),
- * la_forward_ws takes one from the caller.  When the plan has one span per
- * (batch, kv head) -- many sequences or heads, short N -- the call is a single
- * chunk-loop launch that reads the initial state and writes the final one
- * itself, and the workspace holds only B * Hkv counters.
+ * la_forward_ws takes one from the caller.  The chunk loop is a persistent
+ * kernel: one CTA per SM walks work items (a span of one (batch, kv head)
+ * sequence with all its query heads).  When the plan has one span per
+ * sequence -- many sequences or kv heads, short N -- the call is that one
+ * launch: it reads the initial state and writes the final one itself, and
+ * needs no workspace (la_forward_workspace_bytes returns a nominal 256).
  *
  * Errors: LA_ERR_INVALID_ARG (null or misaligned pointer, B/Hq/Hkv/N <= 0,
  * Hq % Hkv, o overlapping an input), LA_ERR_UNSUPPORTED (d != 128, chunk not
@@ -174,7 +176,7 @@ la_status la_prefill_fused(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v,
  *   - Limit: the span states (B * Hkv * nspan * d * d * 4 bytes) must fit in
  *     32 MiB; the span count is lowered until they do, down to one span per
  *     (batch, kv head), which runs as the single chunk-loop launch and needs
- *     only B * Hkv * 4 bytes (LA_ERR_WORKSPACE beyond 8M kv heads).
+ *     no workspace, so every problem size is accepted.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls share the array: calls whose work overlaps on the GPU race
@@ -217,7 +219,8 @@ la_status la_prefill_span_states(const la_bf16 *k, const la_bf16 *v, int B, int 
 la_status la_prefill_scan(float *ws, float *S, int B, int Hkv, int d, const la_plan *plan,
                           la_stream stream);
 
-/* Stage 3: O for every span, starting each from ws[b,g,j]. */
+/* Stage 3: O for every span, starting each from ws[b,g,j] (the persistent
+ * chunk loop: min(B * Hkv * nspan, SM count) CTAs walk the spans round-robin). */
 la_status la_prefill_main(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
                           const float *ws, int B, int Hq, int Hkv, int64_t N, int d,
                           const la_plan *plan, la_stream stream);

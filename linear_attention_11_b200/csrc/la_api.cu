@@ -79,19 +79,21 @@ la_status plan_impl(int B, int Hq, int Hkv, int64_t N, int d, int chunk, int sms
     HPT = 1;
   }
   const int64_t tiles = (N + T - 1) / T;
-  const int64_t units = (int64_t)B * Hkv * (G / HPT);
-  // Pick the span count: the main kernel runs units * nspan CTAs, one per SM
-  // at a time; estimated time ~ waves * (tiles per span + a fixed per-CTA cost
-  // of about three tiles).
+  const int64_t units = (int64_t)B * Hkv;
+  const int64_t nsub = G / HPT;
+  // Pick the span count: the persistent chunk loop deals units * nspan items
+  // (a span of one kv group, nsub tiles per chunk step) round-robin over the
+  // SMs; estimated time ~ rounds * (tiles per item + a per-item cost of about
+  // three tiles).
   const int64_t max_span = std::min<int64_t>(tiles, 4096);
   int64_t best = 1;
   double best_cost = 1e300;
   for (int64_t ns = 1; ns <= max_span; ++ns) {
-    const int64_t ctas = units * ns;
-    if (ctas > 0x7fffffff) break;
-    const int64_t waves = (ctas + sms - 1) / sms;
-    const int64_t per = (tiles + ns - 1) / ns;
-    const double cost = (double)waves * (double)(per + 3);
+    const int64_t items = units * ns;
+    if (items > 0x7fffffff) break;
+    const int64_t rounds = (items + sms - 1) / sms;
+    const int64_t per = (tiles + ns - 1) / ns * nsub;
+    const double cost = (double)rounds * (double)(per + 3);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = ns;
@@ -218,17 +220,16 @@ __global__ void selftest_wait_kernel(unsigned* status, const unsigned* flag, int
 
 }  // namespace
 
-size_t forward_workspace_bytes(const la_plan& plan, int B, int Hkv) {
-  if (plan.nspan == 1) return (((size_t)B * Hkv * sizeof(unsigned)) + 255) & ~(size_t)255;
-  return (size_t)plan.workspace_bytes;
+size_t forward_workspace_bytes(const la_plan& plan) {
+  return plan.nspan == 1 ? 256 : (size_t)plan.workspace_bytes;
 }
 
-la_status forward_single_span(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
-                              float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
-                              unsigned* tickets, cudaStream_t stream) {
-  if (plan.nspan != 1) return LA_ERR_INVALID_ARG;
+la_status forward_persistent(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
+                             float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
+                             cudaStream_t stream) {
   unsigned* status = nullptr;
-  if (!device_info(&status, nullptr)) return LA_ERR_CUDA;
+  int sms = 0;
+  if (!device_info(&status, &sms)) return LA_ERR_CUDA;
   PrefillMaps maps;
   if (!make_tmap_bf16(&maps.q, q, N, (int64_t)B * Hq, plan.tile) ||
       !make_tmap_bf16(&maps.o, o, N, (int64_t)B * Hq, plan.tile) ||
@@ -236,14 +237,20 @@ la_status forward_single_span(const la_bf16* q, const la_bf16* k, const la_bf16*
       !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
     return LA_ERR_CUDA;
   PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
-  const bool need_tickets = S && g.G / g.heads_per_tile > 1;
-  if (need_tickets) {
-    if (!tickets) return LA_ERR_WORKSPACE;
-    if (cudaMemsetAsync(tickets, 0, (size_t)B * Hkv * sizeof(unsigned), stream) != cudaSuccess)
-      return LA_ERR_CUDA;
-  }
-  return from_cuda(launch_prefill_main(g, maps, S, status, stream, 1, 0, S,
-                                       need_tickets ? tickets : nullptr));
+  return from_cuda(launch_prefill_persist(g, maps, S, S, status, sms, stream, false));
+}
+
+la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
+                           float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
+                           void* workspace, cudaStream_t stream) {
+  if (plan.nspan == 1) return forward_persistent(q, k, v, o, S, B, Hq, Hkv, N, plan, stream);
+  const la_stream st = static_cast<la_stream>(stream);
+  float* ws = static_cast<float*>(workspace);
+  const int d = kHeadDim;
+  la_status r;
+  if ((r = la_prefill_span_states(k, v, B, Hkv, N, d, &plan, ws, st)) != LA_OK) return r;
+  if ((r = la_prefill_scan(ws, S, B, Hkv, d, &plan, st)) != LA_OK) return r;
+  return la_prefill_main(q, k, v, o, ws, B, Hq, Hkv, N, d, &plan, st);
 }
 
 cudaError_t launch_selftest_wait(unsigned* status, int64_t timeout_ns, cudaStream_t stream) {
@@ -285,7 +292,7 @@ LA_EXPORT la_status la_prefill_plan(int B, int Hq, int Hkv, int64_t N, int d, in
 LA_EXPORT size_t la_forward_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d, int chunk) {
   la_plan p;
   if (la_prefill_plan(B, Hq, Hkv, N, d, chunk, &p) != LA_OK) return 0;
-  return forward_workspace_bytes(p, B, Hkv);
+  return forward_workspace_bytes(p);
 }
 
 LA_EXPORT la_status la_prefill_span_states(const la_bf16* k, const la_bf16* v, int B, int Hkv,
@@ -342,7 +349,10 @@ LA_EXPORT la_status la_prefill_main(const la_bf16* q, const la_bf16* k, const la
       !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan->tile))
     return LA_ERR_CUDA;
   PrefillGeometry g = geometry(plan, B, Hq, Hkv, N);
-  return from_cuda(launch_prefill_main(g, maps, ws, status, static_cast<cudaStream_t>(stream)));
+  int sms = 0;
+  if (!device_info(nullptr, &sms)) return LA_ERR_CUDA;
+  return from_cuda(launch_prefill_persist(g, maps, ws, nullptr, status, sms,
+                                          static_cast<cudaStream_t>(stream), true));
 }
 
 LA_EXPORT size_t la_prefill_fused_workspace_bytes(int B, int Hq, int Hkv, int64_t N, int d,
@@ -400,15 +410,10 @@ LA_EXPORT la_status la_forward_ws(const la_bf16* q, const la_bf16* k, const la_b
   if (st != LA_OK) return st;
   if ((st = check_prefill_ptrs(q, k, v, o, S, B, Hq, Hkv, N, d)) != LA_OK) return st;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      workspace_bytes < forward_workspace_bytes(plan, B, Hkv))
+      workspace_bytes < forward_workspace_bytes(plan))
     return LA_ERR_WORKSPACE;
-  if (plan.nspan == 1)  // one span per (batch, kv head): the chunk loop alone
-    return forward_single_span(q, k, v, o, S, B, Hq, Hkv, N, plan,
-                               static_cast<unsigned*>(workspace), static_cast<cudaStream_t>(stream));
-  float* ws = static_cast<float*>(workspace);
-  if ((st = la_prefill_span_states(k, v, B, Hkv, N, d, &plan, ws, stream)) != LA_OK) return st;
-  if ((st = la_prefill_scan(ws, S, B, Hkv, d, &plan, stream)) != LA_OK) return st;
-  return la_prefill_main(q, k, v, o, ws, B, Hq, Hkv, N, d, &plan, stream);
+  return forward_dispatch(q, k, v, o, S, B, Hq, Hkv, N, plan, workspace,
+                          static_cast<cudaStream_t>(stream));
 }
 
 LA_EXPORT la_status la_forward_state(const la_bf16* q, const la_bf16* k, const la_bf16* v,

@@ -38,28 +38,34 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, i
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
                                cudaStream_t stream);
-// qdiv: query rows of head h come from head h / qdiv of the query tensor map;
-// reverse: anti-causal pass (sum over s >= t), the tiles of every span walked
-// from the end.  The forward pass is qdiv = 1, reverse = 0.  ws == nullptr
-// starts every span from a zero state.  s_out (nspan == 1 only; else
-// cudaErrorInvalidValue): the final state [B*Hkv, d, d] is written there; when
-// s_out is ws itself (in place) and G / heads_per_tile > 1, tickets must point
-// to B*Hkv zeroed counters.
+// Chunk loop with one CTA per (batch, kv head, head subset, span), used by
+// the backward passes.  qdiv: query rows of head h come from head h / qdiv of
+// the query tensor map; reverse: anti-causal pass (sum over s >= t), the
+// tiles of every span walked from the end.
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
                                 const float* ws, unsigned* status, cudaStream_t stream,
-                                int qdiv = 1, int reverse = 0, float* s_out = nullptr,
-                                unsigned* tickets = nullptr);
+                                int qdiv = 1, int reverse = 0);
+// Persistent schedule of the chunk loop: min(B*Hkv*nspan, num_ctas) CTAs walk
+// the items (one span of one (batch, kv head) sequence each, every query head
+// of the group) round-robin.  ws: entering state of item bg * nspan + j
+// (nullptr: zero); s_out (nspan == 1 only): final states [B*Hkv, d, d], may be
+// ws itself.  dependent: launched as a programmatic dependent of the previous
+// kernel in the stream.
+cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
+                                   const float* ws, float* s_out, unsigned* status, int num_ctas,
+                                   cudaStream_t stream, bool dependent);
 size_t fused_workspace_bytes(int B, int Hkv, int nspan);
-// The whole bf16 prefill of a plan with nspan == 1 as one chunk-loop launch
-// that reads S (nullable: zero) and writes the final state back into it.
-// `tickets`: device memory for B*Hkv counters (zeroed here), needed when S is
-// given and a kv group spans several CTAs.  Arguments already validated.
-la_status forward_single_span(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
-                              float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
-                              unsigned* tickets, cudaStream_t stream);
-// Workspace bytes la_forward_ws needs for `plan`: the span states, or only
-// the tickets of the single-span launch.
-size_t forward_workspace_bytes(const la_plan& plan, int B, int Hkv);
+// Workspace bytes la_forward_ws needs for `plan` (never zero): the span
+// states, or nothing (a nominal 256 bytes) with one span per sequence, which
+// runs as the persistent chunk loop alone with the state read and written in
+// place.
+size_t forward_workspace_bytes(const la_plan& plan);
+// The whole prefill (validated arguments): one persistent chunk-loop launch
+// when the plan has one span per sequence, else span states, scan and the
+// persistent chunk loop; workspace of forward_workspace_bytes bytes.
+la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
+                           float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
+                           void* workspace, cudaStream_t stream);
 cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
                                  void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);

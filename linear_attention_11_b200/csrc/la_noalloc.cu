@@ -74,21 +74,14 @@ LA_EXPORT la_status la_forward_noalloc(const la_bf16* q, const la_bf16* k, const
       overlap(S, sbytes, v, kbytes))
     return LA_ERR_INVALID_ARG;
   // Fewer spans if the planned span states exceed the array; a single span
-  // needs only the counters of the one-launch path (B * Hkv * 4 bytes).
+  // needs none (the chunk loop reads and writes the state itself).
   const int64_t per_span = (int64_t)B * Hkv * d * d * (int64_t)sizeof(float);
   if (plan.nspan > 1 && plan.workspace_bytes > (int64_t)kScratchBytes) {
     plan.nspan = (int32_t)std::max<int64_t>(1, (int64_t)kScratchBytes / per_span);
     plan.workspace_bytes = per_span * plan.nspan;
   }
-  float* ws = static_cast<float*>(scratch_on_current_device());
+  void* ws = scratch_on_current_device();
   if (!ws) return LA_ERR_CUDA;
-  if (plan.nspan == 1) {
-    if (la::forward_workspace_bytes(plan, B, Hkv) > kScratchBytes) return LA_ERR_WORKSPACE;
-    return la::forward_single_span(q, k, v, o, S, B, Hq, Hkv, N, plan,
-                                   reinterpret_cast<unsigned*>(ws),
-                                   static_cast<cudaStream_t>(stream));
-  }
-  if ((st = la_prefill_span_states(k, v, B, Hkv, N, d, &plan, ws, stream)) != LA_OK) return st;
-  if ((st = la_prefill_scan(ws, S, B, Hkv, d, &plan, stream)) != LA_OK) return st;
-  return la_prefill_main(q, k, v, o, ws, B, Hq, Hkv, N, d, &plan, stream);
+  return la::forward_dispatch(q, k, v, o, S, B, Hq, Hkv, N, plan, ws,
+                              static_cast<cudaStream_t>(stream));
 }

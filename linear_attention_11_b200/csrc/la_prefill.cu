@@ -13,11 +13,10 @@
 //                        K^T V = sum of K_c^T V_c over its chunks (fp32).
 //   prefill_main_kernel  one CTA per (batch, kv head, head subset, span): the
 //                        chunk loop of [VGX] over the span, starting from the
-//                        state that enters it (prepared by the scan kernel).
-//                        With one span per (batch, kv head) it can also run
-//                        alone: it reads the initial state itself and writes
-//                        the final one from tensor memory after the last
-//                        chunk's update (no span-state or scan kernel).
+//                        state that enters it (prepared by the scan kernel),
+//                        causal or anti-causal; the backward passes run it.
+//                        The forward prefill runs the persistent schedule of
+//                        the same tile arithmetic (la_prefill_persist.cu).
 //
 // Main-kernel tile: 128 rows = HPT query heads of one kv group x T tokens
 // (T = 64, HPT = 2 or T = 128, HPT = 1); d = 128.  Per tile c:
@@ -54,48 +53,14 @@ namespace la {
 namespace {
 
 struct MainParams {
-  const float* ws;  // state entering span j of unit bg at ws[bg * nspan + j]; nullptr: zero
+  const float* ws;
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total;
   int qdiv;     // query rows of head h come from head h / qdiv of the query tensor
   int reverse;  // 1: anti-causal (s >= t), tiles of a span walked from the end
-  // Final state (nspan == 1 only): after the last tile the state in tensor
-  // memory is entering state + K^T V of the whole sequence, and one CTA of
-  // each (batch, kv head) writes it to s_out[bg].  s_out may be the ws array
-  // itself (in place): then `tickets` (nsub > 1) holds one zeroed counter per
-  // bg; every CTA takes a ticket after reading its entering state, and the
-  // one that draws the last ticket -- all its siblings have read by then --
-  // writes.  Without tickets the head subset 0 writes.
-  float* s_out;
-  unsigned* tickets;
 };
 
-// Shared memory of the main kernel: a ring of Q tiles, a separate ring of K/V
-// tiles, the bf16 state copy, and (at T = 64) a dedicated output staging tile.
-// Q(i) is released once Q(i) S has been issued and completed; K/V(i) once the
-// state update of tile i has; so copies of later tiles start early and more
-// bytes stay in flight.  At T = 128 there is no room for a separate staging
-// tile and the output goes through the Q slot (released after its store has
-// read it).
 template <int T, int QST, int KVST>
-struct MainLayout {
-  static constexpr bool kDedicatedO = (T == 64);
-  static constexpr int kKBytes = T * kHeadDim * 2;
-  static constexpr int kKVBytes = 2 * kKBytes;
-  static constexpr int kKVOff = QST * kQBytes;
-  static constexpr int kSOff = kKVOff + KVST * kKVBytes;
-  static constexpr int kOOff = kSOff + kSBytes;
-  static constexpr int kBarOff = kOOff + (kDedicatedO ? kQBytes : 0);
-  // q_full[QST], q_empty[QST], kv_full[KVST], kv_empty[KVST], a_full, p_full,
-  // o_full[2], o_empty[2], s_full, sb_full, mma_done, store_ready, ostage_free
-  static constexpr int kNumBars = 2 * QST + 2 * KVST + 11;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
-};
-
-// kFinal: the final state is written (MainParams::s_out); a separate
-// instantiation, so the staged kernel carries none of that code.
-template <int T, int QST, int KVST, bool kFinal>
 __global__ void __launch_bounds__(320, 1)
     prefill_main_kernel(const __grid_constant__ CUtensorMap map_q,
                         const __grid_constant__ CUtensorMap map_k,
@@ -299,15 +264,6 @@ __global__ void __launch_bounds__(320, 1)
           mma_commit(&kv_empty[i % KVST]);
           if (!kLookahead && !issue_qk(i + 1)) break;
         } else {
-          if constexpr (kFinal) {  // the last chunk's update completes the final state
-#pragma unroll
-            for (int kk = 0; kk < T / 16; ++kk) {
-              const uint64_t da = smem_desc_sw128(k_addr + kk * 2048, T * 128, 1024);
-              const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
-              mma_ss(tmem + kColS, da, db, IDESC_KV, 1u);
-            }
-            mma_commit(s_full);
-          }
           mma_commit(&kv_empty[i % KVST]);
         }
       }
@@ -335,21 +291,15 @@ __global__ void __launch_bounds__(320, 1)
     // launch); only the workspace read waits for it.
     griddep_wait();
     {
-      // with an in-place final state another CTA of this kernel may write these
-      // addresses later, so no read-only-path loads then
-      const float4* src =
-          p.ws ? reinterpret_cast<const float4*>(p.ws +
-                                                 ((size_t)bg * p.nspan + j) * (kHeadDim * kHeadDim) +
-                                                 (size_t)r * kHeadDim)
-               : nullptr;
+      const float4* src = reinterpret_cast<const float4*>(
+          p.ws + ((size_t)bg * p.nspan + j) * (kHeadDim * kHeadDim) + (size_t)r * kHeadDim);
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb) {
         const int blk = blk0 + bb;
         uint32_t v[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (src) f = kFinal ? src[blk * 8 + i] : __ldg(src + blk * 8 + i);
+          const float4 f = __ldg(src + blk * 8 + i);
           v[4 * i + 0] = __float_as_uint(f.x);
           v[4 * i + 1] = __float_as_uint(f.y);
           v[4 * i + 2] = __float_as_uint(f.z);
@@ -362,20 +312,6 @@ __global__ void __launch_bounds__(320, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(sb_full);
-    }
-    // Which CTA of this (batch, kv head) writes the final state.  All 256 math
-    // threads reach these barriers unconditionally.
-    bool writer = false;
-    if constexpr (kFinal) {
-      writer = p.tickets ? false : hs == 0;
-      if (p.tickets) {
-        volatile int* writer_flag = abort_flag + 1;
-        named_barrier_sync(1, 256);  // every entering-state load of this CTA has returned
-        if (warp == 2 && lane == 0)
-          *writer_flag = atom_add_acq_rel_gpu(&p.tickets[bg], 1u) == (unsigned)(p.nsub - 1);
-        named_barrier_sync(1, 256);
-        writer = *writer_flag != 0;
-      }
     }
 
     // half of the bf16 state copy for the next tile's Q S
@@ -495,27 +431,6 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (store_thread) bulk_wait_group<0>();
-    }
-    // final state: entering state + K^T V of every tile, completed by the last
-    // update (s_full completion number ntiles - 1)
-    if (kFinal && ok && ntiles > 0) {
-      if (warp_wait(s_full, (ntiles - 1) & 1, p.status, abort_flag) && writer) {
-        tc_fence_after();
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
-        tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
-        tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(p.s_out + (size_t)bg * (kHeadDim * kHeadDim) +
-                                                (size_t)r * kHeadDim + blk0 * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(v0[4 * i]), __uint_as_float(v0[4 * i + 1]),
-                               __uint_as_float(v0[4 * i + 2]), __uint_as_float(v0[4 * i + 3]));
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[8 + i] = make_float4(__uint_as_float(v1[4 * i]), __uint_as_float(v1[4 * i + 1]),
-                                   __uint_as_float(v1[4 * i + 2]), __uint_as_float(v1[4 * i + 3]));
-      }
     }
   }
 
@@ -692,12 +607,9 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
   return cudaGetLastError();
 }
 
-// Launch with programmatic stream serialization when `dependent` (the kernel
-// may start while the previous kernel of the stream finishes; it waits for it
-// before its first dependent read), plainly otherwise.
 template <typename K>
 cudaError_t launch_dependent(K kernel, dim3 grid, int threads, int smem, cudaStream_t stream,
-                             const PrefillMaps& maps, const MainParams& p, bool dependent) {
+                             const PrefillMaps& maps, const MainParams& p) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(threads);
@@ -707,37 +619,27 @@ cudaError_t launch_dependent(K kernel, dim3 grid, int threads, int smem, cudaStr
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = dependent ? 1 : 0;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, maps.q, maps.k, maps.v, maps.o, p);
-}
-
-template <int T, int QST, int KVST, bool kFinal>
-cudaError_t launch_main(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
-                        const MainParams& p, bool dependent) {
-  using L = MainLayout<T, QST, KVST>;
-  static_assert(L::kBytes <= 232448, "shared memory");
-  cudaError_t e = set_smem(prefill_main_kernel<T, QST, KVST, kFinal>, L::kBytes);
-  if (e != cudaSuccess) return e;
-  return launch_dependent(prefill_main_kernel<T, QST, KVST, kFinal>, grid, 320, L::kBytes, stream,
-                          maps, p, dependent);
 }
 
 cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
                                 const float* ws, unsigned* status, cudaStream_t stream, int qdiv,
-                                int reverse, float* s_out, unsigned* tickets) {
+                                int reverse) {
   const int nsub = g.G / g.heads_per_tile;
-  if (s_out && g.nspan != 1) return cudaErrorInvalidValue;
-  if (s_out && s_out == ws && nsub > 1 && !tickets) return cudaErrorInvalidValue;
-  MainParams p{ws,         status,  g.Hq,  g.Hkv, g.G,     nsub,
-               g.nspan,    g.tiles_total, qdiv, reverse, s_out, nsub > 1 ? tickets : nullptr};
+  MainParams p{ws, status, g.Hq, g.Hkv, g.G, nsub, g.nspan, g.tiles_total, qdiv, reverse};
   const dim3 grid((unsigned)(g.B * g.Hkv * g.nspan * nsub));
-  // a standalone launch (final state out) follows no kernel it depends on
-  if (s_out) {
-    if (g.tile == 64) return launch_main<64, 2, 3, true>(grid, stream, maps, p, false);
-    return launch_main<128, 2, 2, true>(grid, stream, maps, p, false);
+  cudaError_t e;
+  if (g.tile == 64) {
+    using L = MainLayout<64, 2, 3>;
+    static_assert(L::kBytes <= 232448, "shared memory");
+    if ((e = set_smem(prefill_main_kernel<64, 2, 3>, L::kBytes)) != cudaSuccess) return e;
+    return launch_dependent(prefill_main_kernel<64, 2, 3>, grid, 320, L::kBytes, stream, maps, p);
   }
-  if (g.tile == 64) return launch_main<64, 2, 3, false>(grid, stream, maps, p, true);
-  return launch_main<128, 2, 2, false>(grid, stream, maps, p, true);
+  using L = MainLayout<128, 2, 2>;
+  static_assert(L::kBytes <= 232448, "shared memory");
+  if ((e = set_smem(prefill_main_kernel<128, 2, 2>, L::kBytes)) != cudaSuccess) return e;
+  return launch_dependent(prefill_main_kernel<128, 2, 2>, grid, 320, L::kBytes, stream, maps, p);
 }
 
 }  // namespace la

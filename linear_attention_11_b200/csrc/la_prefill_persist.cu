@@ -1,0 +1,549 @@
+// la_prefill_persist.cu -- persistent schedule of the chunk-loop kernel.
+//
+// Per 128-row tile the arithmetic is that of prefill_main_kernel (the causal
+// chunk form of "如何理解MiniMax股价创历史新高？拆解国产大模型技术底座", section
+// "Lightning Attention：长上下文为什么突然变得便宜了": O_c = Q_c S + tril(Q_c
+// K_c^T) V_c, then S += K_c^T V_c; grouped kv heads as in "MiniMax-01与
+// Lightning Attention", section 1.1).  What differs is the schedule:
+//   - one CTA per SM walks a list of work items, item = one span of one
+//     (batch, kv head) sequence, items dealt round-robin; the copy, MMA and
+//     math pipelines run on across item boundaries, so the fill of one item
+//     overlaps the drain of the one before;
+//   - an item covers every query head of its kv group: per chunk step the
+//     group's G / HPT tiles (HPT heads each) share one K/V tile and one state,
+//     and the state update follows the last of them;
+//   - the math warps read each item's entering state at the item boundary
+//     (span-state workspace, caller's initial state, or zero), prefetched into
+//     L2 one item ahead; with one span per sequence the CTA that owns the
+//     whole sequence writes the final state (tensor memory after the last
+//     chunk's update) at the item's end, in place if asked.
+//
+// Roles (320 threads) and tensor memory as in prefill_main_kernel: warp 0
+// lane 0 streams Q tiles, lane 1 K/V tiles (and the L2 prefetch); warp 1
+// issues the MMAs; warps 2-5 mask score tiles, warps 6-9 store output tiles;
+// both warpgroups handle half of the state columns.  TMEM: O buffers at
+// columns 0 and 128 (score tiles first), P at 256, state at 384.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "la_internal.h"
+#include "la_ptx.cuh"
+#include "la_tile.cuh"
+
+namespace la {
+namespace {
+
+struct PersistParams {
+  const float* ws;  // entering state of item it at ws[it] (d x d fp32 each); nullptr: zero
+  float* s_out;     // one span per sequence: final state of sequence bg at s_out[bg]
+  unsigned* status;
+  int Hq, Hkv, G, nsub, nspan, tiles_total, items;
+};
+
+template <int T, int QST, int KVST>
+__global__ void __launch_bounds__(320, 1)
+    prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
+                           const __grid_constant__ CUtensorMap map_k,
+                           const __grid_constant__ CUtensorMap map_v,
+                           const __grid_constant__ CUtensorMap map_o, const PersistParams p) {
+  using L = MainLayout<T, QST, KVST>;
+  constexpr int HPT = kTileRows / T;
+  constexpr bool kDedicatedO = L::kDedicatedO;
+  constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, T, 0, 0);
+  constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, 0, 1);
+  constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
+  constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, 1, 1);
+  constexpr bool kLookahead = KVST >= 3;
+  constexpr int kDD = kHeadDim * kHeadDim;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sm = smem_raw + (base - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = q_full + QST;
+  uint64_t* kv_full = q_empty + QST;
+  uint64_t* kv_empty = kv_full + KVST;
+  uint64_t* a_full = kv_empty + KVST;
+  uint64_t* p_full = a_full + 1;
+  uint64_t* o_full = p_full + 1;    // two: tile i completes o_full[i & 1]
+  uint64_t* o_empty = o_full + 2;   // two
+  uint64_t* s_full = o_empty + 2;   // one completion per chunk step (state update)
+  uint64_t* sb_full = s_full + 1;   // one completion per state version (bf16 copy ready)
+  uint64_t* mma_done = sb_full + 1;
+  uint64_t* store_ready = mma_done + 1;
+  uint64_t* ostage_free = store_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
+
+  const uint32_t sS = base + L::kSOff;
+  auto sQ = [&](int i) { return base + (uint32_t)((i % QST) * kQBytes); };
+  auto sK = [&](int c) { return base + (uint32_t)(L::kKVOff + (c % KVST) * L::kKVBytes); };
+  auto sV = [&](int c) { return sK(c) + (uint32_t)L::kKBytes; };
+  auto sO = [&](int i) { return kDedicatedO ? base + (uint32_t)L::kOOff : sQ(i); };
+
+  // item it: sequence bg = it / nspan, chunk steps [tb, te) of span it % nspan
+  auto span_of = [&](int it, int& bg, int& tb, int& te) {
+    const int j = it % p.nspan;
+    bg = it / p.nspan;
+    tb = (int)(((int64_t)j * p.tiles_total) / p.nspan);
+    te = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
+  };
+  const int stride = (int)gridDim.x;
+  auto next_item = [&](int it) { return it + stride < p.items ? it + stride : -1; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < QST; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], kDedicatedO ? 1 : 2);  // MMA commit (+ output-store release)
+    }
+    for (int i = 0; i < KVST; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(a_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(&o_full[0], 1);
+    mbar_init(&o_full[1], 1);
+    mbar_init(&o_empty[0], 128);
+    mbar_init(&o_empty[1], 128);
+    mbar_init(s_full, 1);
+    mbar_init(sb_full, 256);
+    mbar_init(mma_done, 1);
+    mbar_init(store_ready, 128);
+    mbar_init(ostage_free, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ copies
+    if (lane == 0) {
+      prefetch_tmap(&map_q);
+      prefetch_tmap(&map_o);
+      const uint64_t pol_q = policy_evict_first();
+      int i = 0;
+      bool go = true;
+      for (int it = blockIdx.x; it < p.items && go; it += stride) {
+        int bg, tb, te;
+        span_of(it, bg, tb, te);
+        const int b = bg / p.Hkv, g = bg % p.Hkv;
+        for (int cs = tb; cs < te && go; ++cs) {
+          for (int hs = 0; hs < p.nsub; ++hs, ++i) {
+            const int s = i % QST;
+            if (i >= QST && !mbar_wait(&q_empty[s], ((i / QST) - 1) & 1, p.status, abort_flag)) {
+              go = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&q_full[s], kQBytes);
+            uint8_t* q_dst = sm + (sQ(i) - base);
+#pragma unroll
+            for (int hh = 0; hh < HPT; ++hh) {
+              const int qh = b * p.Hq + g * p.G + hs * HPT + hh;
+              tma_load_3d(q_dst + hh * T * 128, &map_q, &q_full[s], 0, cs * T, qh, pol_q);
+              tma_load_3d(q_dst + kHalf + hh * T * 128, &map_q, &q_full[s], 64, cs * T, qh,
+                          pol_q);
+            }
+          }
+        }
+      }
+      if (*abort_flag) {  // let copies already issued land before the block exits
+        for (int k = (i > QST ? i - QST : 0); k < i; ++k) mbar_wait_drain(&q_full[k % QST], (k / QST) & 1);
+      }
+    } else if (lane == 1) {
+      prefetch_tmap(&map_k);
+      prefetch_tmap(&map_v);
+      const uint64_t pol_kv = policy_evict_first();
+      int gc = 0;
+      bool go = true;
+      for (int it = blockIdx.x; it < p.items && go; it += stride) {
+        int bg, tb, te;
+        span_of(it, bg, tb, te);
+        const int nx = next_item(it);
+        if (p.ws && nx >= 0)  // the next item's entering state, read at this item's end
+          prefetch_l2_bulk(p.ws + (size_t)nx * kDD, (uint32_t)(kDD * sizeof(float)));
+        for (int cs = tb; cs < te; ++cs, ++gc) {
+          const int s = gc % KVST;
+          if (gc >= KVST && !mbar_wait(&kv_empty[s], ((gc / KVST) - 1) & 1, p.status, abort_flag)) {
+            go = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[s], L::kKVBytes);
+          uint8_t* k_dst = sm + (sK(gc) - base);
+          uint8_t* v_dst = sm + (sV(gc) - base);
+          tma_load_3d(k_dst, &map_k, &kv_full[s], 0, cs * T, bg, pol_kv);
+          tma_load_3d(k_dst + T * 128, &map_k, &kv_full[s], 64, cs * T, bg, pol_kv);
+          tma_load_3d(v_dst, &map_v, &kv_full[s], 0, cs * T, bg, pol_kv);
+          tma_load_3d(v_dst + T * 128, &map_v, &kv_full[s], 64, cs * T, bg, pol_kv);
+        }
+      }
+      if (*abort_flag) {
+        for (int k = (gc > KVST ? gc - KVST : 0); k < gc; ++k)
+          mbar_wait_drain(&kv_full[k % KVST], (k / KVST) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // Per tile i (chunk step gc, head subset hs): QS(i) PV(i); then, inside a
+    // chunk step, QK(i+1); after the last head subset, QK(i+1) and the state
+    // update KV(gc) in the order of prefill_main_kernel (update first without
+    // a third K/V slot).  Every item ends with its update, so the state in
+    // tensor memory is final there.
+    if (elect_one()) {
+      auto issue_qk = [&](int i, int gci) -> bool {
+        const uint32_t ob = (uint32_t)(i & 1);
+        if (!mbar_wait(&q_full[i % QST], (i / QST) & 1, p.status, abort_flag)) return false;
+        if (!mbar_wait(&kv_full[gci % KVST], (gci / KVST) & 1, p.status, abort_flag)) return false;
+        if (i >= 2 && !mbar_wait(&o_empty[ob], ((i >> 1) - 1) & 1, p.status, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t q_addr = sQ(i), k_addr = sK(gci);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // A = Q K^T, both K-major
+          const uint32_t koff = (uint32_t)((kk & 3) * 32);
+          const uint64_t da = smem_desc_sw128(q_addr + (kk >> 2) * kHalf + koff, 16, 1024);
+          const uint64_t db = smem_desc_sw128(k_addr + (kk >> 2) * (T * 128) + koff, 16, 1024);
+          mma_ss(tmem + ob * 128, da, db, IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(a_full);
+        return true;
+      };
+      auto issue_kv = [&](int gci) {
+        const uint32_t k_addr = sK(gci), v_addr = sV(gci);
+#pragma unroll
+        for (int kk = 0; kk < T / 16; ++kk) {  // S += K^T V (both MN-major)
+          const uint64_t da = smem_desc_sw128(k_addr + kk * 2048, T * 128, 1024);
+          const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
+          mma_ss(tmem + kColS, da, db, IDESC_KV, 1u);
+        }
+        mma_commit(s_full);
+        mma_commit(&kv_empty[gci % KVST]);
+      };
+      int i = 0, gc = 0;
+      bool ok = issue_qk(0, 0);
+      for (int it = blockIdx.x; it < p.items && ok; it += stride) {
+        int bg, tb, te;
+        span_of(it, bg, tb, te);
+        const bool last_item = next_item(it) < 0;
+        for (int cs = tb; cs < te && ok; ++cs) {
+          for (int hs = 0; hs < p.nsub && ok; ++hs) {
+            const uint32_t ob = (uint32_t)(i & 1);
+            const uint32_t ocol = ob * 128;
+            const uint32_t pcol = 256 + ob * (T / 2);
+            if (!mbar_wait(p_full, i & 1, p.status, abort_flag)) { ok = false; break; }
+            if (hs == 0 && !mbar_wait(sb_full, gc & 1, p.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t q_addr = sQ(i), v_addr = sV(gc);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {  // O = Q S (S: MN-major, 16 key rows per k-step)
+              const uint64_t da =
+                  smem_desc_sw128(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+              const uint64_t db = smem_desc_sw128(sS + kk * 2048, kHalf, 1024);
+              mma_ss(tmem + ocol, da, db, IDESC_QS, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < T / 16; ++kk) {  // O += P V (P from TMEM)
+              const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
+              mma_ts(tmem + ocol, tmem + pcol + kk * 8, db, IDESC_PV, 1u);
+            }
+            mma_commit(&o_full[ob]);
+            mma_commit(&q_empty[i % QST]);
+            const bool last_hs = hs == p.nsub - 1;
+            const bool item_end = last_hs && cs == te - 1;
+            const bool has_next = !(last_item && item_end);
+            // the next tile's scores before the update only inside an item: at
+            // an item's end the update goes first, so the state hand-over to
+            // the next item does not wait for that item's first Q tile
+            const bool qk_first = kLookahead && !item_end;
+            if (!last_hs) {
+              if (!issue_qk(i + 1, gc)) ok = false;
+            } else {
+              if (qk_first && !issue_qk(i + 1, gc + 1)) ok = false;
+              if (ok) issue_kv(gc);
+              if (ok && !qk_first && has_next && !issue_qk(i + 1, gc + 1)) ok = false;
+              ++gc;
+            }
+            ++i;
+          }
+        }
+      }
+      mma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ math warpgroups
+    const bool wg1 = warp < 6;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // TMEM lane = tile row = state row
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int t_in = r % T;
+    const int diag_blk = t_in / 32;
+    const int blk0 = wg1 ? 0 : 2;  // state column blocks this warpgroup handles
+    const bool store_thread = (warp == 6 && lane == 0);
+    bool ok = true;
+
+    // This warpgroup's half of row r of item it's entering state -> tensor
+    // memory and the bf16 copy; then signal the state version.
+    auto load_state = [&](int it) {
+      const float4* src =
+          p.ws ? reinterpret_cast<const float4*>(p.ws + (size_t)it * kDD + (size_t)r * kHeadDim)
+               : nullptr;
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb) {
+        const int blk = blk0 + bb;
+        uint32_t v[32];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (src) f = src[blk * 8 + m];  // plain loads: the state may be updated in place
+          v[4 * m + 0] = __float_as_uint(f.x);
+          v[4 * m + 1] = __float_as_uint(f.y);
+          v[4 * m + 2] = __float_as_uint(f.z);
+          v[4 * m + 3] = __float_as_uint(f.w);
+        }
+        tmem_st32(tmem + lane_base + kColS + blk * 32, v);
+        store_row32_sw128(sS, r, blk, v);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(sb_full);
+    };
+
+    // After the update of chunk step gc: within an item, the bf16 copy for
+    // the next chunk step; at an item's end, the final state out (one span per
+    // sequence) and the next item's entering state in.
+    auto state_step = [&](int gc, bool item_end, int bg, int nx) -> bool {
+      if (!warp_wait(s_full, gc & 1, p.status, abort_flag)) return false;
+      tc_fence_after();
+      if (!item_end) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
+        tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
+        tmem_wait_ld();
+        store_row32_sw128(sS, r, blk0, v0);
+        store_row32_sw128(sS, r, blk0 + 1, v1);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(sb_full);
+        return true;
+      }
+      if (p.s_out) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
+        tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(p.s_out + (size_t)bg * kDD + (size_t)r * kHeadDim +
+                                                blk0 * 32);
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          dst[m] = make_float4(__uint_as_float(v0[4 * m]), __uint_as_float(v0[4 * m + 1]),
+                               __uint_as_float(v0[4 * m + 2]), __uint_as_float(v0[4 * m + 3]));
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          dst[8 + m] = make_float4(__uint_as_float(v1[4 * m]), __uint_as_float(v1[4 * m + 1]),
+                                   __uint_as_float(v1[4 * m + 2]), __uint_as_float(v1[4 * m + 3]));
+      }
+      if (nx >= 0) load_state(nx);
+      return true;
+    };
+
+    // The kernel may start before the kernel writing the entering states has
+    // finished (programmatic dependent launch): wait before the first read.
+    griddep_wait();
+    load_state(blockIdx.x);
+
+    if (wg1) {
+      auto mask_tile = [&](int i) -> bool {
+        const uint32_t ob = (uint32_t)(i & 1);
+        const uint32_t ocol = ob * 128;
+        const uint32_t pcol = 256 + ob * (T / 2);
+        if (!warp_wait(a_full, i & 1, p.status, abort_flag)) return false;
+        tc_fence_after();
+        // 64 score columns per round; at T = 128 blocks entirely above the
+        // diagonal of this warp's rows are not read
+#pragma unroll 1
+        for (int h = 0; h < T / 64; ++h) {
+          uint32_t a[2][32];
+          bool need[2];
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            const int blk = 2 * h + bb;
+            need[bb] = T == 64 || blk <= diag_blk;
+            if (need[bb]) tmem_ld32(tmem + lane_base + ocol + blk * 32, a[bb]);
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            const int blk = 2 * h + bb;
+            uint32_t pk[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              const int s0 = blk * 32 + 2 * m;
+              const float f0 = need[bb] && s0 <= t_in ? __uint_as_float(a[bb][2 * m]) : 0.0f;
+              const float f1 = need[bb] && s0 + 1 <= t_in ? __uint_as_float(a[bb][2 * m + 1]) : 0.0f;
+              pk[m] = pack_bf16x2(f0, f1);
+            }
+            tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        return true;
+      };
+      ok = mask_tile(0);
+      int i = 0, gc = 0;
+      for (int it = blockIdx.x; it < p.items && ok; it += stride) {
+        int bg, tb, te;
+        span_of(it, bg, tb, te);
+        const int nx = next_item(it);
+        for (int cs = tb; cs < te && ok; ++cs) {
+          for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
+            const bool last_hs = hs == p.nsub - 1;
+            const bool item_end = last_hs && cs == te - 1;
+            const bool has_next = !(item_end && nx < 0);
+            // the MMA order decides which of the two is ready first; one call
+            // site each (two inlined copies of either spill registers at T = 128)
+            const bool step_first = last_hs && (!kLookahead || item_end);
+#pragma unroll 1
+            for (int ph = 0; ph < 2 && ok; ++ph) {
+              const bool do_step = last_hs && (ph == (step_first ? 0 : 1));
+              const bool do_mask = has_next && (ph == (step_first ? 1 : 0));
+              if (do_mask && !mask_tile(i + 1)) ok = false;
+              if (ok && do_step && !state_step(gc, item_end, bg, nx)) ok = false;
+            }
+            if (!ok) break;
+            if (last_hs) ++gc;
+          }
+        }
+      }
+    } else {
+      int i = 0, gc = 0;
+      for (int it = blockIdx.x; it < p.items && ok; it += stride) {
+        int bg, tb, te;
+        span_of(it, bg, tb, te);
+        const int b = bg / p.Hkv, g = bg % p.Hkv;
+        const int nx = next_item(it);
+        for (int cs = tb; cs < te && ok; ++cs) {
+          for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
+            const bool last_hs = hs == p.nsub - 1;
+            const bool item_end = last_hs && cs == te - 1;
+            if (last_hs && !state_step(gc, item_end, bg, nx)) { ok = false; break; }
+            if (last_hs) ++gc;
+            // output epilogue: TMEM -> bf16 -> staging tile -> bulk store
+            const uint32_t ob = (uint32_t)(i & 1);
+            const uint32_t ocol = ob * 128;
+            if (!warp_wait(&o_full[ob], (i >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+            if (kDedicatedO && i > 0 &&
+                !warp_wait(ostage_free, (i - 1) & 1, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t stage_o = sO(i);
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+              uint32_t v0[32], v1[32];
+              tmem_ld32(tmem + lane_base + ocol + (2 * bb) * 32, v0);
+              tmem_ld32(tmem + lane_base + ocol + (2 * bb + 1) * 32, v1);
+              tmem_wait_ld();
+              store_row32_sw128(stage_o, r, 2 * bb, v0);
+              store_row32_sw128(stage_o, r, 2 * bb + 1, v1);
+            }
+            tc_fence_before();
+            mbar_arrive(&o_empty[ob]);
+            fence_proxy_async_smem();
+            mbar_arrive(store_ready);
+            if (warp == 6) {
+              if (!warp_wait(store_ready, i & 1, p.status, abort_flag)) { ok = false; break; }
+            }
+            if (store_thread) {
+              const uint8_t* src = sm + (stage_o - base);
+#pragma unroll
+              for (int hh = 0; hh < HPT; ++hh) {
+                const int oh = b * p.Hq + g * p.G + hs * HPT + hh;
+                tma_store_3d(&map_o, src + hh * T * 128, 0, cs * T, oh);
+                tma_store_3d(&map_o, src + kHalf + hh * T * 128, 64, cs * T, oh);
+              }
+              bulk_commit_group();
+              bulk_wait_group_read<0>();  // the store has read the staging tile
+              if (kDedicatedO)
+                mbar_arrive(ostage_free);
+              else
+                mbar_arrive(&q_empty[i % QST]);
+            }
+          }
+        }
+      }
+      if (store_thread) bulk_wait_group<0>();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int T, int QST, int KVST>
+cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
+                           const PersistParams& p, bool dependent) {
+  using L = MainLayout<T, QST, KVST>;
+  static_assert(L::kBytes <= 232448, "shared memory");
+  cudaError_t e = set_smem(prefill_persist_kernel<T, QST, KVST>, L::kBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(320);
+  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, prefill_persist_kernel<T, QST, KVST>, maps.q, maps.k, maps.v,
+                            maps.o, p);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
+                                   const float* ws, float* s_out, unsigned* status, int num_ctas,
+                                   cudaStream_t stream, bool dependent) {
+  if (s_out && g.nspan != 1) return cudaErrorInvalidValue;
+  const int nsub = g.G / g.heads_per_tile;
+  const int64_t items = (int64_t)g.B * g.Hkv * g.nspan;
+  if (items <= 0 || items > 0x7fffffff || num_ctas <= 0) return cudaErrorInvalidValue;
+  PersistParams p{ws,    s_out, status, g.Hq,          g.Hkv,
+                  g.G,   nsub,  g.nspan, g.tiles_total, (int)items};
+  const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
+  if (g.tile == 64) return launch_persist<64, 3, 2>(grid, stream, maps, p, dependent);
+  return launch_persist<128, 2, 2>(grid, stream, maps, p, dependent);
+}
+
+}  // namespace la

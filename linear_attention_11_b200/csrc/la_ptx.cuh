@@ -122,16 +122,6 @@ __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// *p += v with acquire-release ordering at GPU scope; returns the old value.
-__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
-
 // Wait until *flag != 0 (acquire, GPU scope), bounded like mbar_wait; every
 // lane of the warp takes the same outcome.
 __device__ __forceinline__ bool warp_wait_flag(const unsigned* flag, unsigned* status,
@@ -190,6 +180,12 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
       "l"(policy)
       : "memory");
+}
+
+// Bulk prefetch of [p, p + bytes) into L2 (bytes a multiple of 16, p 16-byte
+// aligned); no completion to wait for.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // 3-D tiled store shared -> global (bulk-group completion).

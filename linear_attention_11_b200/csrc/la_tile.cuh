@@ -30,5 +30,27 @@ __device__ __forceinline__ void store_row32_sw128(uint32_t base, int r, int blk,
   }
 }
 
+// Shared memory of the main kernel: a ring of Q tiles, a separate ring of K/V
+// tiles, the bf16 state copy, and (at T = 64) a dedicated output staging tile.
+// Q(i) is released once Q(i) S has been issued and completed; K/V(i) once the
+// state update of tile i has; so copies of later tiles start early and more
+// bytes stay in flight.  At T = 128 there is no room for a separate staging
+// tile and the output goes through the Q slot (released after its store has
+// read it).
+template <int T, int QST, int KVST>
+struct MainLayout {
+  static constexpr bool kDedicatedO = (T == 64);
+  static constexpr int kKBytes = T * kHeadDim * 2;
+  static constexpr int kKVBytes = 2 * kKBytes;
+  static constexpr int kKVOff = QST * kQBytes;
+  static constexpr int kSOff = kKVOff + KVST * kKVBytes;
+  static constexpr int kOOff = kSOff + kSBytes;
+  static constexpr int kBarOff = kOOff + (kDedicatedO ? kQBytes : 0);
+  // q_full[QST], q_empty[QST], kv_full[KVST], kv_empty[KVST], a_full, p_full,
+  // o_full[2], o_empty[2], s_full, sb_full, mma_done, store_ready, ostage_free
+  static constexpr int kNumBars = 2 * QST + 2 * KVST + 11;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
+};
 
 }  // namespace la

@@ -276,25 +276,34 @@ def test_forward_host_pipelined(la, N, piece, with_state):
 
 
 # ------------------------------------------------------------------ one span per kv head
-# With many (batch, kv head) units and short sequences the plan has one span
-# each; la_forward / la_forward_state / la_forward_ws then run the chunk loop
-# alone: it reads the initial state and writes the final one from tensor
-# memory.  In place with several CTAs per kv group (head subsets) a ticket
-# picks the CTA that writes.
-SINGLE = [
-    # B, Hq, Hkv, N, chunk   (tile / CTAs per kv group)
-    (40, 16, 4, 100, 64),    # T=64, two CTAs per group (tickets), ragged tail
-    (40, 16, 4, 100, 128),   # T=128, four CTAs per group
-    (160, 4, 4, 130, 64),    # single-head groups: 128-token tiles, one CTA per group
-    (64, 6, 2, 64, 64),      # group of 3 -> 128-token tiles, three CTAs per group
+# With many (batch, kv head) sequences and short N the plan has one span each,
+# and la_forward / la_forward_state / la_forward_ws run the persistent chunk
+# loop alone (one CTA per SM walks whole kv groups): it reads the initial
+# state and writes the final one from tensor memory, in place.
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+PERSISTENT = [
+    # B, Hq, Hkv, N, chunk
+    (40, 16, 4, 100, 64),    # T=64, two tiles per chunk step, ragged tail
+    (40, 16, 4, 300, 64),    # several chunk steps per item
+    (40, 16, 4, 100, 128),   # T=128, four tiles per chunk step
+    (160, 4, 4, 130, 64),    # single-head groups: 128-token tiles
+    (50, 18, 3, 77, 64),     # group of 6: three tiles per chunk step
     (100, 8, 2, 1, 64),      # one token
+    (37, 32, 4, 64, 64),     # 148 sequences: one item per CTA
+    (300, 2, 1, 65, 128),    # 300 items over the SMs, uneven rounds
+]
+FEWER_THAN_SMS = [
+    (30, 16, 4, 100, 64),    # 120 sequences: some SMs idle, one item each
+    (30, 16, 4, 100, 128),
+    (64, 6, 2, 64, 64),      # group of 3 -> 128-token tiles
 ]
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,N,chunk", SINGLE)
-def test_single_span_state_in_out(la, B, Hq, Hkv, N, chunk):
-    assert la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).nspan == 1
-    q, k, v = _qkv(B, Hq, Hkv, N, seed=700 + B + N)
+def _state_in_out(la, B, Hq, Hkv, N, chunk, seed):
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=seed)
     S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(N)) / 128
     ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy())
     qd, kd, vd = _cuda(q, k, v)
@@ -308,11 +317,27 @@ def test_single_span_state_in_out(la, B, Hq, Hkv, N, chunk):
     assert_bf16_close(o0.cpu(), oracle.recurrent(q, k, v)[0], "O from zero state")
 
 
-def test_single_span_matches_staged_scheme(la):
+@pytest.mark.parametrize("B,Hq,Hkv,N,chunk", PERSISTENT)
+def test_persistent_state_in_out(la, B, Hq, Hkv, N, chunk):
+    assert B * Hkv >= _sms()
+    assert la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).nspan == 1
+    _state_in_out(la, B, Hq, Hkv, N, chunk, seed=700 + B + N)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,chunk", FEWER_THAN_SMS)
+def test_one_span_fewer_sequences_than_sms(la, B, Hq, Hkv, N, chunk):
+    assert B * Hkv < _sms()
+    assert la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).nspan == 1
+    _state_in_out(la, B, Hq, Hkv, N, chunk, seed=750 + B + N)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N", [(48, 8, 2, 200), (160, 8, 2, 130)])
+def test_one_launch_path_matches_staged_scheme(la, B, Hq, Hkv, N):
     """The one-launch path and the three stages with the same one-span plan
-    compute the same outputs bit for bit (same entering state, same chunk
-    loop); the final states agree to fp32 rounding of the two sums."""
-    B, Hq, Hkv, N, chunk = 48, 8, 2, 200, 64
+    compute the same outputs bit for bit (same entering state, same tile
+    arithmetic in the same order); the final states agree to fp32 rounding
+    of the two sums (accumulated in tensor memory vs. span sum + scan)."""
+    chunk = 64
     plan = la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk)
     assert plan.nspan == 1
     qd, kd, vd = _cuda(*_qkv(B, Hq, Hkv, N, seed=801))
@@ -331,46 +356,44 @@ def test_single_span_matches_staged_scheme(la):
 
 
 def test_single_span_workspace(la):
-    """la_forward_ws needs only B*Hkv counters on the one-launch path; the
-    same workspace serves repeated in-place calls (counters re-zeroed)."""
-    B, Hq, Hkv, N, chunk = 40, 16, 4, 96, 64
-    assert la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).nspan == 1
-    nbytes = la.api.la_forward_workspace_bytes(B, Hq, Hkv, N, 128, chunk)
-    assert nbytes == 256 * ((B * Hkv * 4 + 255) // 256)
-    q, k, v = _qkv(B, Hq, Hkv, 2 * N, seed=901)
-    ref_o, ref_S = oracle.recurrent(q, k, v)
-    qd, kd, vd = _cuda(q, k, v)
-    ws = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device=DEV)  # not zero on entry
-    S = torch.zeros(B, Hkv, 128, 128, dtype=torch.float32, device=DEV)
-    outs = []
-    for piece in range(2):
-        sl = slice(piece * N, (piece + 1) * N)
-        o = torch.empty_like(qd[:, :, sl])
-        la.api.la_forward_ws(*(t[:, :, sl].contiguous() for t in (qd, kd, vd)), o, S, ws, chunk=chunk)
-        outs.append(o)
-    torch.cuda.synchronize()
-    assert_bf16_close(torch.cat(outs, dim=2).cpu(), ref_o, "O in two pieces")
-    assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
-    with pytest.raises(la.LAError) as e:
-        la.api.la_forward_ws(qd[:, :, :N].contiguous(), kd[:, :, :N].contiguous(),
-                             vd[:, :, :N].contiguous(), torch.empty_like(qd[:, :, :N]), S,
-                             ws[: nbytes - 256], chunk=chunk)
-    assert e.value.code == 5
+    """With one span per sequence la_forward_ws needs no workspace (a nominal
+    256 bytes, contents irrelevant); the state carries across two in-place
+    calls on consecutive pieces."""
+    for B, Hq, Hkv, N in ((30, 16, 4, 96), (40, 16, 4, 96)):
+        chunk = 64
+        assert la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).nspan == 1
+        nbytes = la.api.la_forward_workspace_bytes(B, Hq, Hkv, N, 128, chunk)
+        assert nbytes == 256
+        q, k, v = _qkv(B, Hq, Hkv, 2 * N, seed=901)
+        ref_o, ref_S = oracle.recurrent(q, k, v)
+        qd, kd, vd = _cuda(q, k, v)
+        ws = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device=DEV)  # not zero on entry
+        S = torch.zeros(B, Hkv, 128, 128, dtype=torch.float32, device=DEV)
+        outs = []
+        for piece in range(2):
+            sl = slice(piece * N, (piece + 1) * N)
+            o = torch.empty_like(qd[:, :, sl])
+            la.api.la_forward_ws(*(t[:, :, sl].contiguous() for t in (qd, kd, vd)), o, S, ws,
+                                 chunk=chunk)
+            outs.append(o)
+        torch.cuda.synchronize()
+        assert_bf16_close(torch.cat(outs, dim=2).cpu(), ref_o, f"O in two pieces, B={B}")
+        assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
 
 
-def test_multi_token_decode_shape(la):
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_multi_token_decode_shape(la, chunk):
     """64 known tokens for each of 256 sequences (64 query / 16 kv heads)
     through the one-launch path, continuing from a decode state: every output
     and the final state against the oracle's recurrence."""
     w = synth.DECODE_B256
     B, Hq, Hkv, T = w.B, w.Hq, w.Hkv, 64
-    assert la.api.la_prefill_plan(B, Hq, Hkv, T, 128, 64).nspan == 1
     S0 = synth.decode_state(w)
     q, k, v = synth.random_qkv(B, Hq, Hkv, T, 128, torch.bfloat16, w.seed + 1000)
     ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy(), o_dtype=np.float32)
     qd, kd, vd = _cuda(q, k, v)
     S = S0.to(DEV)
-    o = la.la_forward_state(qd, kd, vd, S=S, chunk=64)
+    o = la.la_forward_state(qd, kd, vd, S=S, chunk=chunk)
     torch.cuda.synchronize()
     assert la.la_device_status()[1] == 0
     assert_bf16_close(o.cpu(), ref_o, "multi-token O")
