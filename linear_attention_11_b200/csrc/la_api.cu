@@ -205,6 +205,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, i
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_state(CUtensorMap* map, const void* base, int64_t units) {
+  CUtensorMap probe;
+  if (!make_tmap_bf16(&probe, base, 128, 1, 64)) return false;  // resolves the encoder once
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)kHeadDim, (cuuint64_t)units};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 4, (cuuint64_t)kHeadDim * kHeadDim * 4};
+  const cuuint32_t box[3] = {32, (cuuint32_t)kHeadDim, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base),
+                             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 __global__ void selftest_wait_kernel(unsigned* status, const unsigned* flag, int64_t limit_ns) {

@@ -34,6 +34,9 @@ unsigned* device_status_ptr();
 // Builds a 3-D bf16 tensor map; returns false on failure.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, int64_t heads,
                     int box_rows);
+// 3-D fp32 tensor map over `units` d x d states [units, 128, 128]; box
+// {32, 128, 1} (32 columns of one state), 128-byte swizzle.
+bool make_tmap_state(CUtensorMap* map, const void* base, int64_t units);
 
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,

@@ -42,13 +42,19 @@ struct PersistParams {
   int Hq, Hkv, G, nsub, nspan, tiles_total, items;
 };
 
-template <int T, int QST, int KVST>
+// kStage: entering and final states pass through a 64 KB fp32 tile in shared
+// memory by bulk tensor copies (map_s over the states, [units, 128, 128]),
+// loaded an item ahead by a third copy lane; without it the math warps read
+// and write them row by row.  kDedO: a dedicated output staging tile (else
+// the output goes through the Q slot).
+template <int T, int QST, int KVST, bool kDedO, bool kStage>
 __global__ void __launch_bounds__(320, 1)
     prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
                            const __grid_constant__ CUtensorMap map_k,
                            const __grid_constant__ CUtensorMap map_v,
-                           const __grid_constant__ CUtensorMap map_o, const PersistParams p) {
-  using L = MainLayout<T, QST, KVST>;
+                           const __grid_constant__ CUtensorMap map_o,
+                           const __grid_constant__ CUtensorMap map_s, const PersistParams p) {
+  using L = MainLayout<T, QST, KVST, kDedO, kStage>;
   constexpr int HPT = kTileRows / T;
   constexpr bool kDedicatedO = L::kDedicatedO;
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, T, 0, 0);
@@ -76,10 +82,15 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* mma_done = sb_full + 1;
   uint64_t* store_ready = mma_done + 1;
   uint64_t* ostage_free = store_ready + 1;
+  uint64_t* st_full = ostage_free + 1;   // staged entering state of the CTA's k-th item landed
+  uint64_t* st_empty = st_full + 1;      // staging tile free again (read, final state stored)
+  uint64_t* stage_done = st_empty + 1;   // math warps done with the staging tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
 
   const uint32_t sS = base + L::kSOff;
+  const uint32_t sSt = base + L::kStOff;
+  const bool staged = kStage && p.ws != nullptr;
   auto sQ = [&](int i) { return base + (uint32_t)((i % QST) * kQBytes); };
   auto sK = [&](int c) { return base + (uint32_t)(L::kKVOff + (c % KVST) * L::kKVBytes); };
   auto sV = [&](int c) { return sK(c) + (uint32_t)L::kKBytes; };
@@ -118,6 +129,9 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(mma_done, 1);
     mbar_init(store_ready, 128);
     mbar_init(ostage_free, 1);
+    mbar_init(st_full, 1);
+    mbar_init(st_empty, 1);
+    mbar_init(stage_done, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -174,7 +188,7 @@ __global__ void __launch_bounds__(320, 1)
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
-        if (p.ws && nx >= 0)  // the next item's entering state, read at this item's end
+        if (!staged && p.ws && nx >= 0)  // the next item's entering state, read at its end
           prefetch_l2_bulk(p.ws + (size_t)nx * kDD, (uint32_t)(kDD * sizeof(float)));
         for (int cs = tb; cs < te; ++cs, ++gc) {
           const int s = gc % KVST;
@@ -195,6 +209,22 @@ __global__ void __launch_bounds__(320, 1)
         for (int k = (gc > KVST ? gc - KVST : 0); k < gc; ++k)
           mbar_wait_drain(&kv_full[k % KVST], (k / KVST) & 1);
       }
+    } else if (lane == 2 && staged) {
+      // entering state of the CTA's k-th item into the staging tile, once the
+      // tile is free (item k-1's state read and its final state stored)
+      prefetch_tmap(&map_s);
+      griddep_wait();
+      const uint64_t pol_s = policy_evict_first();
+      int k = 0;
+      for (int it = blockIdx.x; it < p.items; it += stride, ++k) {
+        if (k >= 1 && !mbar_wait(st_empty, (k - 1) & 1, p.status, abort_flag)) break;
+        mbar_arrive_expect_tx(st_full, kStateBytes);
+        uint8_t* dst = sm + (sSt - base);
+#pragma unroll
+        for (int bx = 0; bx < 4; ++bx)
+          tma_load_3d(dst + bx * kStateBoxBytes, &map_s, st_full, 32 * bx, 0, it, pol_s);
+      }
+      if (*abort_flag && k > 0) mbar_wait_drain(st_full, (k - 1) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -326,12 +356,46 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(sb_full);
     };
 
+    // Staged states: this warpgroup's half of row r of the next entering state
+    // from the staging tile into tensor memory and the bf16 copy (have_in),
+    // and of the final state from tensor memory into the same staging slots
+    // (have_out; each thread reads its own slots before writing them).
+    auto stage_swap = [&](bool have_in, bool have_out) {
+      // 16 columns at a time: the incoming and outgoing rows together would
+      // otherwise take 64 registers and spill
+#pragma unroll 1
+      for (int q = 2 * blk0; q < 2 * blk0 + 4; ++q) {
+        uint32_t v[16];
+        if (have_in) load_state_row16(sSt, r, q, v);
+        if (have_out) {
+          uint32_t w[16];
+          tmem_ld16(tmem + lane_base + kColS + q * 16, w);
+          tmem_wait_ld();
+          store_state_row16(sSt, r, q, w);
+        }
+        if (have_in) {
+          tmem_st16(tmem + lane_base + kColS + q * 16, v);
+          store_row16_sw128(sS, r, q, v);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      if (have_in) mbar_arrive(sb_full);
+      mbar_arrive(stage_done);
+    };
+
     // After the update of chunk step gc: within an item, the bf16 copy for
-    // the next chunk step; at an item's end, the final state out (one span per
-    // sequence) and the next item's entering state in.
-    auto state_step = [&](int gc, bool item_end, int bg, int nx) -> bool {
+    // the next chunk step; at an item's end (the CTA's item k), the final state
+    // out (one span per sequence) and the next item's entering state in.
+    auto state_step = [&](int gc, bool item_end, int bg, int nx, int k) -> bool {
       if (!warp_wait(s_full, gc & 1, p.status, abort_flag)) return false;
       tc_fence_after();
+      if (item_end && staged) {
+        if (nx >= 0 && !warp_wait(st_full, (k + 1) & 1, p.status, abort_flag)) return false;
+        stage_swap(nx >= 0, p.s_out != nullptr);
+        return true;
+      }
       if (!item_end) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
@@ -367,7 +431,12 @@ __global__ void __launch_bounds__(320, 1)
     // The kernel may start before the kernel writing the entering states has
     // finished (programmatic dependent launch): wait before the first read.
     griddep_wait();
-    load_state(blockIdx.x);
+    if (staged) {
+      ok = warp_wait(st_full, 0, p.status, abort_flag);
+      if (ok) stage_swap(true, false);
+    } else {
+      load_state(blockIdx.x);
+    }
 
     if (wg1) {
       auto mask_tile = [&](int i) -> bool {
@@ -408,9 +477,9 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(p_full);
         return true;
       };
-      ok = mask_tile(0);
+      ok = ok && mask_tile(0);
       int i = 0, gc = 0;
-      for (int it = blockIdx.x; it < p.items && ok; it += stride) {
+      for (int it = blockIdx.x, k = 0; it < p.items && ok; it += stride, ++k) {
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
@@ -427,7 +496,7 @@ __global__ void __launch_bounds__(320, 1)
               const bool do_step = last_hs && (ph == (step_first ? 0 : 1));
               const bool do_mask = has_next && (ph == (step_first ? 1 : 0));
               if (do_mask && !mask_tile(i + 1)) ok = false;
-              if (ok && do_step && !state_step(gc, item_end, bg, nx)) ok = false;
+              if (ok && do_step && !state_step(gc, item_end, bg, nx, k)) ok = false;
             }
             if (!ok) break;
             if (last_hs) ++gc;
@@ -435,8 +504,29 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     } else {
+      // Warp 6, after the math warps are done with the staging tile (use c:
+      // 0 = the first entering state, k + 1 = the end of item k): bulk-store
+      // the final state of sequence bg from it if asked, then hand the tile
+      // back to the copy lane.
+      auto stage_release = [&](int c, int bg, bool store) -> bool {
+        if (!warp_wait(stage_done, c & 1, p.status, abort_flag)) return false;
+        if (lane == 0) {
+          if (store) {
+            const uint8_t* src = sm + (sSt - base);
+#pragma unroll
+            for (int bx = 0; bx < 4; ++bx)
+              tma_store_3d(&map_s, src + bx * kStateBoxBytes, 32 * bx, 0, bg);
+            bulk_commit_group();
+            bulk_wait_group_read<0>();
+          }
+          mbar_arrive(st_empty);
+        }
+        __syncwarp();
+        return true;
+      };
+      if (staged && ok && warp == 6) ok = stage_release(0, 0, false);
       int i = 0, gc = 0;
-      for (int it = blockIdx.x; it < p.items && ok; it += stride) {
+      for (int it = blockIdx.x, k = 0; it < p.items && ok; it += stride, ++k) {
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int b = bg / p.Hkv, g = bg % p.Hkv;
@@ -445,7 +535,11 @@ __global__ void __launch_bounds__(320, 1)
           for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
             const bool last_hs = hs == p.nsub - 1;
             const bool item_end = last_hs && cs == te - 1;
-            if (last_hs && !state_step(gc, item_end, bg, nx)) { ok = false; break; }
+            if (last_hs && !state_step(gc, item_end, bg, nx, k)) { ok = false; break; }
+            if (staged && item_end && warp == 6 && !stage_release(k + 1, bg, p.s_out != nullptr)) {
+              ok = false;
+              break;
+            }
             if (last_hs) ++gc;
             // output epilogue: TMEM -> bf16 -> staging tile -> bulk store
             const uint32_t ob = (uint32_t)(i & 1);
@@ -509,12 +603,13 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int T, int QST, int KVST>
+template <int T, int QST, int KVST, bool kDedO, bool kStage>
 cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
-                           const PersistParams& p, bool dependent) {
-  using L = MainLayout<T, QST, KVST>;
+                           const CUtensorMap& map_s, const PersistParams& p, bool dependent) {
+  using L = MainLayout<T, QST, KVST, kDedO, kStage>;
   static_assert(L::kBytes <= 232448, "shared memory");
-  cudaError_t e = set_smem(prefill_persist_kernel<T, QST, KVST>, L::kBytes);
+  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage>;
+  cudaError_t e = set_smem(kernel, L::kBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -526,8 +621,7 @@ cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& ma
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = dependent ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, prefill_persist_kernel<T, QST, KVST>, maps.q, maps.k, maps.v,
-                            maps.o, p);
+  return cudaLaunchKernelEx(&cfg, kernel, maps.q, maps.k, maps.v, maps.o, map_s, p);
 }
 
 }  // namespace
@@ -542,8 +636,17 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
   PersistParams p{ws,    s_out, status, g.Hq,          g.Hkv,
                   g.G,   nsub,  g.nspan, g.tiles_total, (int)items};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
-  if (g.tile == 64) return launch_persist<64, 3, 2>(grid, stream, maps, p, dependent);
-  return launch_persist<128, 2, 2>(grid, stream, maps, p, dependent);
+  // One span per sequence with a state to carry: every item reads and writes
+  // 64 KB of state, staged through shared memory by bulk tensor copies (room
+  // for the tile: two Q slots, output through the Q slot).  Otherwise states
+  // are rare and the smem goes to the rings.
+  if (g.tile == 64 && g.nspan == 1 && ws && (!s_out || s_out == ws)) {
+    CUtensorMap map_s;
+    if (!make_tmap_state(&map_s, ws, (int64_t)g.B * g.Hkv)) return cudaErrorInvalidValue;
+    return launch_persist<64, 2, 2, false, true>(grid, stream, maps, map_s, p, dependent);
+  }
+  if (g.tile == 64) return launch_persist<64, 3, 2, true, false>(grid, stream, maps, maps.q, p, dependent);
+  return launch_persist<128, 2, 2, false, false>(grid, stream, maps, maps.q, p, dependent);
 }
 
 }  // namespace la
