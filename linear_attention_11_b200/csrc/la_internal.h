@@ -38,9 +38,11 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, i
 // {32, 128, 1} (32 columns of one state), 128-byte swizzle.
 bool make_tmap_state(CUtensorMap* map, const void* base, int64_t units);
 
+// skip_last: spans 0 .. nspan-2 only (the last span's state is needed only
+// for the final state, which the chunk loop then writes).
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
-                               cudaStream_t stream);
+                               cudaStream_t stream, bool skip_last = false);
 // Chunk loop with one CTA per (batch, kv head, head subset, span), used by
 // the backward passes.  qdiv: query rows of head h come from head h / qdiv of
 // the query tensor map; reverse: anti-causal pass (sum over s >= t), the
@@ -51,12 +53,20 @@ cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& map
 // Persistent schedule of the chunk loop: min(B*Hkv*nspan, num_ctas) CTAs walk
 // the items (one span of one (batch, kv head) sequence each, every query head
 // of the group) round-robin.  ws: entering state of item bg * nspan + j
-// (nullptr: zero); s_out (nspan == 1 only): final states [B*Hkv, d, d], may be
-// ws itself.  dependent: launched as a programmatic dependent of the previous
-// kernel in the stream.
+// (nullptr: zero); s_out (nullable): final states [B*Hkv, d, d], written by
+// the items of the last spans; with nspan == 1 it may be ws itself.
+// dependent: launched as a programmatic dependent of the previous kernel in
+// the stream.  stage_states (honoured at tile 64 with nspan == 1 and s_out
+// null or ws): states pass through shared memory by bulk tensor copies, for
+// short items where they are a large share of the bytes (see
+// stage_states_pays).
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
-                                   cudaStream_t stream, bool dependent);
+                                   cudaStream_t stream, bool dependent, bool stage_states);
+// Whether staging the states pays for a one-span plan: the staged layout
+// (two Q slots, output through a Q slot) streams tiles slower, so only items
+// of at most four tiles use it.
+bool stage_states_pays(const PrefillGeometry& g);
 size_t fused_workspace_bytes(int B, int Hkv, int nspan);
 // Workspace bytes la_forward_ws needs for `plan` (never zero): the span
 // states, or nothing (a nominal 256 bytes) with one span per sequence, which
@@ -73,9 +83,10 @@ cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& ma
                                  void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);
 // reverse: ws[j] <- S0 + sum_{i>j} ws[i] (the state entering span j of a
-// backwards walk); S receives S0 + sum_i ws[i] either way.
+// backwards walk); S receives S0 + sum_i ws[i] either way.  write_final =
+// false (forward only): ws[nspan-1] is not read and S is only read (S0).
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
-                              cudaStream_t stream, int reverse = 0);
+                              cudaStream_t stream, int reverse = 0, bool write_final = true);
 cudaError_t launch_decode(float* S, const void* q, const void* k, const void* v, void* o, int B,
                           int Hq, int Hkv, int d, cudaStream_t stream);
 cudaError_t launch_decode_steps(float* S, const void* q, const void* k, const void* v, void* o,

@@ -448,6 +448,7 @@ struct SpanParams {
   float* ws;
   unsigned* status;
   int nspan, tiles_total;
+  int nrun;  // spans computed per (batch, kv head): nspan, or nspan - 1 (the last one skipped)
 };
 
 template <int T, int STAGES>
@@ -476,8 +477,8 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
 
   griddep_launch_dependents();  // the scan may be scheduled; it waits for this grid
-  const int j = blockIdx.x % p.nspan;
-  const int bg = blockIdx.x / p.nspan;
+  const int j = blockIdx.x % p.nrun;
+  const int bg = blockIdx.x / p.nrun;
   const int tile_begin = (int)(((int64_t)j * p.tiles_total) / p.nspan);
   const int tile_end = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
   const int ntiles = tile_end - tile_begin;
@@ -591,9 +592,11 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
-                               cudaStream_t stream) {
-  SpanParams p{ws, status, g.nspan, g.tiles_total};
-  const dim3 grid((unsigned)(g.B * g.Hkv * g.nspan));
+                               cudaStream_t stream, bool skip_last) {
+  const int nrun = g.nspan - (skip_last ? 1 : 0);
+  if (nrun <= 0) return cudaSuccess;
+  SpanParams p{ws, status, g.nspan, g.tiles_total, nrun};
+  const dim3 grid((unsigned)(g.B * g.Hkv * nrun));
   cudaError_t e;
   if (g.tile == 64) {
     using L = SpanLayout<64, 4>;

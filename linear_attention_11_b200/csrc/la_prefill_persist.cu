@@ -37,7 +37,7 @@ namespace {
 
 struct PersistParams {
   const float* ws;  // entering state of item it at ws[it] (d x d fp32 each); nullptr: zero
-  float* s_out;     // one span per sequence: final state of sequence bg at s_out[bg]
+  float* s_out;     // final state of sequence bg at s_out[bg], written by its last span's item
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total, items;
 };
@@ -408,7 +408,8 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(sb_full);
         return true;
       }
-      if (p.s_out) {
+      // the final state of sequence bg is complete at the end of its last span
+      if (p.s_out && ((int)blockIdx.x + k * stride) % p.nspan == p.nspan - 1) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
         tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
@@ -628,19 +629,17 @@ cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& ma
 
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
-                                   cudaStream_t stream, bool dependent) {
-  if (s_out && g.nspan != 1) return cudaErrorInvalidValue;
+                                   cudaStream_t stream, bool dependent, bool stage_states) {
+  if (s_out && s_out == ws && g.nspan != 1) return cudaErrorInvalidValue;
   const int nsub = g.G / g.heads_per_tile;
   const int64_t items = (int64_t)g.B * g.Hkv * g.nspan;
   if (items <= 0 || items > 0x7fffffff || num_ctas <= 0) return cudaErrorInvalidValue;
   PersistParams p{ws,    s_out, status, g.Hq,          g.Hkv,
                   g.G,   nsub,  g.nspan, g.tiles_total, (int)items};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
-  // One span per sequence with a state to carry: every item reads and writes
-  // 64 KB of state, staged through shared memory by bulk tensor copies (room
-  // for the tile: two Q slots, output through the Q slot).  Otherwise states
-  // are rare and the smem goes to the rings.
-  if (g.tile == 64 && g.nspan == 1 && ws && (!s_out || s_out == ws)) {
+  // Staged states (room for the tile: two Q slots, output through the Q
+  // slot); otherwise the smem goes to the rings.
+  if (stage_states && g.tile == 64 && g.nspan == 1 && ws && (!s_out || s_out == ws)) {
     CUtensorMap map_s;
     if (!make_tmap_state(&map_s, ws, (int64_t)g.B * g.Hkv)) return cudaErrorInvalidValue;
     return launch_persist<64, 2, 2, false, true>(grid, stream, maps, map_s, p, dependent);

@@ -331,12 +331,14 @@ def test_one_span_fewer_sequences_than_sms(la, B, Hq, Hkv, N, chunk):
     _state_in_out(la, B, Hq, Hkv, N, chunk, seed=750 + B + N)
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,N", [(48, 8, 2, 200), (160, 8, 2, 130)])
+@pytest.mark.parametrize("B,Hq,Hkv,N", [(48, 8, 2, 200), (160, 8, 2, 130), (200, 8, 2, 64)])
 def test_one_launch_path_matches_staged_scheme(la, B, Hq, Hkv, N):
     """The one-launch path and the three stages with the same one-span plan
     compute the same outputs bit for bit (same entering state, same tile
     arithmetic in the same order); the final states agree to fp32 rounding
-    of the two sums (accumulated in tensor memory vs. span sum + scan)."""
+    of the two sums (accumulated in tensor memory vs. span sum + scan).
+    The last shape has two tiles per item, where states are staged through
+    shared memory."""
     chunk = 64
     plan = la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk)
     assert plan.nspan == 1
