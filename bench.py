@@ -27,6 +27,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import math
 import os
 import statistics
@@ -156,11 +157,14 @@ def timed(fn, steps, stream):
 
 def kernel_source_sha256():
     """Hash of the chunk-loop kernel's source (its file and the device headers
-    it includes), the key under which ncu figures of it are committed."""
+    it includes) with // comments and whitespace removed, the key under which
+    ncu figures of it are committed."""
     csrc = os.path.join(ROOT, "linear_attention_11_b200", "csrc")
     h = hashlib.sha256()
     for name in ("la_prefill_persist.cu", "la_tile.cuh", "la_ptx.cuh"):
-        h.update(open(os.path.join(csrc, name), "rb").read())
+        text = open(os.path.join(csrc, name), encoding="utf-8").read()
+        code = re.sub(r"//[^\n]*", "", text)  # no string literal in these files holds "//"
+        h.update("".join(code.split()).encode())
     return h.hexdigest()
 
 

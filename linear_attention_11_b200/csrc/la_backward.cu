@@ -18,7 +18,9 @@
 //   dS0  = dSf + sum_{h in g} sum_t q_{t,h}^T do_{t,h}
 //        -> the per-head final states of the dv pass summed over each group.
 // Every pass runs the tensor-core kernels of the prefill (span states, scan,
-// chunk loop), the anti-causal ones in their reverse mode.
+// persistent chunk loop), the anti-causal ones in their reverse mode; the dv
+// and dk walks share one set of span states (the dk walk reads them
+// transposed).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -132,29 +134,37 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
   const size_t sq_bytes = round((size_t)B * Hkv * dd * 4);
   const size_t sm_bytes = round((size_t)B * Hq * dd * 4);
   const size_t part_bytes = round((size_t)B * Hq * N * d * 2);
-  const size_t wsq = round((size_t)plan_q.workspace_bytes), wsm = round((size_t)plan_m.workspace_bytes);
-  const size_t total = sq_bytes + sm_bytes + part_bytes + wsq + wsm;
+  const size_t wsq = round(forward_workspace_bytes(plan_q));
+  const size_t wsm = plan_m.nspan > 1 ? round((size_t)plan_m.workspace_bytes) : 0;
+  const size_t total = sq_bytes + 2 * sm_bytes + part_bytes + wsq + wsm;
   char* pool = nullptr;
   if (cudaMallocAsync(reinterpret_cast<void**>(&pool), total, s) != cudaSuccess) return LA_ERR_CUDA;
-  float* S_q = reinterpret_cast<float*>(pool);
-  float* S_m = reinterpret_cast<float*>(pool + sq_bytes);
-  la_bf16* part = reinterpret_cast<la_bf16*>(pool + sq_bytes + sm_bytes);
-  float* ws_q = reinterpret_cast<float*>(pool + sq_bytes + sm_bytes + part_bytes);
-  float* ws_m = reinterpret_cast<float*>(pool + sq_bytes + sm_bytes + part_bytes + wsq);
+  char* cur = pool;
+  auto take = [&](size_t n) { char* p = cur; cur += n; return p; };
+  float* S_q = reinterpret_cast<float*>(take(sq_bytes));
+  float* S_in = reinterpret_cast<float*>(take(sm_bytes));   // dSf on each group's first head
+  float* S_fin = reinterpret_cast<float*>(take(sm_bytes));  // per-head final states of the dv walk
+  la_bf16* part = reinterpret_cast<la_bf16*>(take(part_bytes));
+  void* ws_q = take(wsq);
+  float* ws_m = wsm ? reinterpret_cast<float*>(take(wsm)) : nullptr;
 
   auto cu = [&](cudaError_t e) {
     if (e != cudaSuccess && st == LA_OK) st = LA_ERR_CUDA;
   };
   const size_t row = (size_t)N * d, total8 = (size_t)B * Hkv * row / 8;
   const unsigned red_blocks = (unsigned)((total8 + 255) / 256);
+  int dev = 0, sms = 0;
+  cu(cudaGetDevice(&dev));
+  cu(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
 
   // ---- dq: the forward pass on (dO, V, K) from S0^T
   cu(place_states(S0, S_q, B, Hkv, 1, d, 1, s));
-  if (st == LA_OK) st = la_prefill_span_states(v, k, B, Hkv, N, d, &plan_q, ws_q, stream);
-  if (st == LA_OK) st = la_prefill_scan(ws_q, S_q, B, Hkv, d, &plan_q, stream);
-  if (st == LA_OK) st = la_prefill_main(dO, v, k, dq, ws_q, B, Hq, Hkv, N, d, &plan_q, stream);
+  if (st == LA_OK) st = forward_dispatch(dO, v, k, dq, S_q, B, Hq, Hkv, N, plan_q, ws_q, s);
 
-  // ---- dv, then dk: anti-causal passes per query head, summed over groups
+  // ---- dv, then dk: anti-causal walks per query head, summed over groups.
+  // One state serves both: D = sum_t q_t^T do_t over the later chunks (dv
+  // walk, from dSf), and its transpose (dk walk, from dSf^T), so the dk walk
+  // reads the dv walk's entering states transposed.
   PrefillGeometry gm;
   gm.B = B;
   gm.Hq = Hq;
@@ -165,33 +175,48 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
   gm.heads_per_tile = plan_m.heads_per_tile;
   gm.tiles_total = plan_m.tiles_total;
   gm.nspan = plan_m.nspan;
+  cu(place_states(dSf, S_in, B, Hq, G, d, 0, s));
+  if (plan_m.nspan > 1)
+    cu(cudaMemcpyAsync(S_fin, S_in, (size_t)B * Hq * dd * 4, cudaMemcpyDeviceToDevice, s));
   for (int pass = 0; pass < 2 && st == LA_OK; ++pass) {
-    // dv: queries K, keys Q, values dO, initial dSf;  dk: queries V, keys dO, values Q, dSf^T
+    // dv: queries K, keys Q, values dO;  dk: queries V, keys dO, values Q
     const la_bf16* qsrc = pass == 0 ? k : v;
     const la_bf16* ksrc = pass == 0 ? q : dO;
     const la_bf16* vsrc = pass == 0 ? dO : q;
     la_bf16* dst = pass == 0 ? dv : dk;
-    cu(place_states(dSf, S_m, B, Hq, G, d, pass == 1 ? 1 : 0, s));
     PrefillMaps maps;
-    if (st == LA_OK &&
-        (!make_tmap_bf16(&maps.q, qsrc, N, (int64_t)B * Hkv, gm.tile) ||
-         !make_tmap_bf16(&maps.k, ksrc, N, (int64_t)B * Hq, gm.tile) ||
-         !make_tmap_bf16(&maps.v, vsrc, N, (int64_t)B * Hq, gm.tile) ||
-         !make_tmap_bf16(&maps.o, part, N, (int64_t)B * Hq, gm.tile)))
+    if (!make_tmap_bf16(&maps.q, qsrc, N, (int64_t)B * Hkv, gm.tile) ||
+        !make_tmap_bf16(&maps.k, ksrc, N, (int64_t)B * Hq, gm.tile) ||
+        !make_tmap_bf16(&maps.v, vsrc, N, (int64_t)B * Hq, gm.tile) ||
+        !make_tmap_bf16(&maps.o, part, N, (int64_t)B * Hq, gm.tile)) {
       st = LA_ERR_CUDA;
-    if (st == LA_OK) cu(launch_span_states(gm, maps.k, maps.v, ws_m, status, s));
-    if (st == LA_OK) cu(launch_state_scan(ws_m, S_m, B * Hq, gm.nspan, d, s, 1));
-    if (st == LA_OK) cu(launch_prefill_main(gm, maps, ws_m, status, s, G, 1));
+      break;
+    }
+    if (plan_m.nspan > 1) {
+      if (pass == 0) {  // span states of D and the reverse scan (S_fin: dSf -> final)
+        cu(launch_span_states(gm, maps.k, maps.v, ws_m, status, s));
+        if (st == LA_OK) cu(launch_state_scan(ws_m, S_fin, B * Hq, gm.nspan, d, s, 1));
+      }
+      // the dv walk may overlap the scan's tail (it waits before reading
+      // states); the dk walk writes the partial sums the dv reduction reads,
+      // so it starts only after it
+      if (st == LA_OK)
+        cu(launch_prefill_persist(gm, maps, ws_m, nullptr, status, sms, s, pass == 0, false, G,
+                                  1, pass));
+    } else if (st == LA_OK) {  // one span: from dSf (dSf^T), the dv walk writes the final states
+      cu(launch_prefill_persist(gm, maps, S_in, pass == 0 ? S_fin : nullptr, status, sms, s, false,
+                                false, G, 1, pass));
+    }
     if (st == LA_OK) {
       reduce_heads_kernel<<<red_blocks, 256, 0, s>>>(
           reinterpret_cast<const __nv_bfloat16*>(part), reinterpret_cast<__nv_bfloat16*>(dst), G,
           row, total8);
       cu(cudaGetLastError());
     }
-    if (pass == 0 && dS0 && st == LA_OK) {
-      reduce_states_kernel<<<dim3(16, (unsigned)(B * Hkv)), 256, 0, s>>>(S_m, dS0, G, (int)dd);
-      cu(cudaGetLastError());
-    }
+  }
+  if (dS0 && st == LA_OK) {
+    reduce_states_kernel<<<dim3(16, (unsigned)(B * Hkv)), 256, 0, s>>>(S_fin, dS0, G, (int)dd);
+    cu(cudaGetLastError());
   }
   cu(cudaFreeAsync(pool, s));
   return st;

@@ -43,26 +43,23 @@ bool make_tmap_state(CUtensorMap* map, const void* base, int64_t units);
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
                                cudaStream_t stream, bool skip_last = false);
-// Chunk loop with one CTA per (batch, kv head, head subset, span), used by
-// the backward passes.  qdiv: query rows of head h come from head h / qdiv of
-// the query tensor map; reverse: anti-causal pass (sum over s >= t), the
-// tiles of every span walked from the end.
-cudaError_t launch_prefill_main(const PrefillGeometry& g, const PrefillMaps& maps,
-                                const float* ws, unsigned* status, cudaStream_t stream,
-                                int qdiv = 1, int reverse = 0);
-// Persistent schedule of the chunk loop: min(B*Hkv*nspan, num_ctas) CTAs walk
-// the items (one span of one (batch, kv head) sequence each, every query head
-// of the group) round-robin.  ws: entering state of item bg * nspan + j
-// (nullptr: zero); s_out (nullable): final states [B*Hkv, d, d], written by
-// the items of the last spans; with nspan == 1 it may be ws itself.
-// dependent: launched as a programmatic dependent of the previous kernel in
-// the stream.  stage_states (honoured at tile 64 with nspan == 1 and s_out
-// null or ws): states pass through shared memory by bulk tensor copies, for
-// short items where they are a large share of the bytes (see
-// stage_states_pays).
+// Persistent chunk loop: min(B*Hkv*nspan, num_ctas) CTAs walk the items (one
+// span of one (batch, kv head) sequence each, every query head of the group)
+// round-robin.  ws: entering state of item bg * nspan + j (nullptr: zero);
+// s_out (nullable): final states [B*Hkv, d, d], written by the items of the
+// last spans in walk order; with nspan == 1 it may be ws itself.  dependent:
+// launched as a programmatic dependent of the previous kernel in the stream.
+// stage_states (honoured at tile 64, nspan == 1, forward, s_out null or ws):
+// states pass through shared memory by bulk tensor copies, for short items
+// where they are a large share of the bytes (see stage_states_pays).
+// qdiv: query rows of head h come from head h / qdiv of the query tensor map;
+// reverse: anti-causal walk (sum over s >= t), each span from its end, tile
+// 128 only (the backward); transpose_in (reverse only): entering states read
+// transposed (not with s_out == ws).
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
-                                   cudaStream_t stream, bool dependent, bool stage_states);
+                                   cudaStream_t stream, bool dependent, bool stage_states,
+                                   int qdiv = 1, int reverse = 0, int transpose_in = 0);
 // Whether staging the states pays for a one-span plan: the staged layout
 // (two Q slots, output through a Q slot) streams tiles slower, so only items
 // of at most four tiles use it.

@@ -1,10 +1,19 @@
-// la_prefill_persist.cu -- persistent schedule of the chunk-loop kernel.
+// la_prefill_persist.cu -- the chunk loop of the prefill (and of the
+// backward's anti-causal walks) as a persistent tensor-core kernel.
 //
-// Per 128-row tile the arithmetic is that of prefill_main_kernel (the causal
-// chunk form of "如何理解MiniMax股价创历史新高？拆解国产大模型技术底座", section
-// "Lightning Attention：长上下文为什么突然变得便宜了": O_c = Q_c S + tril(Q_c
-// K_c^T) V_c, then S += K_c^T V_c; grouped kv heads as in "MiniMax-01与
-// Lightning Attention", section 1.1).  What differs is the schedule:
+// Per 128-row tile it computes the causal chunk form of "如何理解MiniMax股价创
+// 历史新高？拆解国产大模型技术底座", section "Lightning Attention：长上下文为什么
+// 突然变得便宜了": O_c = Q_c S + tril(Q_c K_c^T) V_c, then S += K_c^T V_c, with
+// grouped kv heads as in "MiniMax-01与Lightning Attention", section 1.1.
+// Tile: 128 rows = HPT query heads x T tokens (T = 64, HPT = 2, or T = 128,
+// HPT = 1), d = 128:
+//   A  = Q_c K_c^T      tcgen05 M=128 N=T  K=128 (SS) -> TMEM
+//   P  = bf16(tril(A))  TMEM -> registers -> TMEM (diagonal kept)
+//   O  = Q_c bf16(S)    tcgen05 M=128 N=128 K=128 (SS)
+//   O += P V_c          tcgen05 M=128 N=128 K=T (A from TMEM)
+//   S += K_c^T V_c      tcgen05 M=128 N=128 K=T (SS, both MN-major)
+//   O -> bf16 -> smem -> bulk tensor store (clipped at N; loads past N read 0)
+// Schedule:
 //   - one CTA per SM walks a list of work items, item = one span of one
 //     (batch, kv head) sequence, items dealt round-robin; the copy, MMA and
 //     math pipelines run on across item boundaries, so the fill of one item
@@ -18,8 +27,8 @@
 //     whole sequence writes the final state (tensor memory after the last
 //     chunk's update) at the item's end, in place if asked.
 //
-// Roles (320 threads) and tensor memory as in prefill_main_kernel: warp 0
-// lane 0 streams Q tiles, lane 1 K/V tiles (and the L2 prefetch); warp 1
+// Roles (320 threads): warp 0 lane 0 streams Q tiles, lane 1 K/V tiles (and
+// the L2 prefetch), lane 2 staged states; warp 1 owns the tensor memory and
 // issues the MMAs; warps 2-5 mask score tiles, warps 6-9 store output tiles;
 // both warpgroups handle half of the state columns.  TMEM: O buffers at
 // columns 0 and 128 (score tiles first), P at 256, state at 384.
@@ -40,14 +49,19 @@ struct PersistParams {
   float* s_out;     // final state of sequence bg at s_out[bg], written by its last span's item
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total, items;
+  int qdiv;          // query rows of head h come from head h / qdiv of the query tensor
+  int reverse;       // anti-causal (s >= t): each span walked from its end
+  int transpose_in;  // entering states read transposed (register path)
 };
 
 // kStage: entering and final states pass through a 64 KB fp32 tile in shared
 // memory by bulk tensor copies (map_s over the states, [units, 128, 128]),
 // loaded an item ahead by a third copy lane; without it the math warps read
 // and write them row by row.  kDedO: a dedicated output staging tile (else
-// the output goes through the Q slot).
-template <int T, int QST, int KVST, bool kDedO, bool kStage>
+// the output goes through the Q slot).  kRev: the anti-causal passes of the
+// backward (sum over s >= t, spans walked from their end, entering states
+// optionally read transposed).
+template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kRev>
 __global__ void __launch_bounds__(320, 1)
     prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
                            const __grid_constant__ CUtensorMap map_k,
@@ -104,6 +118,8 @@ __global__ void __launch_bounds__(320, 1)
     te = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
   };
   const int stride = (int)gridDim.x;
+  // n-th chunk step of the span [tb, te): forwards, or from the end in reverse
+  auto chunk_at = [&](int tb, int te, int n) { return kRev ? te - 1 - n : tb + n; };
   auto next_item = [&](int it) { return it + stride < p.items ? it + stride : -1; };
 
   const int warp = threadIdx.x >> 5;
@@ -156,7 +172,8 @@ __global__ void __launch_bounds__(320, 1)
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int b = bg / p.Hkv, g = bg % p.Hkv;
-        for (int cs = tb; cs < te && go; ++cs) {
+        for (int n = 0; n < te - tb && go; ++n) {
+          const int cs = chunk_at(tb, te, n);
           for (int hs = 0; hs < p.nsub; ++hs, ++i) {
             const int s = i % QST;
             if (i >= QST && !mbar_wait(&q_empty[s], ((i / QST) - 1) & 1, p.status, abort_flag)) {
@@ -167,7 +184,7 @@ __global__ void __launch_bounds__(320, 1)
             uint8_t* q_dst = sm + (sQ(i) - base);
 #pragma unroll
             for (int hh = 0; hh < HPT; ++hh) {
-              const int qh = b * p.Hq + g * p.G + hs * HPT + hh;
+              const int qh = (b * p.Hq + g * p.G + hs * HPT + hh) / p.qdiv;
               tma_load_3d(q_dst + hh * T * 128, &map_q, &q_full[s], 0, cs * T, qh, pol_q);
               tma_load_3d(q_dst + kHalf + hh * T * 128, &map_q, &q_full[s], 64, cs * T, qh,
                           pol_q);
@@ -190,7 +207,8 @@ __global__ void __launch_bounds__(320, 1)
         const int nx = next_item(it);
         if (!staged && p.ws && nx >= 0)  // the next item's entering state, read at its end
           prefetch_l2_bulk(p.ws + (size_t)nx * kDD, (uint32_t)(kDD * sizeof(float)));
-        for (int cs = tb; cs < te; ++cs, ++gc) {
+        for (int n = 0; n < te - tb; ++n, ++gc) {
+          const int cs = chunk_at(tb, te, n);
           const int s = gc % KVST;
           if (gc >= KVST && !mbar_wait(&kv_empty[s], ((gc / KVST) - 1) & 1, p.status, abort_flag)) {
             go = false;
@@ -231,8 +249,8 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ MMA issuer
     // Per tile i (chunk step gc, head subset hs): QS(i) PV(i); then, inside a
     // chunk step, QK(i+1); after the last head subset, QK(i+1) and the state
-    // update KV(gc) in the order of prefill_main_kernel (update first without
-    // a third K/V slot).  Every item ends with its update, so the state in
+    // update KV(gc) (update first without a third K/V slot, so the next tile's
+    // copy is not waited for).  Every item ends with its update, so the state in
     // tensor memory is final there.
     if (elect_one()) {
       auto issue_qk = [&](int i, int gci) -> bool {
@@ -270,7 +288,8 @@ __global__ void __launch_bounds__(320, 1)
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const bool last_item = next_item(it) < 0;
-        for (int cs = tb; cs < te && ok; ++cs) {
+        for (int n = 0; n < te - tb && ok; ++n) {
+          const int cs = chunk_at(tb, te, n);
           for (int hs = 0; hs < p.nsub && ok; ++hs) {
             const uint32_t ob = (uint32_t)(i & 1);
             const uint32_t ocol = ob * 128;
@@ -294,7 +313,7 @@ __global__ void __launch_bounds__(320, 1)
             mma_commit(&o_full[ob]);
             mma_commit(&q_empty[i % QST]);
             const bool last_hs = hs == p.nsub - 1;
-            const bool item_end = last_hs && cs == te - 1;
+            const bool item_end = last_hs && n == te - tb - 1;
             const bool has_next = !(last_item && item_end);
             // the next tile's scores before the update only inside an item: at
             // an item's end the update goes first, so the state hand-over to
@@ -324,6 +343,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int t_in = r % T;
     const int diag_blk = t_in / 32;
+    constexpr bool reverse = kRev;
     const int blk0 = wg1 ? 0 : 2;  // state column blocks this warpgroup handles
     const bool store_thread = (warp == 6 && lane == 0);
     bool ok = true;
@@ -334,18 +354,25 @@ __global__ void __launch_bounds__(320, 1)
       const float4* src =
           p.ws ? reinterpret_cast<const float4*>(p.ws + (size_t)it * kDD + (size_t)r * kHeadDim)
                : nullptr;
+      const float* col = p.ws ? p.ws + (size_t)it * kDD + r : nullptr;  // column r (transposed)
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb) {
         const int blk = blk0 + bb;
         uint32_t v[32];
+        if (kRev && p.transpose_in && col) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (src) f = src[blk * 8 + m];  // plain loads: the state may be updated in place
-          v[4 * m + 0] = __float_as_uint(f.x);
-          v[4 * m + 1] = __float_as_uint(f.y);
-          v[4 * m + 2] = __float_as_uint(f.z);
-          v[4 * m + 3] = __float_as_uint(f.w);
+          for (int e = 0; e < 32; ++e)  // read-only here: s_out is never ws with transpose_in
+            v[e] = __float_as_uint(__ldg(col + (size_t)(blk * 32 + e) * kHeadDim));
+        } else {
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (src) f = src[blk * 8 + m];  // plain loads: the state may be updated in place
+            v[4 * m + 0] = __float_as_uint(f.x);
+            v[4 * m + 1] = __float_as_uint(f.y);
+            v[4 * m + 2] = __float_as_uint(f.z);
+            v[4 * m + 3] = __float_as_uint(f.w);
+          }
         }
         tmem_st32(tmem + lane_base + kColS + blk * 32, v);
         store_row32_sw128(sS, r, blk, v);
@@ -409,7 +436,9 @@ __global__ void __launch_bounds__(320, 1)
         return true;
       }
       // the final state of sequence bg is complete at the end of its last span
-      if (p.s_out && ((int)blockIdx.x + k * stride) % p.nspan == p.nspan - 1) {
+      // in walk order (span 0 in reverse)
+      const int jspan = ((int)blockIdx.x + k * stride) % p.nspan;
+      if (p.s_out && jspan == (reverse ? 0 : p.nspan - 1)) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
         tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
@@ -455,7 +484,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int bb = 0; bb < 2; ++bb) {
             const int blk = 2 * h + bb;
-            need[bb] = T == 64 || blk <= diag_blk;
+            need[bb] = T == 64 || (reverse ? blk >= diag_blk : blk <= diag_blk);
             if (need[bb]) tmem_ld32(tmem + lane_base + ocol + blk * 32, a[bb]);
           }
           tmem_wait_ld();
@@ -466,8 +495,10 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
               const int s0 = blk * 32 + 2 * m;
-              const float f0 = need[bb] && s0 <= t_in ? __uint_as_float(a[bb][2 * m]) : 0.0f;
-              const float f1 = need[bb] && s0 + 1 <= t_in ? __uint_as_float(a[bb][2 * m + 1]) : 0.0f;
+              const bool keep0 = need[bb] && (reverse ? s0 >= t_in : s0 <= t_in);
+              const bool keep1 = need[bb] && (reverse ? s0 + 1 >= t_in : s0 + 1 <= t_in);
+              const float f0 = keep0 ? __uint_as_float(a[bb][2 * m]) : 0.0f;
+              const float f1 = keep1 ? __uint_as_float(a[bb][2 * m + 1]) : 0.0f;
               pk[m] = pack_bf16x2(f0, f1);
             }
             tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
@@ -484,10 +515,11 @@ __global__ void __launch_bounds__(320, 1)
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
-        for (int cs = tb; cs < te && ok; ++cs) {
+        for (int n = 0; n < te - tb && ok; ++n) {
+          const int cs = chunk_at(tb, te, n);
           for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
             const bool last_hs = hs == p.nsub - 1;
-            const bool item_end = last_hs && cs == te - 1;
+            const bool item_end = last_hs && n == te - tb - 1;
             const bool has_next = !(item_end && nx < 0);
             // the MMA order decides which of the two is ready first; one call
             // site each (two inlined copies of either spill registers at T = 128)
@@ -532,10 +564,11 @@ __global__ void __launch_bounds__(320, 1)
         span_of(it, bg, tb, te);
         const int b = bg / p.Hkv, g = bg % p.Hkv;
         const int nx = next_item(it);
-        for (int cs = tb; cs < te && ok; ++cs) {
+        for (int n = 0; n < te - tb && ok; ++n) {
+          const int cs = chunk_at(tb, te, n);
           for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
             const bool last_hs = hs == p.nsub - 1;
-            const bool item_end = last_hs && cs == te - 1;
+            const bool item_end = last_hs && n == te - tb - 1;
             if (last_hs && !state_step(gc, item_end, bg, nx, k)) { ok = false; break; }
             if (staged && item_end && warp == 6 && !stage_release(k + 1, bg, p.s_out != nullptr)) {
               ok = false;
@@ -604,12 +637,12 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int T, int QST, int KVST, bool kDedO, bool kStage>
+template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kRev = false>
 cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
                            const CUtensorMap& map_s, const PersistParams& p, bool dependent) {
   using L = MainLayout<T, QST, KVST, kDedO, kStage>;
   static_assert(L::kBytes <= 232448, "shared memory");
-  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage>;
+  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage, kRev>;
   cudaError_t e = set_smem(kernel, L::kBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -629,21 +662,29 @@ cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& ma
 
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
-                                   cudaStream_t stream, bool dependent, bool stage_states) {
+                                   cudaStream_t stream, bool dependent, bool stage_states,
+                                   int qdiv, int reverse, int transpose_in) {
   if (s_out && s_out == ws && g.nspan != 1) return cudaErrorInvalidValue;
   const int nsub = g.G / g.heads_per_tile;
   const int64_t items = (int64_t)g.B * g.Hkv * g.nspan;
   if (items <= 0 || items > 0x7fffffff || num_ctas <= 0) return cudaErrorInvalidValue;
-  PersistParams p{ws,    s_out, status, g.Hq,          g.Hkv,
-                  g.G,   nsub,  g.nspan, g.tiles_total, (int)items};
+  if (qdiv < 1 || (transpose_in && s_out == ws && s_out)) return cudaErrorInvalidValue;
+  PersistParams p{ws,    s_out, status,        g.Hq,       g.Hkv, g.G,     nsub,
+                  g.nspan, g.tiles_total, (int)items, qdiv, reverse, transpose_in};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
   // Staged states (room for the tile: two Q slots, output through the Q
   // slot); otherwise the smem goes to the rings.
-  if (stage_states && g.tile == 64 && g.nspan == 1 && ws && (!s_out || s_out == ws)) {
+  if (stage_states && !reverse && !transpose_in && g.tile == 64 && g.nspan == 1 && ws &&
+      (!s_out || s_out == ws)) {
     CUtensorMap map_s;
     if (!make_tmap_state(&map_s, ws, (int64_t)g.B * g.Hkv)) return cudaErrorInvalidValue;
     return launch_persist<64, 2, 2, false, true>(grid, stream, maps, map_s, p, dependent);
   }
+  if (reverse) {  // the backward's anti-causal passes: one query head per tile
+    if (g.tile != 128) return cudaErrorInvalidValue;
+    return launch_persist<128, 2, 2, false, false, true>(grid, stream, maps, maps.q, p, dependent);
+  }
+  if (transpose_in) return cudaErrorInvalidValue;
   if (g.tile == 64) return launch_persist<64, 3, 2, true, false>(grid, stream, maps, maps.q, p, dependent);
   return launch_persist<128, 2, 2, false, false>(grid, stream, maps, maps.q, p, dependent);
 }
