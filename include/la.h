@@ -124,7 +124,7 @@ la_status la_forward_ws(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la
  * q, k, v, o are host pointers, page-locked (cudaHostAlloc / cudaHostRegister)
  * so the copies run asynchronously, in the layouts above; S (nullable) is a
  * DEVICE state as in la_forward_state.  The sequence is processed in pieces of
- * `piece` tokens (0: about N/8; rounded up to whole tiles): piece p is copied
+ * `piece` tokens (0: about N/16; rounded up to whole tiles): piece p is copied
  * in on a copy-in stream, computed on `stream` with the state carried from
  * piece p-1 ([MX01] section 4.1: the state is the whole resume point), and
  * copied out on a copy-out stream, so the two copy directions and the compute
