@@ -14,7 +14,8 @@
 // thread keeps its updated rows in registers for the G dot products, and the
 // per-row-group partial sums are reduced through shared memory.  S is read and
 // written exactly once with streaming cache hints.  The single step runs 512
-// threads per CTA, the multi-step kernel 256.
+// threads per CTA (256 for groups above 16 heads); the multi-step kernel keeps
+// one state column per thread.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -23,7 +24,6 @@
 namespace la {
 namespace {
 
-constexpr int kDecodeThreads = 256;
 constexpr int kMaxGroup = 32;  // query heads per kv head supported by the decode step
 
 template <int D, int NT>
@@ -97,117 +97,130 @@ __global__ void __launch_bounds__(NT)
 // Several decode steps per launch: the state of one (batch, kv head) stays in
 // registers across `steps` tokens, so it crosses HBM once per launch instead
 // of once per token.  Step t: S += k_t^T v_t; o_{t,h} = q_{t,h} S, in token
-// order -- the same recurrence as decode_step_kernel, applied `steps` times.
-// Inputs follow the prefill layout with N = steps: q, o [B, Hq, steps, D],
-// k, v [B, Hkv, steps, D].  The next step's q, k, v are loaded into registers
-// while the current step computes.
-template <int D>
-__global__ void __launch_bounds__(kDecodeThreads)
+// order -- the same recurrence as decode_step_kernel, applied `steps` times,
+// with the same fmaf(k_r, v_c, S_rc) per element, so the state is bit for bit
+// that of single steps.  Inputs follow the prefill layout with N = steps:
+// q, o [B, Hq, steps, D], k, v [B, Hkv, steps, D].
+//
+// One thread per state column c (D threads per unit, column in D registers):
+// the update is elementwise and o_{t,h}[c] = sum_r q_{t,h}[r] S[r][c] is a
+// per-thread sum, so no cross-thread reduction is needed; k and q come from
+// shared memory as broadcast float4 reads.  Query heads go in passes of GB
+// (the update rides on the first pass).  The next step's k, v, q are loaded
+// into registers while the current step computes, then written to the other
+// half of a double buffer: one barrier per step.
+template <int D, int GB>
+__global__ void __launch_bounds__(D)
     decode_steps_kernel(float* __restrict__ S, const __nv_bfloat16* __restrict__ q,
                         const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                         __nv_bfloat16* __restrict__ o, int Hq, int Hkv, int steps) {
-  constexpr int TPR = D / 4;
-  constexpr int RP = kDecodeThreads / TPR;
-  constexpr int RPT = D / RP;
-  extern __shared__ float sh[];
+  extern __shared__ float4 sh4[];
+  float* sh = reinterpret_cast<float*>(sh4);
   const int G = Hq / Hkv;
-  const int per_step = (G + 2) * D;  // k, v, then the G query rows of one step
-  float* tok = sh;                   // [per_step] current step
-  float* red = tok + per_step;       // [G][RP][D]
-
+  const int rec = (G + 2) * D;  // one step's k, v, q_0 .. q_{G-1} (fp32)
   const int unit = blockIdx.x;  // b * Hkv + g
   const int b = unit / Hkv, g = unit % Hkv;
-  const int tid = threadIdx.x;
-  const __nv_bfloat16* kp = k + (size_t)unit * steps * D;
-  const __nv_bfloat16* vp = v + (size_t)unit * steps * D;
+  const int c = threadIdx.x;    // state column
+  const __nv_bfloat16* kp = k + (size_t)unit * steps * D + c;
+  const __nv_bfloat16* vp = v + (size_t)unit * steps * D + c;
   const size_t qh0 = (size_t)b * Hq + (size_t)g * G;  // first query head of the group
+  const __nv_bfloat16* qp = q + qh0 * steps * D + c;
+  __nv_bfloat16* op = o + qh0 * steps * D + c;
 
-  // element e of step t's (k, v, q_0..q_{G-1}) record
-  auto fetch = [&](int t, int e) -> float {
-    if (e < D) return __bfloat162float(kp[(size_t)t * D + e]);
-    if (e < 2 * D) return __bfloat162float(vp[(size_t)t * D + e - D]);
-    const int h = (e - 2 * D) / D, c = (e - 2 * D) % D;
-    return __bfloat162float(q[((qh0 + h) * steps + t) * D + c]);
+  // step t's record element c of every row -> registers (the launcher picks
+  // GB so that G <= kMaxG)
+  constexpr int kMaxG = GB == 8 ? kMaxGroup : 2 * GB - 1;
+  __nv_bfloat16 pre[2 + kMaxG];
+  auto fetch = [&](int t) {
+    pre[0] = kp[(size_t)t * D];
+    pre[1] = vp[(size_t)t * D];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h)
+      if (h < G) pre[2 + h] = qp[((size_t)h * steps + t) * D];
   };
-  constexpr int kMaxPer = (kMaxGroup + 2) * 128 / kDecodeThreads;  // elements per thread per step
-  float nxt[kMaxPer];
-  const int nper = (per_step + kDecodeThreads - 1) / kDecodeThreads;
+  auto stash = [&](float* buf) {
 #pragma unroll
-  for (int u = 0; u < kMaxPer; ++u) {
-    const int e = tid + u * kDecodeThreads;
-    if (u < nper && e < per_step) nxt[u] = fetch(0, e);
-  }
+    for (int j = 0; j < 2 + kMaxG; ++j)
+      if (j < 2 + G) buf[j * D + c] = __bfloat162float(pre[j]);
+  };
 
-  const int tx = tid % TPR, ty = tid / TPR;
-  const int col = 4 * tx;
-  float4* Su = reinterpret_cast<float4*>(S + (size_t)unit * D * D);
-  float4 srow[RPT];
+  float s[D];
+  const float* Su = S + (size_t)unit * D * D + c;
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) srow[r] = __ldcs(Su + (size_t)(ty + r * RP) * TPR + tx);
+  for (int r = 0; r < D; ++r) s[r] = __ldcs(Su + (size_t)r * D);
+  fetch(0);
+  stash(sh);
+  __syncthreads();
 
   for (int t = 0; t < steps; ++t) {
-    __syncthreads();  // the previous step is done with tok and red
+    const float* buf = sh + (size_t)(t & 1) * rec;
+    if (t + 1 < steps) fetch(t + 1);  // in flight while this step computes
+    const float vc = buf[D + c];
+    const float4* k4 = reinterpret_cast<const float4*>(buf);
+    for (int hb = 0; hb < G; hb += GB) {
+      float acc[GB][2];  // two partial sums per head (even / odd row quads): shorter chains
 #pragma unroll
-    for (int u = 0; u < kMaxPer; ++u) {
-      const int e = tid + u * kDecodeThreads;
-      if (u < nper && e < per_step) tok[e] = nxt[u];
-    }
-    __syncthreads();
-    if (t + 1 < steps) {  // next step's record, in flight while this one computes
+      for (int j = 0; j < GB; ++j) acc[j][0] = acc[j][1] = 0.f;
+      const float4* q4 = reinterpret_cast<const float4*>(buf + (size_t)(2 + hb) * D);
+      const int nh = G - hb;  // heads left; a short last pass is predicated
 #pragma unroll
-      for (int u = 0; u < kMaxPer; ++u) {
-        const int e = tid + u * kDecodeThreads;
-        if (u < nper && e < per_step) nxt[u] = fetch(t + 1, e);
+      for (int r4 = 0; r4 < D / 4; ++r4) {
+        if (hb == 0) {
+          const float4 kk = k4[r4];
+          s[4 * r4 + 0] = fmaf(kk.x, vc, s[4 * r4 + 0]);
+          s[4 * r4 + 1] = fmaf(kk.y, vc, s[4 * r4 + 1]);
+          s[4 * r4 + 2] = fmaf(kk.z, vc, s[4 * r4 + 2]);
+          s[4 * r4 + 3] = fmaf(kk.w, vc, s[4 * r4 + 3]);
+        }
+#pragma unroll
+        for (int j = 0; j < GB; ++j) {
+          if (j < nh) {
+            const float4 qq = q4[(size_t)j * (D / 4) + r4];
+            float& a = acc[j][r4 & 1];
+            a = fmaf(qq.x, s[4 * r4 + 0], a);
+            a = fmaf(qq.y, s[4 * r4 + 1], a);
+            a = fmaf(qq.z, s[4 * r4 + 2], a);
+            a = fmaf(qq.w, s[4 * r4 + 3], a);
+          }
+        }
       }
-    }
-    const float4 vv = make_float4(tok[D + col], tok[D + col + 1], tok[D + col + 2], tok[D + col + 3]);
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const float kr = tok[ty + r * RP];
-      srow[r].x = fmaf(kr, vv.x, srow[r].x);
-      srow[r].y = fmaf(kr, vv.y, srow[r].y);
-      srow[r].z = fmaf(kr, vv.z, srow[r].z);
-      srow[r].w = fmaf(kr, vv.w, srow[r].w);
+      for (int j = 0; j < GB; ++j)
+        if (j < nh)
+          op[((size_t)(hb + j) * steps + t) * D] = __float2bfloat16_rn(acc[j][0] + acc[j][1]);
     }
-    for (int h = 0; h < G; ++h) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float* qh = tok + 2 * D + h * D;
-#pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        const float qr = qh[ty + r * RP];
-        acc.x = fmaf(qr, srow[r].x, acc.x);
-        acc.y = fmaf(qr, srow[r].y, acc.y);
-        acc.z = fmaf(qr, srow[r].z, acc.z);
-        acc.w = fmaf(qr, srow[r].w, acc.w);
-      }
-      *reinterpret_cast<float4*>(red + ((size_t)h * RP + ty) * D + col) = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < G * D; e += kDecodeThreads) {
-      const int h = e / D, c = e % D;
-      float sum = 0.f;
-#pragma unroll
-      for (int y = 0; y < RP; ++y) sum += red[((size_t)h * RP + y) * D + c];
-      o[((qh0 + h) * steps + t) * D + c] = __float2bfloat16_rn(sum);
-    }
+    if (t + 1 < steps) stash(sh + (size_t)((t + 1) & 1) * rec);
+    __syncthreads();  // the next step's record is complete; this step's is no longer read
   }
+  float* Sw = S + (size_t)unit * D * D + c;
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) __stcs(Su + (size_t)(ty + r * RP) * TPR + tx, srow[r]);
+  for (int r = 0; r < D; ++r) __stcs(Sw + (size_t)r * D, s[r]);
 }
 
-template <int D>
-cudaError_t launch_decode_steps_d(float* S, const void* q, const void* k, const void* v, void* o,
-                                  int B, int Hq, int Hkv, int steps, cudaStream_t stream) {
-  constexpr int RP = kDecodeThreads / (D / 4);
+template <int D, int GB>
+cudaError_t launch_decode_steps_gb(float* S, const void* q, const void* k, const void* v, void* o,
+                                   int B, int Hq, int Hkv, int steps, cudaStream_t stream) {
   const int G = Hq / Hkv;
-  const size_t smem = sizeof(float) * ((size_t)(G + 2) * D + (size_t)G * RP * D);
-  cudaError_t e = cudaFuncSetAttribute(decode_steps_kernel<D>,
+  const size_t smem = sizeof(float) * 2 * (size_t)(G + 2) * D;
+  cudaError_t e = cudaFuncSetAttribute(decode_steps_kernel<D, GB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_steps_kernel<D><<<(unsigned)(B * Hkv), kDecodeThreads, smem, stream>>>(
+  decode_steps_kernel<D, GB><<<(unsigned)(B * Hkv), D, smem, stream>>>(
       S, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), Hq, Hkv, steps);
   return cudaGetLastError();
+}
+
+// Heads per pass: the largest power of two up to min(G, 8), so groups of 1, 2,
+// 4 and 8 heads take one pass with no predicated-off work.
+template <int D>
+cudaError_t launch_decode_steps_d(float* S, const void* q, const void* k, const void* v, void* o,
+                                  int B, int Hq, int Hkv, int steps, cudaStream_t stream) {
+  const int G = Hq / Hkv;
+  if (G >= 8) return launch_decode_steps_gb<D, 8>(S, q, k, v, o, B, Hq, Hkv, steps, stream);
+  if (G >= 4) return launch_decode_steps_gb<D, 4>(S, q, k, v, o, B, Hq, Hkv, steps, stream);
+  if (G >= 2) return launch_decode_steps_gb<D, 2>(S, q, k, v, o, B, Hq, Hkv, steps, stream);
+  return launch_decode_steps_gb<D, 1>(S, q, k, v, o, B, Hq, Hkv, steps, stream);
 }
 
 // 512 threads (8 rows of S per thread at d = 128): more of each state in flight
