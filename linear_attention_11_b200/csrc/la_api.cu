@@ -65,6 +65,8 @@ la_status check_shape(int B, int Hq, int Hkv, int64_t N, int d) {
   return LA_OK;
 }
 
+constexpr double kQBytesHost = 128.0 * 128 * 2;  // one 128-row bf16 tile (Q or O)
+
 la_status plan_impl(int B, int Hq, int Hkv, int64_t N, int d, int chunk, int sms, la_plan* out) {
   la_status st = check_shape(B, Hq, Hkv, N, d);
   if (st != LA_OK) return st;
@@ -83,9 +85,14 @@ la_status plan_impl(int B, int Hq, int Hkv, int64_t N, int d, int chunk, int sms
   const int64_t nsub = G / HPT;
   // Pick the span count: the persistent chunk loop deals units * nspan items
   // (a span of one kv group, nsub tiles per chunk step) round-robin over the
-  // SMs; estimated time ~ rounds * (tiles per item + a per-item cost of about
-  // three tiles).
+  // SMs; estimated time in tile times ~ rounds * (tiles per item + a per-item
+  // cost of about three tiles), plus, with more than one span, the span-state
+  // pass over (nspan - 1) / nspan of K and V, at the whole GPU's bandwidth:
+  // its bytes / (bytes of one tile x SMs).
   const int64_t max_span = std::min<int64_t>(tiles, 4096);
+  const double kv_tile = 2.0 * T * kHeadDim * 2;                   // K and V of one chunk step
+  const double tile_bytes = 2.0 * kQBytesHost + kv_tile / (double)nsub;  // Q, O + K,V share
+  const double span_pass = (double)units * tiles * kv_tile / (tile_bytes * sms);
   int64_t best = 1;
   double best_cost = 1e300;
   for (int64_t ns = 1; ns <= max_span; ++ns) {
@@ -93,7 +100,8 @@ la_status plan_impl(int B, int Hq, int Hkv, int64_t N, int d, int chunk, int sms
     if (items > 0x7fffffff) break;
     const int64_t rounds = (items + sms - 1) / sms;
     const int64_t per = (tiles + ns - 1) / ns * nsub;
-    const double cost = (double)rounds * (double)(per + 3);
+    const double cost =
+        (double)rounds * (double)(per + 3) + span_pass * (double)(ns - 1) / (double)ns;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = ns;
