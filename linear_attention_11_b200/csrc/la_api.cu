@@ -250,8 +250,23 @@ bool stage_states_pays(const PrefillGeometry& g) {
   return g.nspan == 1 && (int64_t)g.tiles_total * (g.G / g.heads_per_tile) <= 4;
 }
 
+int span_parts(const la_plan& plan, int units, int sms) {
+  if (plan.nspan <= 1) return 1;
+  // the forward computes the states of the first nspan - 1 spans; cut each
+  // into parts until those CTAs cover the SMs, keeping two tiles per part
+  const int64_t ctas = (int64_t)units * (plan.nspan - 1);
+  int64_t parts = (sms + ctas - 1) / ctas;
+  parts = std::min<int64_t>(parts, std::max<int64_t>(1, plan.tiles_total / (2 * plan.nspan)));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(parts, 64));
+}
+
 size_t forward_workspace_bytes(const la_plan& plan) {
-  return plan.nspan == 1 ? 256 : (size_t)plan.workspace_bytes;
+  if (plan.nspan == 1) return 256;
+  int sms = 0;
+  if (!device_info(nullptr, &sms)) return (size_t)plan.workspace_bytes;
+  const int64_t per_seq = (int64_t)plan.nspan * kHeadDim * kHeadDim * (int64_t)sizeof(float);
+  const int units = (int)(plan.workspace_bytes / per_seq);
+  return (size_t)plan.workspace_bytes * (size_t)span_parts(plan, units, sms);
 }
 
 la_status forward_persistent(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
@@ -273,7 +288,7 @@ la_status forward_persistent(const la_bf16* q, const la_bf16* k, const la_bf16* 
 
 la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
                            float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
-                           void* workspace, cudaStream_t stream) {
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (plan.nspan == 1) return forward_persistent(q, k, v, o, S, B, Hq, Hkv, N, plan, stream);
   // Span states of all spans but the last (the last one only feeds the final
   // state, which the chunk loop's last-span items write from tensor memory),
@@ -289,9 +304,18 @@ la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v,
     return LA_ERR_CUDA;
   PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
   float* ws = static_cast<float*>(workspace);
-  cudaError_t e = launch_span_states(g, maps.k, maps.v, ws, status, stream, true);
-  if (e == cudaSuccess) e = launch_state_scan(ws, S, B * Hkv, plan.nspan, kHeadDim, stream, 0, false);
-  if (e == cudaSuccess) e = launch_prefill_persist(g, maps, ws, S, status, sms, stream, true, false);
+  // span parts, as many as wanted and as the workspace holds
+  int parts = span_parts(plan, B * Hkv, sms);
+  const size_t per_part = (size_t)plan.workspace_bytes;
+  if (per_part == 0 || workspace_bytes < per_part) return LA_ERR_WORKSPACE;
+  parts = (int)std::min<size_t>((size_t)parts, workspace_bytes / per_part);
+  const int nsub_spans = plan.nspan * parts;
+  cudaError_t e = launch_span_states(g, maps.k, maps.v, ws, status, stream, true, parts);
+  if (e == cudaSuccess)
+    e = launch_state_scan(ws, S, B * Hkv, nsub_spans, kHeadDim, stream, 0,
+                          nsub_spans - parts);
+  if (e == cudaSuccess)
+    e = launch_prefill_persist(g, maps, ws, S, status, sms, stream, true, false, 1, 0, 0, parts);
   return from_cuda(e);
 }
 
@@ -455,7 +479,7 @@ LA_EXPORT la_status la_forward_ws(const la_bf16* q, const la_bf16* k, const la_b
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       workspace_bytes < forward_workspace_bytes(plan))
     return LA_ERR_WORKSPACE;
-  return forward_dispatch(q, k, v, o, S, B, Hq, Hkv, N, plan, workspace,
+  return forward_dispatch(q, k, v, o, S, B, Hq, Hkv, N, plan, workspace, workspace_bytes,
                           static_cast<cudaStream_t>(stream));
 }
 

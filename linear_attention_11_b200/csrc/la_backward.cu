@@ -134,7 +134,8 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
   const size_t sq_bytes = round((size_t)B * Hkv * dd * 4);
   const size_t sm_bytes = round((size_t)B * Hq * dd * 4);
   const size_t part_bytes = round((size_t)B * Hq * N * d * 2);
-  const size_t wsq = round(forward_workspace_bytes(plan_q));
+  const size_t wsq_bytes = forward_workspace_bytes(plan_q);
+  const size_t wsq = round(wsq_bytes);
   const size_t wsm = plan_m.nspan > 1 ? round((size_t)plan_m.workspace_bytes) : 0;
   const size_t total = sq_bytes + 2 * sm_bytes + part_bytes + wsq + wsm;
   char* pool = nullptr;
@@ -159,7 +160,8 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
 
   // ---- dq: the forward pass on (dO, V, K) from S0^T
   cu(place_states(S0, S_q, B, Hkv, 1, d, 1, s));
-  if (st == LA_OK) st = forward_dispatch(dO, v, k, dq, S_q, B, Hq, Hkv, N, plan_q, ws_q, s);
+  if (st == LA_OK)
+    st = forward_dispatch(dO, v, k, dq, S_q, B, Hq, Hkv, N, plan_q, ws_q, wsq_bytes, s);
 
   // ---- dv, then dk: anti-causal walks per query head, summed over groups.
   // One state serves both: D = sum_t q_t^T do_t over the later chunks (dv

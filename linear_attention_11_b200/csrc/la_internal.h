@@ -39,15 +39,19 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, i
 bool make_tmap_state(CUtensorMap* map, const void* base, int64_t units);
 
 // skip_last: spans 0 .. nspan-2 only (the last span's state is needed only
-// for the final state, which the chunk loop then writes).
+// for the final state, which the chunk loop then writes).  parts: each span
+// cut into `parts` sub-spans computed by separate CTAs (more CTAs when there
+// are few sequences and spans); ws then holds nspan * parts states per
+// sequence, in order.
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
-                               cudaStream_t stream, bool skip_last = false);
+                               cudaStream_t stream, bool skip_last = false, int parts = 1);
 // Persistent chunk loop: min(B*Hkv*nspan, num_ctas) CTAs walk the items (one
 // span of one (batch, kv head) sequence each, every query head of the group)
 // round-robin.  ws: entering state of item bg * nspan + j (nullptr: zero);
 // s_out (nullable): final states [B*Hkv, d, d], written by the items of the
-// last spans in walk order; with nspan == 1 it may be ws itself.  dependent:
+// last spans in walk order; with nspan == 1 it may be ws itself.  ws_stride:
+// entering state of item it at ws[it * ws_stride] (spans cut into parts).  dependent:
 // launched as a programmatic dependent of the previous kernel in the stream.
 // stage_states (honoured at tile 64, nspan == 1, forward, s_out null or ws):
 // states pass through shared memory by bulk tensor copies, for short items
@@ -59,31 +63,37 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
                                    cudaStream_t stream, bool dependent, bool stage_states,
-                                   int qdiv = 1, int reverse = 0, int transpose_in = 0);
+                                   int qdiv = 1, int reverse = 0, int transpose_in = 0,
+                                   int ws_stride = 1);
 // Whether staging the states pays for a one-span plan: the staged layout
 // (two Q slots, output through a Q slot) streams tiles slower, so only items
 // of at most four tiles use it.
 bool stage_states_pays(const PrefillGeometry& g);
 size_t fused_workspace_bytes(int B, int Hkv, int nspan);
+// Sub-spans per span for the span-state pass of the forward: enough CTAs for
+// the SMs when sequences x spans are few (1 when nspan == 1).
+int span_parts(const la_plan& plan, int units, int sms);
 // Workspace bytes la_forward_ws needs for `plan` (never zero): the span
-// states, or nothing (a nominal 256 bytes) with one span per sequence, which
-// runs as the persistent chunk loop alone with the state read and written in
-// place.
+// (sub-span) states, or nothing (a nominal 256 bytes) with one span per
+// sequence, which runs as the persistent chunk loop alone with the state read
+// and written in place.
 size_t forward_workspace_bytes(const la_plan& plan);
 // The whole prefill (validated arguments): one persistent chunk-loop launch
 // when the plan has one span per sequence, else span states, scan and the
-// persistent chunk loop; workspace of forward_workspace_bytes bytes.
+// persistent chunk loop; the span parts are lowered to what workspace_bytes
+// holds (at least the plan's own workspace_bytes).
 la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
                            float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
-                           void* workspace, cudaStream_t stream);
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
 cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
                                  void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);
 // reverse: ws[j] <- S0 + sum_{i>j} ws[i] (the state entering span j of a
-// backwards walk); S receives S0 + sum_i ws[i] either way.  write_final =
-// false (forward only): ws[nspan-1] is not read and S is only read (S0).
+// backwards walk); S receives S0 + sum_i ws[i] either way.  nread < nspan
+// (forward only): entries from nread on are not read, ws[nread] receives its
+// entering state and S is only read (S0); nread < 0 means nspan.
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
-                              cudaStream_t stream, int reverse = 0, bool write_final = true);
+                              cudaStream_t stream, int reverse = 0, int nread = -1);
 cudaError_t launch_decode(float* S, const void* q, const void* k, const void* v, void* o, int B,
                           int Hq, int Hkv, int d, cudaStream_t stream);
 cudaError_t launch_decode_steps(float* S, const void* q, const void* k, const void* v, void* o,

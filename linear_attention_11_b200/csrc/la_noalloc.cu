@@ -82,6 +82,6 @@ LA_EXPORT la_status la_forward_noalloc(const la_bf16* q, const la_bf16* k, const
   }
   void* ws = scratch_on_current_device();
   if (!ws) return LA_ERR_CUDA;
-  return la::forward_dispatch(q, k, v, o, S, B, Hq, Hkv, N, plan, ws,
+  return la::forward_dispatch(q, k, v, o, S, B, Hq, Hkv, N, plan, ws, kScratchBytes,
                               static_cast<cudaStream_t>(stream));
 }

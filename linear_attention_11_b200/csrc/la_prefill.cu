@@ -29,7 +29,7 @@ struct SpanParams {
   float* ws;
   unsigned* status;
   int nspan, tiles_total;
-  int nrun;  // spans computed per (batch, kv head): nspan, or nspan - 1 (the last one skipped)
+  int nrun;  // spans computed per (batch, kv head): the first nrun of the nspan
 };
 
 template <int T, int STAGES>
@@ -173,10 +173,12 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
-                               cudaStream_t stream, bool skip_last) {
-  const int nrun = g.nspan - (skip_last ? 1 : 0);
+                               cudaStream_t stream, bool skip_last, int parts) {
+  if (parts < 1) return cudaErrorInvalidValue;
+  const int nparts = g.nspan * parts;                        // sub-spans per sequence
+  const int nrun = (g.nspan - (skip_last ? 1 : 0)) * parts;  // of them computed
   if (nrun <= 0) return cudaSuccess;
-  SpanParams p{ws, status, g.nspan, g.tiles_total, nrun};
+  SpanParams p{ws, status, nparts, g.tiles_total, nrun};
   const dim3 grid((unsigned)(g.B * g.Hkv * nrun));
   cudaError_t e;
   if (g.tile == 64) {

@@ -52,6 +52,7 @@ struct PersistParams {
   int qdiv;          // query rows of head h come from head h / qdiv of the query tensor
   int reverse;       // anti-causal (s >= t): each span walked from its end
   int transpose_in;  // entering states read transposed (register path)
+  int ws_stride;     // entering state of item it at ws[it * ws_stride]
 };
 
 // kStage: entering and final states pass through a 64 KB fp32 tile in shared
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(320, 1)
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
         if (!staged && p.ws && nx >= 0)  // the next item's entering state, read at its end
-          prefetch_l2_bulk(p.ws + (size_t)nx * kDD, (uint32_t)(kDD * sizeof(float)));
+          prefetch_l2_bulk(p.ws + (size_t)nx * p.ws_stride * kDD, (uint32_t)(kDD * sizeof(float)));
         for (int n = 0; n < te - tb; ++n, ++gc) {
           const int cs = chunk_at(tb, te, n);
           const int s = gc % KVST;
@@ -351,10 +352,10 @@ __global__ void __launch_bounds__(320, 1)
     // This warpgroup's half of row r of item it's entering state -> tensor
     // memory and the bf16 copy; then signal the state version.
     auto load_state = [&](int it) {
+      const float* st = p.ws ? p.ws + (size_t)it * p.ws_stride * kDD : nullptr;
       const float4* src =
-          p.ws ? reinterpret_cast<const float4*>(p.ws + (size_t)it * kDD + (size_t)r * kHeadDim)
-               : nullptr;
-      const float* col = p.ws ? p.ws + (size_t)it * kDD + r : nullptr;  // column r (transposed)
+          st ? reinterpret_cast<const float4*>(st + (size_t)r * kHeadDim) : nullptr;
+      const float* col = st ? st + r : nullptr;  // column r (transposed)
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb) {
         const int blk = blk0 + bb;
@@ -663,19 +664,20 @@ cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& ma
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
                                    cudaStream_t stream, bool dependent, bool stage_states,
-                                   int qdiv, int reverse, int transpose_in) {
+                                   int qdiv, int reverse, int transpose_in, int ws_stride) {
   if (s_out && s_out == ws && g.nspan != 1) return cudaErrorInvalidValue;
   const int nsub = g.G / g.heads_per_tile;
   const int64_t items = (int64_t)g.B * g.Hkv * g.nspan;
   if (items <= 0 || items > 0x7fffffff || num_ctas <= 0) return cudaErrorInvalidValue;
-  if (qdiv < 1 || (transpose_in && s_out == ws && s_out)) return cudaErrorInvalidValue;
-  PersistParams p{ws,    s_out, status,        g.Hq,       g.Hkv, g.G,     nsub,
-                  g.nspan, g.tiles_total, (int)items, qdiv, reverse, transpose_in};
+  if (qdiv < 1 || ws_stride < 1 || (transpose_in && s_out == ws && s_out))
+    return cudaErrorInvalidValue;
+  PersistParams p{ws,      s_out,         status,     g.Hq, g.Hkv,   g.G,          nsub,
+                  g.nspan, g.tiles_total, (int)items, qdiv, reverse, transpose_in, ws_stride};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
   // Staged states (room for the tile: two Q slots, output through the Q
   // slot); otherwise the smem goes to the rings.
-  if (stage_states && !reverse && !transpose_in && g.tile == 64 && g.nspan == 1 && ws &&
-      (!s_out || s_out == ws)) {
+  if (stage_states && !reverse && !transpose_in && ws_stride == 1 && g.tile == 64 &&
+      g.nspan == 1 && ws && (!s_out || s_out == ws)) {
     CUtensorMap map_s;
     if (!make_tmap_state(&map_s, ws, (int64_t)g.B * g.Hkv)) return cudaErrorInvalidValue;
     return launch_persist<64, 2, 2, false, true>(grid, stream, maps, map_s, p, dependent);

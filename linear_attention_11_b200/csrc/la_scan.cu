@@ -4,8 +4,8 @@
 // where K_i^T V_i is span i's contribution; the state after the last span is
 // the final state S0 + K^T V ("MiniMax-01与Lightning Attention", section 2.2,
 // kv_sum over the whole sequence).  When the chunk loop writes the final state
-// itself, the last span's K^T V is never computed and only the entering
-// states are written.  Elementwise fp32 adds, HBM/L2-bound: one
+// itself, the last span's K^T V is never computed (nread < nspan) and only the
+// entering states are written.  Elementwise fp32 adds, HBM/L2-bound: one
 // thread owns one float4 of the d x d matrix of one unit and walks the spans
 // in order, loading eight spans ahead to keep loads in flight.  Launched as a
 // programmatic dependent of the span-state kernel: it lets the chunk-loop
@@ -24,7 +24,7 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
 
 __global__ void __launch_bounds__(256)
     state_scan_kernel(float4* __restrict__ ws, float4* __restrict__ S, int nspan, int n4,
-                      int blocks_per_unit, int reverse, int write_final) {
+                      int blocks_per_unit, int reverse, int nread) {
   griddep_launch_dependents();  // the chunk-loop kernel may start its copies
   griddep_wait();               // the span states are complete
   const size_t unit = blockIdx.x / blocks_per_unit;
@@ -41,9 +41,8 @@ __global__ void __launch_bounds__(256)
     if (S) S[unit * n4 + p] = carry;
     return;
   }
-  // without the final state the last span's own state is neither needed nor
-  // computed: only its entering state is written
-  const int nread = write_final ? nspan : nspan - 1;
+  // nread < nspan: entries from nread on were not computed (they only feed
+  // the final state); the entering state of entry nread is written, no final
   int j = 0;
   for (; j + 8 <= nread; j += 8) {
     float4 x[8];
@@ -60,8 +59,8 @@ __global__ void __launch_bounds__(256)
     w[(size_t)j * n4] = carry;
     carry = add4(carry, x);
   }
-  if (!write_final) {
-    w[(size_t)(nspan - 1) * n4] = carry;
+  if (nread < nspan) {
+    w[(size_t)nread * n4] = carry;
     return;
   }
   if (S) S[unit * n4 + p] = carry;
@@ -70,8 +69,9 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
-                              cudaStream_t stream, int reverse, bool write_final) {
-  if (reverse && !write_final) return cudaErrorInvalidValue;
+                              cudaStream_t stream, int reverse, int nread) {
+  if (nread < 0) nread = nspan;
+  if (nread < 1 || nread > nspan || (reverse && nread != nspan)) return cudaErrorInvalidValue;
   const int n4 = d * d / 4;
   const int bpu = (n4 + 255) / 256;
   cudaLaunchConfig_t cfg = {};
@@ -85,8 +85,7 @@ cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, state_scan_kernel, reinterpret_cast<float4*>(ws),
-                            reinterpret_cast<float4*>(S), nspan, n4, bpu, reverse,
-                            write_final ? 1 : 0);
+                            reinterpret_cast<float4*>(S), nspan, n4, bpu, reverse, nread);
 }
 
 }  // namespace la

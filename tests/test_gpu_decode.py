@@ -71,7 +71,11 @@ def _stack_steps(w, steps, B=None):
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,d,steps", [(3, 4, 2, 128, 5), (2, 6, 3, 64, 17), (1, 32, 1, 128, 3),
-                                               (4, 8, 8, 128, 1), (2, 2, 1, 64, 40)])
+                                               (4, 8, 8, 128, 1), (2, 2, 1, 64, 40),
+                                               # groups of 3, 6, 12: passes of 2, 4, 8 heads
+                                               # with a shorter last pass
+                                               (2, 9, 3, 128, 7), (1, 12, 2, 128, 9),
+                                               (1, 24, 2, 64, 6)])
 def test_decode_steps_matches_recurrence(la, B, Hq, Hkv, d, steps):
     w = synth.Decode("t", B, Hq, Hkv, d, steps, 13)
     S0 = synth.decode_state(w)

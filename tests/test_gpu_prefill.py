@@ -400,3 +400,25 @@ def test_multi_token_decode_shape(la, chunk):
     assert la.la_device_status()[1] == 0
     assert_bf16_close(o.cpu(), ref_o, "multi-token O")
     assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
+
+
+def test_span_parts(la):
+    """Few sequences and spans (64 kv heads, 2 spans): each span's state is
+    computed by several CTAs (sub-spans) and the scan folds them in; entering
+    states, outputs and the final state against the oracle."""
+    B, Hq, Hkv, N, chunk = 4, 16, 16, 2048, 64
+    plan = la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk)
+    assert plan.nspan == 2
+    assert la.api.la_forward_workspace_bytes(B, Hq, Hkv, N, 128, chunk) > plan.workspace_bytes
+    q, k, v = _qkv(B, Hq, Hkv, N, seed=1201)
+    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(1202)) / 128
+    ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy(), o_dtype=np.float32)
+    qd, kd, vd = _cuda(q, k, v)
+    S = S0.to(DEV)
+    o = la.la_forward_state(qd, kd, vd, S=S, chunk=chunk)
+    o0 = la.la_forward(qd, kd, vd, chunk=chunk)
+    torch.cuda.synchronize()
+    assert la.la_device_status()[1] == 0
+    assert_bf16_close(o.cpu(), ref_o, "O")
+    assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
+    assert_bf16_close(o0.cpu(), oracle.recurrent(q, k, v, o_dtype=np.float32)[0], "O from zero")
