@@ -45,14 +45,13 @@ namespace la {
 namespace {
 
 struct PersistParams {
-  const float* ws;  // entering state of item it at ws[it] (d x d fp32 each); nullptr: zero
+  const float* ws;  // entering state of item it at ws[it * ws_stride] (d x d fp32); nullptr: zero
   float* s_out;     // final state of sequence bg at s_out[bg], written by its last span's item
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total, items;
   int qdiv;          // query rows of head h come from head h / qdiv of the query tensor
-  int reverse;       // anti-causal (s >= t): each span walked from its end
-  int transpose_in;  // entering states read transposed (register path)
-  int ws_stride;     // entering state of item it at ws[it * ws_stride]
+  int transpose_in;  // entering states read transposed (register path, anti-causal walks)
+  int ws_stride;     // spans cut into this many sub-spans in the workspace
 };
 
 // kStage: entering and final states pass through a 64 KB fp32 tile in shared
@@ -206,7 +205,7 @@ __global__ void __launch_bounds__(320, 1)
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
-        if (!staged && p.ws && nx >= 0)  // the next item's entering state, read at its end
+        if (!staged && p.ws && nx >= 0)  // next item's entering state, read at this item's end
           prefetch_l2_bulk(p.ws + (size_t)nx * p.ws_stride * kDD, (uint32_t)(kDD * sizeof(float)));
         for (int n = 0; n < te - tb; ++n, ++gc) {
           const int cs = chunk_at(tb, te, n);
@@ -671,8 +670,8 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
   if (items <= 0 || items > 0x7fffffff || num_ctas <= 0) return cudaErrorInvalidValue;
   if (qdiv < 1 || ws_stride < 1 || (transpose_in && s_out == ws && s_out))
     return cudaErrorInvalidValue;
-  PersistParams p{ws,      s_out,         status,     g.Hq, g.Hkv,   g.G,          nsub,
-                  g.nspan, g.tiles_total, (int)items, qdiv, reverse, transpose_in, ws_stride};
+  PersistParams p{ws,      s_out,         status,     g.Hq, g.Hkv,        g.G,      nsub,
+                  g.nspan, g.tiles_total, (int)items, qdiv, transpose_in, ws_stride};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
   // Staged states (room for the tile: two Q slots, output through the Q
   // slot); otherwise the smem goes to the rings.
