@@ -42,6 +42,10 @@ sys.path.insert(0, ROOT)
 
 from linear_attention_11_b200 import synth  # noqa: E402
 
+# the headline metric: prefill Mtok/s (value), its roofline fraction
+# (roofline), and the decode step's GB/s (decode)
+METRIC = "causal lightning-attn prefill Mtok/s & % roofline; decode-step GB/s, 1 B200"
+
 WORKLOADS = {"gqa32k": synth.GQA_32K, "mha8k": synth.MHA_8K, "long1m": synth.LONG_1M}
 
 
@@ -215,6 +219,13 @@ def cpu_baseline(w, sample_tokens=None, target_s=10.0):
 
 
 # ------------------------------------------------------------------ arms
+def bench_config(w, chunk, world):
+    """The workload as both arms name it (N ranks: N replicas of it)."""
+    return {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N, "chunk": chunk,
+            "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -234,12 +245,11 @@ def run_reference(args, w):
             per.append(time.perf_counter() - t0)
     dt = sum(per)
     value = w.B * n * steps / dt / 1e6
-    line = {"impl": "reference", "metric": "causal lightning-attn prefill throughput",
+    line = {"impl": "reference", "metric": METRIC,
             "value": value, "unit": "Mtok/s", "n_gpus": args.gpus, "steps": steps,
             "warmup": warm, "ms_per_step": 1e3 * dt / steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N,
-                       "chunk": args.chunk or w.chunks[0], "parallelism": "replicas"},
+            "config": bench_config(w, args.chunk or w.chunks[0], args.gpus),
             "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": cores, "kind": "oracle",
                              "sample": f"each step: the first {n} tokens of the workload "
                                        f"(B={w.B}, all {w.Hq} query heads), fp64 recurrent form"},
@@ -462,13 +472,11 @@ def run_ours(args, w):
                     "tolerance of the oracle, not bitwise equal to single steps"}
 
     line = {
-        "metric": "causal lightning-attn prefill throughput (Mtok/s); decode-step GB/s",
+        "metric": METRIC,
         "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": B * world, "seq_len": N, "chunk": chunk,
-                   "Hq": Hq, "Hkv": Hkv, "d": d, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (no flush)"},
+        "config": bench_config(w, chunk, world),
         "clocks": clocks,
         "gpu_launches": 3 * args.steps,  # span states, scan, chunk loop per step
         "roofline": roofline,
