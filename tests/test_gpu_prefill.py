@@ -422,3 +422,50 @@ def test_span_parts(la):
     assert_bf16_close(o.cpu(), ref_o, "O")
     assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
     assert_bf16_close(o0.cpu(), oracle.recurrent(q, k, v, o_dtype=np.float32)[0], "O from zero")
+
+
+# ------------------------------------------------------------------ degenerate inputs
+def test_empty_inputs_are_rejected(la):
+    """N = 0 or B = 0: nothing to compute; the ABI rejects the shape."""
+    for shape in ((1, 2, 0, 128), (0, 2, 64, 128)):
+        q = torch.zeros(shape, dtype=torch.bfloat16, device=DEV)
+        with pytest.raises(la.LAError) as e:
+            la.la_forward(q, q.clone(), q.clone(), chunk=64)
+        assert e.value.code == 1
+    S = torch.zeros(0, 1, 128, 128, dtype=torch.float32, device=DEV)
+    qt = torch.zeros(0, 1, 128, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(la.LAError) as e:
+        la.la_decode_step(S, qt, qt.clone(), qt.clone())
+    assert e.value.code == 1
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,chunk", [(2, 8, 2, 1000, 64), (1, 2, 2, 300, 128), (200, 4, 2, 64, 64)])
+def test_zero_keys_leave_only_the_state_term(la, B, Hq, Hkv, N, chunk):
+    """K = 0: every score and every state update vanishes, so O = Q S0 and
+    the final state is S0 bit for bit (on every path: span scheme, one launch,
+    staged states)."""
+    q, _, v = _qkv(B, Hq, Hkv, N, seed=1301 + N)
+    k = torch.zeros(B, Hkv, N, 128, dtype=torch.bfloat16)
+    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(1302)) / 128
+    ref_o, _ = oracle.recurrent(q, k, v, S0=S0.double().numpy(), o_dtype=np.float32)
+    qd, kd, vd = _cuda(q, k, v)
+    S = S0.to(DEV)
+    o = la.la_forward_state(qd, kd, vd, S=S, chunk=chunk)
+    torch.cuda.synchronize()
+    assert_bf16_close(o.cpu(), ref_o, "O = Q S0")
+    assert torch.equal(S.cpu(), S0)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,chunk", [(2, 8, 2, 1000, 64), (200, 4, 2, 64, 64)])
+def test_zero_queries_give_zero_output(la, B, Hq, Hkv, N, chunk):
+    """Q = 0: O is exactly zero; the state still takes every K^T V."""
+    _, k, v = _qkv(B, Hq, Hkv, N, seed=1401 + N)
+    q = torch.zeros(B, Hq, N, 128, dtype=torch.bfloat16)
+    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(1402)) / 128
+    _, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy())
+    qd, kd, vd = _cuda(q, k, v)
+    S = S0.to(DEV)
+    o = la.la_forward_state(qd, kd, vd, S=S, chunk=chunk)
+    torch.cuda.synchronize()
+    assert not torch.any(o)
+    assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
