@@ -226,6 +226,28 @@ la_status la_prefill_main(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, 
                           const la_plan *plan, la_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Sequence sharding: one sequence cut into nseg consecutive segments (one per
+ * GPU, say).  The state entering segment r is S0 + sum_{i<r} K_i^T V_i (the
+ * state is the whole resume point of the recurrence, [MX01] section 4.1,
+ * "Streaming"; K^T V of a segment is its kv_sum, section 2.2).  Each holder
+ * of a segment computes its K^T V, the nseg states are exchanged (an
+ * all-gather: B*Hkv*d*d*4 bytes per segment), each takes the prefix of the
+ * segments before its own, and runs la_forward_state from it.
+ *
+ * la_segment_state: S [B,Hkv,d,d] fp32 (device, 16-byte aligned, written)
+ * <- K^T V of this segment's k, v [B,Hkv,N,d] bf16; d = 128, chunk as
+ * la_forward.  Errors as la_forward.
+ * la_state_prefix: S [B,Hkv,d,d] <- S0 (nullable: 0) + sum_{i<seg} states[i],
+ * states [nseg,B,Hkv,d,d] fp32 contiguous (segment-major, as an all-gather
+ * lays it out), 0 <= seg < nseg; S may be S0 but must not overlap states.
+ * LA_ERR_INVALID_ARG on bad sizes or pointers.
+ * ---------------------------------------------------------------------- */
+la_status la_segment_state(const la_bf16 *k, const la_bf16 *v, float *S, int B, int Hkv,
+                           int64_t N, int d, int chunk, la_stream stream);
+la_status la_state_prefix(const float *states, const float *S0, float *S, int nseg, int seg,
+                          int B, int Hkv, int d, la_stream stream);
+
+/* ------------------------------------------------------------------------
  * Backward of the bf16 prefill (training).  For a loss with gradient dO
  * [B,Hq,N,d] on the output and dSf [B,Hkv,d,d] (nullable = 0) on the final
  * state, with S0 (nullable = 0) the initial state of the forward call:

@@ -16,6 +16,8 @@ from .api import (  # noqa: F401
     la_forward_f32,
     la_forward_host,
     la_forward_state,
+    la_segment_state,
+    la_state_prefix,
     la_status_string,
     library_path,
     load_library,

@@ -25,7 +25,7 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_E
 EXPORTS = ("la_status_string", "la_version", "la_forward", "la_forward_state",
            "la_forward_workspace_bytes", "la_forward_ws", "la_forward_noalloc",
            "la_forward_host", "la_prefill_fused_workspace_bytes", "la_prefill_fused",
-           "la_prefill_plan", "la_backward",
+           "la_prefill_plan", "la_backward", "la_segment_state", "la_state_prefix",
            "la_prefill_span_states", "la_prefill_scan", "la_prefill_main", "la_forward_f32",
            "la_decode_step", "la_decode_steps", "la_device_status", "la_selftest_wait",
            "la_shutdown")
@@ -67,6 +67,8 @@ def _declare(lib):
         "la_prefill_main": ([P, P, P, P, P, I, I, I, L, I, PP, P], I),
         "la_forward_f32": ([P, P, P, P, P, I, I, I, L, I, I, P], I),
         "la_backward": ([P, P, P, P, P, P, P, P, P, P, I, I, I, L, I, I, P], I),
+        "la_segment_state": ([P, P, P, I, I, L, I, I, P], I),
+        "la_state_prefix": ([P, P, P, I, I, I, I, I, P], I),
         "la_decode_step": ([P, P, P, P, P, I, I, I, I, P], I),
         "la_decode_steps": ([P, P, P, P, P, I, I, I, I, I, P], I),
         "la_device_status": ([ctypes.POINTER(ctypes.c_uint), I], I),
@@ -212,6 +214,26 @@ def la_prefill_main(q, k, v, o, ws, plan: la_plan, stream=None):
     _check("la_prefill_main", load_library().la_prefill_main(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ws), B, Hq, Hkv, N, d, ctypes.byref(plan),
         _stream(stream)))
+
+
+def la_segment_state(k, v, S=None, chunk: int = 64, stream=None):
+    """K^T V of one segment's k, v [B,Hkv,N,d] (bf16, CUDA) -> S [B,Hkv,d,d] fp32."""
+    B, Hkv, N, d = k.shape
+    if S is None:
+        S = torch.empty(B, Hkv, d, d, dtype=torch.float32, device=k.device)
+    _check("la_segment_state", load_library().la_segment_state(
+        _ptr(k), _ptr(v), _ptr(S), B, Hkv, N, d, chunk, _stream(stream)))
+    return S
+
+
+def la_state_prefix(states, seg: int, S0=None, S=None, stream=None):
+    """S0 (or 0) + sum of states[:seg]; states [nseg,B,Hkv,d,d] fp32 (CUDA)."""
+    nseg, B, Hkv, d, _ = states.shape
+    if S is None:
+        S = torch.empty(B, Hkv, d, d, dtype=torch.float32, device=states.device)
+    _check("la_state_prefix", load_library().la_state_prefix(
+        _ptr(states), _ptr(S0), _ptr(S), nseg, seg, B, Hkv, d, _stream(stream)))
+    return S
 
 
 def la_backward(q, k, v, dO, S0=None, dSf=None, want_dS0: bool = False, chunk: int = 64,

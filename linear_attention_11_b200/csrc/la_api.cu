@@ -592,6 +592,38 @@ LA_EXPORT la_status la_decode_steps(float* S, const la_bf16* q, const la_bf16* k
                                        static_cast<cudaStream_t>(stream)));
 }
 
+LA_EXPORT la_status la_segment_state(const la_bf16* k, const la_bf16* v, float* S, int B, int Hkv,
+                                     int64_t N, int d, int chunk, la_stream stream) {
+  la_plan plan;
+  la_status st = la_prefill_plan(B, Hkv, Hkv, N, d, chunk, &plan);
+  if (st != LA_OK) return st;
+  if (!k || !v || !S || !aligned16(k) || !aligned16(v) || !aligned16(S)) return LA_ERR_INVALID_ARG;
+  const size_t kbytes = (size_t)B * Hkv * N * d * 2, sbytes = (size_t)B * Hkv * d * d * 4;
+  if (overlap(S, sbytes, k, kbytes) || overlap(S, sbytes, v, kbytes)) return LA_ERR_INVALID_ARG;
+  unsigned* status = nullptr;
+  if (!device_info(&status, nullptr)) return LA_ERR_CUDA;
+  PrefillMaps maps;
+  if (!make_tmap_bf16(&maps.k, k, N, (int64_t)B * Hkv, plan.tile) ||
+      !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
+    return LA_ERR_CUDA;
+  plan.nspan = 1;  // the whole segment as one span: its state is K^T V, written into S
+  PrefillGeometry g = geometry(&plan, B, Hkv, Hkv, N);
+  return from_cuda(launch_span_states(g, maps.k, maps.v, S, status,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+LA_EXPORT la_status la_state_prefix(const float* states, const float* S0, float* S, int nseg,
+                                    int seg, int B, int Hkv, int d, la_stream stream) {
+  if (!states || !S || nseg < 1 || seg < 0 || seg >= nseg || B <= 0 || Hkv <= 0 || d <= 0 ||
+      d % 2 != 0)
+    return LA_ERR_INVALID_ARG;
+  if (!aligned16(states) || !aligned16(S) || (S0 && !aligned16(S0))) return LA_ERR_INVALID_ARG;
+  const size_t per = (size_t)B * Hkv * d * d;
+  if (overlap(S, per * 4, states, per * 4 * nseg) || (S0 && S0 != S && overlap(S, per * 4, S0, per * 4)))
+    return LA_ERR_INVALID_ARG;
+  return from_cuda(launch_state_prefix(states, S0, S, seg, per, static_cast<cudaStream_t>(stream)));
+}
+
 LA_EXPORT la_status la_device_status(unsigned int* flags, int clear) {
   if (!flags) return LA_ERR_INVALID_ARG;
   *flags = 0;

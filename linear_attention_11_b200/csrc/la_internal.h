@@ -94,6 +94,9 @@ cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& ma
 // entering state and S is only read (S0); nread < 0 means nspan.
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
                               cudaStream_t stream, int reverse = 0, int nread = -1);
+// S = S0 (nullable) + sum_{i < seg} states[i * per_seg_floats ...] (float4-wise).
+cudaError_t launch_state_prefix(const float* states, const float* S0, float* S, int seg,
+                                size_t per_seg_floats, cudaStream_t stream);
 cudaError_t launch_decode(float* S, const void* q, const void* k, const void* v, void* o, int B,
                           int Hq, int Hkv, int d, cudaStream_t stream);
 cudaError_t launch_decode_steps(float* S, const void* q, const void* k, const void* v, void* o,

@@ -88,4 +88,28 @@ cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
                             reinterpret_cast<float4*>(S), nspan, n4, bpu, reverse, nread);
 }
 
+namespace {
+
+// S[u] = S0[u] (or 0) + sum_{i < seg} states[i][u], one float4 per thread.
+__global__ void __launch_bounds__(256)
+    state_prefix_kernel(const float4* __restrict__ states, const float4* S0, float4* S,
+                        int seg, size_t per_seg4) {
+  const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= per_seg4) return;
+  float4 acc = S0 ? S0[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < seg; ++i) acc = add4(acc, states[(size_t)i * per_seg4 + e]);
+  S[e] = acc;
+}
+
+}  // namespace
+
+cudaError_t launch_state_prefix(const float* states, const float* S0, float* S, int seg,
+                                size_t per_seg_floats, cudaStream_t stream) {
+  const size_t n4 = per_seg_floats / 4;
+  state_prefix_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(states), reinterpret_cast<const float4*>(S0),
+      reinterpret_cast<float4*>(S), seg, n4);
+  return cudaGetLastError();
+}
+
 }  // namespace la
