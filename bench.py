@@ -345,8 +345,20 @@ def run_ours(args, w):
     wsf = torch.empty(fb, dtype=torch.uint8, device=dev)
     t_fused = ev_mean(lambda: la.api.la_prefill_fused(qd, kd, vd, o, None, wsf, chunk=chunk,
                                                       stream=stream))
+    # the same step captured once in a CUDA graph and replayed (launch costs
+    # of the host call removed): informational
+    gs = torch.cuda.Stream()
+    with torch.cuda.stream(gs):
+        la.la_forward(qd, kd, vd, o=o, chunk=chunk, stream=gs)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=gs):
+        la.la_forward(qd, kd, vd, o=o, chunk=chunk, stream=gs)
+    t_graph = ev_mean(graph.replay, 10)
+    del graph
     alternatives = {
         "two_pass_span_parallel_ms": 1e3 * t / args.steps,
+        "cuda_graph_replay_ms": 1e3 * t_graph,
         "sequential_chunk_loop_ms": 1e3 * t_seq,
         "single_pass_fused_ms": 1e3 * t_fused,
         "note": "sequential = one span per (batch, kv head): one CTA walks every chunk of "
