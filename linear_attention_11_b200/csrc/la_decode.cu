@@ -102,69 +102,86 @@ __global__ void __launch_bounds__(NT)
 // that of single steps.  Inputs follow the prefill layout with N = steps:
 // q, o [B, Hq, steps, D], k, v [B, Hkv, steps, D].
 //
-// One thread per state column c (D threads per unit, column in D registers):
-// the update is elementwise and o_{t,h}[c] = sum_r q_{t,h}[r] S[r][c] is a
-// per-thread sum, so no cross-thread reduction is needed; k and q come from
-// shared memory as broadcast float4 reads.  Query heads go in passes of GB
-// (the update rides on the first pass).  The next step's k, v, q are loaded
-// into registers while the current step computes, then written to the other
-// half of a double buffer: one barrier per step.
+// Two threads per state column c (2 D threads per unit), each holding half
+// of the column (D / 2 rows) in registers: the update is elementwise and
+// o_{t,h}[c] is a dot product over rows, so each thread sums its half and
+// the pair (adjacent lanes) adds the two halves with one shuffle.  k and q
+// come from shared memory as broadcast float4 reads, each half stored with a
+// 4-float pad so the two halves of a warp read different banks.  Query heads
+// go in passes of GB (the update rides on the first pass).  The next step's
+// k, v, q are loaded into registers while the current step computes, then
+// written to the other half of a double buffer: one barrier per step.
+// Two CTAs per SM (128 registers at d = 128), except 2- and 8-head passes at
+// d = 128, which would spill at that bound.
 template <int D, int GB>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(2 * D, (D == 128 && (GB == 8 || GB == 2)) ? 1 : 2)
     decode_steps_kernel(float* __restrict__ S, const __nv_bfloat16* __restrict__ q,
                         const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                         __nv_bfloat16* __restrict__ o, int Hq, int Hkv, int steps) {
+  constexpr int R = D / 2;   // rows per thread
+  constexpr int RP = R + 4;  // padded stride of one half row in shared memory
   extern __shared__ float4 sh4[];
   float* sh = reinterpret_cast<float*>(sh4);
   const int G = Hq / Hkv;
-  const int rec = (G + 2) * D;  // one step's k, v, q_0 .. q_{G-1} (fp32)
+  // one step's record: k and q_0 .. q_{G-1} as [2][RP] halves, then v [D]
+  const int rec = 2 * RP * (G + 1) + D;
+  auto row_off = [&](int j) { return j == 1 ? 2 * RP * (G + 1) : 2 * RP * (j == 0 ? 0 : j - 1); };
   const int unit = blockIdx.x;  // b * Hkv + g
   const int b = unit / Hkv, g = unit % Hkv;
-  const int c = threadIdx.x;    // state column
-  const __nv_bfloat16* kp = k + (size_t)unit * steps * D + c;
-  const __nv_bfloat16* vp = v + (size_t)unit * steps * D + c;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int c = (tid >> 5) * 16 + (lane >> 1);  // state column
+  const int half = lane & 1;                    // rows [half * R, half * R + R)
   const size_t qh0 = (size_t)b * Hq + (size_t)g * G;  // first query head of the group
-  const __nv_bfloat16* qp = q + qh0 * steps * D + c;
-  __nv_bfloat16* op = o + qh0 * steps * D + c;
 
-  // step t's record element c of every row -> registers (the launcher picks
-  // GB so that G <= kMaxG)
+  // staging: thread tid brings element e = tid % D of the record's rows j with
+  // j % 2 == tid / D (rows: 0 = k, 1 = v, 2 + h = q_h)
+  const int e = tid % D, jpar = tid / D;
+  const int eo = e < R ? e : RP + (e - R);  // its place in a split row
   constexpr int kMaxG = GB == 8 ? kMaxGroup : 2 * GB - 1;
-  __nv_bfloat16 pre[2 + kMaxG];
+  constexpr int kMaxRows = (2 + kMaxG + 1) / 2;
+  __nv_bfloat16 pre[kMaxRows];
+  auto row_src = [&](int j, int t) -> const __nv_bfloat16* {
+    if (j == 0) return k + ((size_t)unit * steps + t) * D;
+    if (j == 1) return v + ((size_t)unit * steps + t) * D;
+    return q + ((qh0 + (j - 2)) * steps + t) * D;
+  };
   auto fetch = [&](int t) {
-    pre[0] = kp[(size_t)t * D];
-    pre[1] = vp[(size_t)t * D];
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h)
-      if (h < G) pre[2 + h] = qp[((size_t)h * steps + t) * D];
+    for (int m = 0; m < kMaxRows; ++m) {
+      const int j = 2 * m + jpar;
+      if (j < 2 + G) pre[m] = row_src(j, t)[e];
+    }
   };
   auto stash = [&](float* buf) {
 #pragma unroll
-    for (int j = 0; j < 2 + kMaxG; ++j)
-      if (j < 2 + G) buf[j * D + c] = __bfloat162float(pre[j]);
+    for (int m = 0; m < kMaxRows; ++m) {
+      const int j = 2 * m + jpar;
+      if (j < 2 + G) buf[row_off(j) + (j == 1 ? e : eo)] = __bfloat162float(pre[m]);
+    }
   };
 
-  float s[D];
-  const float* Su = S + (size_t)unit * D * D + c;
+  float s[R];
+  const float* Su = S + (size_t)unit * D * D + (size_t)half * R * D + c;
 #pragma unroll
-  for (int r = 0; r < D; ++r) s[r] = __ldcs(Su + (size_t)r * D);
+  for (int r = 0; r < R; ++r) s[r] = __ldcs(Su + (size_t)r * D);
   fetch(0);
   stash(sh);
   __syncthreads();
 
+  __nv_bfloat16* op = o + qh0 * steps * D + c;
   for (int t = 0; t < steps; ++t) {
     const float* buf = sh + (size_t)(t & 1) * rec;
     if (t + 1 < steps) fetch(t + 1);  // in flight while this step computes
-    const float vc = buf[D + c];
-    const float4* k4 = reinterpret_cast<const float4*>(buf);
+    const float vc = buf[2 * RP * (G + 1) + c];
+    const float4* k4 = reinterpret_cast<const float4*>(buf + half * RP);
     for (int hb = 0; hb < G; hb += GB) {
-      float acc[GB][2];  // two partial sums per head (even / odd row quads): shorter chains
+      float acc[GB][2];  // two partial sums per head: shorter chains
 #pragma unroll
       for (int j = 0; j < GB; ++j) acc[j][0] = acc[j][1] = 0.f;
-      const float4* q4 = reinterpret_cast<const float4*>(buf + (size_t)(2 + hb) * D);
       const int nh = G - hb;  // heads left; a short last pass is predicated
 #pragma unroll
-      for (int r4 = 0; r4 < D / 4; ++r4) {
+      for (int r4 = 0; r4 < R / 4; ++r4) {
         if (hb == 0) {
           const float4 kk = k4[r4];
           s[4 * r4 + 0] = fmaf(kk.x, vc, s[4 * r4 + 0]);
@@ -175,7 +192,8 @@ __global__ void __launch_bounds__(D)
 #pragma unroll
         for (int j = 0; j < GB; ++j) {
           if (j < nh) {
-            const float4 qq = q4[(size_t)j * (D / 4) + r4];
+            const float4 qq =
+                reinterpret_cast<const float4*>(buf + 2 * RP * (1 + hb + j) + half * RP)[r4];
             float& a = acc[j][r4 & 1];
             a = fmaf(qq.x, s[4 * r4 + 0], a);
             a = fmaf(qq.y, s[4 * r4 + 1], a);
@@ -185,27 +203,31 @@ __global__ void __launch_bounds__(D)
         }
       }
 #pragma unroll
-      for (int j = 0; j < GB; ++j)
-        if (j < nh)
-          op[((size_t)(hb + j) * steps + t) * D] = __float2bfloat16_rn(acc[j][0] + acc[j][1]);
+      for (int j = 0; j < GB; ++j) {
+        if (j < nh) {  // uniform over the warp
+          float a = acc[j][0] + acc[j][1];
+          a += __shfl_xor_sync(0xffffffffu, a, 1);  // the other half of the column
+          if (half == 0) op[((size_t)(hb + j) * steps + t) * D] = __float2bfloat16_rn(a);
+        }
+      }
     }
     if (t + 1 < steps) stash(sh + (size_t)((t + 1) & 1) * rec);
     __syncthreads();  // the next step's record is complete; this step's is no longer read
   }
-  float* Sw = S + (size_t)unit * D * D + c;
+  float* Sw = S + (size_t)unit * D * D + (size_t)half * R * D + c;
 #pragma unroll
-  for (int r = 0; r < D; ++r) __stcs(Sw + (size_t)r * D, s[r]);
+  for (int r = 0; r < R; ++r) __stcs(Sw + (size_t)r * D, s[r]);
 }
 
 template <int D, int GB>
 cudaError_t launch_decode_steps_gb(float* S, const void* q, const void* k, const void* v, void* o,
                                    int B, int Hq, int Hkv, int steps, cudaStream_t stream) {
   const int G = Hq / Hkv;
-  const size_t smem = sizeof(float) * 2 * (size_t)(G + 2) * D;
+  const size_t smem = sizeof(float) * 2 * (size_t)(2 * (D / 2 + 4) * (G + 1) + D);
   cudaError_t e = cudaFuncSetAttribute(decode_steps_kernel<D, GB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_steps_kernel<D, GB><<<(unsigned)(B * Hkv), D, smem, stream>>>(
+  decode_steps_kernel<D, GB><<<(unsigned)(B * Hkv), 2 * D, smem, stream>>>(
       S, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), Hq, Hkv, steps);
   return cudaGetLastError();
