@@ -140,9 +140,10 @@ la_status la_forward_host(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, 
                           int64_t piece, la_stream stream);
 
 /* ------------------------------------------------------------------------
- * The prefill as one persistent kernel (an alternative schedule of the same
- * arithmetic; la_forward runs the three-kernel scheme below).  Every (batch, kv head) sequence is cut into `nspan`
- * spans; span-state items (K^T V of a span, then the chained prefix: the state
+ * The prefill as one single-pass persistent kernel (an alternative schedule
+ * of the same arithmetic, slower; la_forward runs the span states, the scan
+ * and the persistent chunk loop of the stages below).  Every (batch, kv head)
+ * sequence is cut into `nspan` spans; span-state items (K^T V of a span, then the chained prefix: the state
  * entering the next span) and chunk-loop items (the chunk loop of one span for
  * a group of query heads, from its entering state) are taken in rounds, one
  * round per span index, so the chunk loops of a span re-read its K and V from
@@ -188,9 +189,12 @@ la_status la_forward_noalloc(const la_bf16 *q, const la_bf16 *k, const la_bf16 *
                              la_stream stream);
 
 /* ------------------------------------------------------------------------
- * The prefill's three stages -- the scheme la_forward, la_forward_state,
- * la_forward_ws and la_forward_noalloc run -- for callers that schedule or time
- * them apart: plan, then span_states, scan, main on one stream.
+ * The prefill's three stages -- the scheme the la_forward* calls run -- for
+ * callers that schedule or time them apart: plan, then span_states, scan,
+ * main on one stream.  (The la_forward* calls refine it: they skip the last
+ * span's K^T V and let the chunk loop write the final state, cut spans into
+ * sub-spans for the first stage when sequences x spans are fewer than the
+ * SMs, and with one span per sequence run the chunk loop alone.)
  *
  * The sequence of every (batch, kv head) is cut into `nspan` spans of whole
  * chunks.  span_states writes each span's K^T V into the workspace; scan turns
