@@ -191,10 +191,10 @@ la_status la_forward_noalloc(const la_bf16 *q, const la_bf16 *k, const la_bf16 *
 /* ------------------------------------------------------------------------
  * The prefill's three stages -- the scheme the la_forward* calls run -- for
  * callers that schedule or time them apart: plan, then span_states, scan,
- * main on one stream.  (The la_forward* calls refine it: they skip the last
- * span's K^T V and let the chunk loop write the final state, cut spans into
- * sub-spans for the first stage when sequences x spans are fewer than the
- * SMs, and with one span per sequence run the chunk loop alone.)
+ * main on one stream.  (The la_forward* calls refine it: without a state to
+ * return they skip the last span's K^T V, they cut spans into sub-spans for
+ * the first stage when sequences x spans are fewer than the SMs, and with
+ * one span per sequence they run the chunk loop alone.)
  *
  * The sequence of every (batch, kv head) is cut into `nspan` spans of whole
  * chunks.  span_states writes each span's K^T V into the workspace; scan turns

@@ -39,7 +39,7 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, i
 bool make_tmap_state(CUtensorMap* map, const void* base, int64_t units);
 
 // skip_last: spans 0 .. nspan-2 only (the last span's state is needed only
-// for the final state, which the chunk loop then writes).  parts: each span
+// for the final state).  parts: each span
 // cut into `parts` sub-spans computed by separate CTAs (more CTAs when there
 // are few sequences and spans); ws then holds nspan * parts states per
 // sequence, in order.
