@@ -271,7 +271,7 @@ size_t forward_workspace_bytes(const la_plan& plan) {
 
 la_status forward_persistent(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
                              float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, bool final_out) {
   unsigned* status = nullptr;
   int sms = 0;
   if (!device_info(&status, &sms)) return LA_ERR_CUDA;
@@ -282,14 +282,16 @@ la_status forward_persistent(const la_bf16* q, const la_bf16* k, const la_bf16* 
       !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
     return LA_ERR_CUDA;
   PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
-  return from_cuda(
-      launch_prefill_persist(g, maps, S, S, status, sms, stream, false, stage_states_pays(g)));
+  return from_cuda(launch_prefill_persist(g, maps, S, final_out ? S : nullptr, status, sms, stream,
+                                          false, stage_states_pays(g)));
 }
 
 la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
                            float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
-                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  if (plan.nspan == 1) return forward_persistent(q, k, v, o, S, B, Hq, Hkv, N, plan, stream);
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                           bool final_out) {
+  if (plan.nspan == 1)
+    return forward_persistent(q, k, v, o, S, B, Hq, Hkv, N, plan, stream, final_out);
   // Span states, entering states (and the final state), chunk loop.
   unsigned* status = nullptr;
   int sms = 0;
@@ -313,7 +315,7 @@ la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v,
   // states is more accurate than the last span's updates accumulated in
   // tensor memory on top of its entering state (1M tokens: final-state rel-L2
   // 3.3e-5 against 8.6e-5), for 1/nspan more of the first pass.
-  const bool final_state = S != nullptr;
+  const bool final_state = S != nullptr && final_out;
   cudaError_t e = launch_span_states(g, maps.k, maps.v, ws, status, stream, !final_state, parts);
   if (e == cudaSuccess)
     e = launch_state_scan(ws, S, B * Hkv, nsub_spans, kHeadDim, stream, 0,

@@ -161,7 +161,7 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
   // ---- dq: the forward pass on (dO, V, K) from S0^T
   cu(place_states(S0, S_q, B, Hkv, 1, d, 1, s));
   if (st == LA_OK)
-    st = forward_dispatch(dO, v, k, dq, S_q, B, Hq, Hkv, N, plan_q, ws_q, wsq_bytes, s);
+    st = forward_dispatch(dO, v, k, dq, S_q, B, Hq, Hkv, N, plan_q, ws_q, wsq_bytes, s, false);
 
   // ---- dv, then dk: anti-causal walks per query head, summed over groups.
   // One state serves both: D = sum_t q_t^T do_t over the later chunks (dv

@@ -82,9 +82,11 @@ size_t forward_workspace_bytes(const la_plan& plan);
 // when the plan has one span per sequence, else span states, scan and the
 // persistent chunk loop; the span parts are lowered to what workspace_bytes
 // holds (at least the plan's own workspace_bytes).
+// final_out = false: S (nullable) supplies S0 only and is not written.
 la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v, la_bf16* o,
                            float* S, int B, int Hq, int Hkv, int64_t N, const la_plan& plan,
-                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                           bool final_out = true);
 cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
                                  void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);
