@@ -382,7 +382,7 @@ def run_ours(args, w):
                     "algorithmic_gb_s": bbytes / tb / 1e9,
                     "frac_of_hbm_roofline": bbytes / tb / 1e9 / pk["hbm_gbs"],
                     "bytes": bbytes, "clocks": bclk,
-                    "passes": "dq causal (grouped) + dv, dk anti-causal per query head + group sums"}
+                    "passes": "dq causal (grouped) + one anti-causal dk, dv walk per kv group"}
         del dOd
 
     # --- end to end: pinned host buffers, copies inside the timed region.

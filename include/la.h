@@ -260,9 +260,10 @@ la_status la_state_prefix(const float *states, const float *S0, float *S, int ns
  *   dv_s = sum_{h in group} sum_{t>=s} (k_s . q_{t,h}) do_{t,h} + k_s dSf
  *   dS0  = dSf + sum_{h in group} sum_t q_{t,h}^T do_{t,h}    (dS0 nullable)
  * (the chain rule through o_t = q_t S_t, S_t = S0 + sum_{s<=t} k_s^T v_s of
- * [VGX]).  dq is the forward pass itself on (dO, V, K, S0^T); dk and dv are
- * anti-causal passes of the same tensor-core kernels, one per query head,
- * summed over each group.  dq [B,Hq,N,d], dk, dv [B,Hkv,N,d] bf16 outputs
+ * [VGX]).  dq is the forward pass itself on (dO, V, K, S0^T); dk and dv come
+ * from one anti-causal walk per kv group (chunks last to first, every query
+ * head of the group summed inside the tensor-core products, spans of it in
+ * parallel).  dS0 may be dSf.  dq [B,Hq,N,d], dk, dv [B,Hkv,N,d] bf16 outputs
  * (no overlap with the inputs).  Scratch comes from the stream-ordered pool.
  * d = 128, chunk in {64, 128} (the chunk of the dq pass; the others use 128).
  * Errors as la_forward_state. */

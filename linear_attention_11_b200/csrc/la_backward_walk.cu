@@ -1,0 +1,712 @@
+// la_backward_walk.cu -- dk and dv of the backward in one anti-causal walk per
+// kv group (tcgen05 tensor cores), and the scan of its span states.
+//
+// From o_t = q_t S_t, S_t = S0 + sum_{s<=t} k_s^T v_s (the causal chunk form
+// of "如何理解MiniMax股价创历史新高？拆解国产大模型技术底座", section
+// "Lightning Attention：长上下文为什么突然变得便宜了"; grouped kv heads as in
+// "MiniMax-01与Lightning Attention", section 1.1), with D_c = dSf + the sum of
+// q_{t,h}^T do_{t,h} over every query head h of the group and every token t
+// after chunk c:
+//   dv_c = sum_h triu(K_c Q_{c,h}^T) dO_{c,h} + K_c D_c
+//   dk_c = sum_h triu(V_c dO_{c,h}^T) Q_{c,h} + V_c D_c^T
+//   D_{c-1} = D_c + sum_h Q_{c,h}^T dO_{c,h},   dS0 = D before the first chunk
+// (triu keeps the diagonal: key token t >= row token s).  The heads of a group
+// share K_c, V_c and one state, so a walk over the group's chunks, last to
+// first, reads every Q and dO tile once for both gradients and sums the heads
+// inside the MMAs (fp32 in tensor memory).
+//
+// Per 128-token chunk c of a group, per 64-token key block (head h, half j):
+//   S1 = K_c Q_hj^T, S2 = V_c dO_hj^T   M=128 N=64  K=128 (SS) -> TMEM
+//   P1, P2 = bf16(triu(S1)), bf16(triu(S2))   TMEM -> registers -> smem
+//   dv += P1 dO_hj, dk += P2 Q_hj       M=128 N=128 K=64 (SS)
+//   D  += Q_hj^T dO_hj                  M=128 N=128 K=64 (SS, both MN-major)
+// and once per chunk, from the bf16 copy of D_c in smem (read MN-major for D,
+// K-major for D^T):  dv += K_c D_c,  dk += V_c D_c^T  (M=128 N=128 K=128).
+//
+// Schedule: one CTA per SM walks (group, span) items round-robin, each span
+// from its last chunk to its first; the entering state of a span (dSf plus
+// the later spans' sums, from group_scan_kernel) is read at the item start,
+// and the item of span 0 writes dS0 at its end.
+// Roles (320 threads): warp 0 lane 0 streams key blocks (Q and dO of one head
+// half-chunk) through a three-stage ring, lane 1 the K/V tiles of each chunk
+// and L2 prefetches of the next chunk; warp 1 owns the tensor memory and
+// issues the MMAs, scores two blocks ahead; warps 2-5 mask the scores and
+// convert the state; warps 6-9 write dv and dk rows out.
+// TMEM: dv at column 0, dk at 128, S1 at 256, S2 at 320, D at 384.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "la_internal.h"
+#include "la_ptx.cuh"
+#include "la_tile.cuh"
+
+namespace la {
+namespace {
+
+constexpr int kChunk = 128;                         // tokens per chunk
+constexpr int kKeyBlk = 64;                         // tokens per key block
+constexpr int kRing = 3;                            // key-block stages
+constexpr int kChunkBytes = kChunk * kHeadDim * 2;  // 32 KB: K_c or V_c
+constexpr int kBlkBytes = kKeyBlk * kHeadDim * 2;   // 16 KB: Q or dO of one block
+constexpr int kBlkHalf = kKeyBlk * 128;             // 8 KB: 64 columns of a key block
+constexpr int kPBytes = kChunk * kKeyBlk * 2;       // 16 KB: one P tile
+constexpr uint32_t kColDv = 0, kColDk = 128, kColS1 = 256, kColS2 = 320;
+
+struct WalkLayout {
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kChunkBytes;
+  static constexpr int kRingOff = 2 * kChunkBytes;                // stage: Q block, dO block
+  static constexpr int kSOff = kRingOff + kRing * 2 * kBlkBytes;  // bf16 copy of D
+  static constexpr int kPOff = kSOff + kSBytes;                   // P1, P2
+  static constexpr int kBarOff = kPOff + 2 * kPBytes;
+  // ring_full[R], ring_empty[R], kv_full, kv_empty, a_full, s_read, p_full,
+  // p_free, o_full, o_empty[2], s_full, sb_full, mma_done
+  static constexpr int kNumBars = 2 * kRing + 12;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
+};
+static_assert(WalkLayout::kBytes <= 232448, "shared memory");
+
+struct WalkParams {
+  const __nv_bfloat16 *q, *k, *v, *dO;  // for the L2 prefetches
+  __nv_bfloat16 *dk, *dv;               // [B*Hkv, N, 128]
+  const float* ws;  // entering state of item it at ws[it * d * d]; nullptr: zero
+  float* s_out;     // dS0 of group bg at s_out[bg] (from span 0's item); nullable
+  unsigned* status;
+  int64_t N;
+  int Hq, Hkv, G, nspan, tiles_total, items;
+};
+
+// Position in a CTA's sequence of key blocks: item it (group bg, chunks
+// [tb, te) walked from te - 1), n-th chunk of the item (chunk index cs), block
+// blk of nb in the chunk (head blk / halves, half blk % halves), the CTA's
+// chunk count gc and block count i.
+struct Cursor {
+  int it, bg, tb, te, n, cs, blk, nb, gc, i;
+  bool valid;
+};
+
+__device__ __forceinline__ void span_of(const WalkParams& p, int it, int& bg, int& tb, int& te) {
+  const int j = it % p.nspan;
+  bg = it / p.nspan;
+  tb = (int)(((int64_t)j * p.tiles_total) / p.nspan);
+  te = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
+}
+
+// 64-token halves of chunk cs that hold tokens (the last chunk may have one).
+__device__ __forceinline__ int halves_of(const WalkParams& p, int cs) {
+  return p.N - (int64_t)cs * kChunk > kKeyBlk ? 2 : 1;
+}
+
+__device__ __forceinline__ void cursor_item(const WalkParams& p, Cursor& c) {
+  span_of(p, c.it, c.bg, c.tb, c.te);
+  c.n = 0;
+  c.cs = c.te - 1;
+  c.nb = p.G * halves_of(p, c.cs);
+  c.blk = 0;
+}
+
+__device__ __forceinline__ void cursor_init(const WalkParams& p, Cursor& c) {
+  c.it = blockIdx.x;
+  c.gc = 0;
+  c.i = 0;
+  c.valid = c.it < p.items;
+  if (c.valid) cursor_item(p, c);
+}
+
+__device__ __forceinline__ void cursor_next(const WalkParams& p, Cursor& c) {
+  ++c.i;
+  if (++c.blk < c.nb) return;
+  c.blk = 0;
+  ++c.gc;
+  if (++c.n < c.te - c.tb) {
+    c.cs = c.te - 1 - c.n;
+    c.nb = p.G * halves_of(p, c.cs);
+    return;
+  }
+  c.it += (int)gridDim.x;
+  c.valid = c.it < p.items;
+  if (c.valid) cursor_item(p, c);
+}
+
+__device__ __forceinline__ void store_p_row(uint32_t tile, int r, const uint32_t (&pk)[32]) {
+  const uint32_t row = tile + (uint32_t)(r * 128);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    st_shared_v4(row + (uint32_t)((c ^ (r & 7)) * 16), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                 pk[4 * c + 3]);
+}
+
+__global__ void __launch_bounds__(320, 1)
+    bwd_walk_kernel(const __grid_constant__ CUtensorMap map_q,
+                    const __grid_constant__ CUtensorMap map_do,
+                    const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, const WalkParams p) {
+  using L = WalkLayout;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, kKeyBlk, 0, 0);
+  constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
+  constexpr uint32_t IDESC_KD = idesc_bf16_f32(128, 128, 0, 1);
+  constexpr uint32_t IDESC_VDT = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t IDESC_D = idesc_bf16_f32(128, 128, 1, 1);
+  constexpr int kDD = kHeadDim * kHeadDim;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sm = smem_raw + (base - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBarOff);
+  uint64_t* ring_full = bars;
+  uint64_t* ring_empty = ring_full + kRing;
+  uint64_t* kv_full = ring_empty + kRing;
+  uint64_t* kv_empty = kv_full + 1;
+  uint64_t* a_full = kv_empty + 1;   // S1, S2 of a block computed
+  uint64_t* s_read = a_full + 1;     // ... and read out by the mask warps
+  uint64_t* p_full = s_read + 1;     // P1, P2 of a block in smem
+  uint64_t* p_free = p_full + 1;     // the P tiles read by their MMAs
+  uint64_t* o_full = p_free + 1;     // dv, dk of a chunk complete
+  uint64_t* o_empty = o_full + 1;    // two: dv, dk read out
+  uint64_t* s_full = o_empty + 2;    // D updated with a chunk
+  uint64_t* sb_full = s_full + 1;    // bf16 copy of D (and D itself at an item start) ready
+  uint64_t* mma_done = sb_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
+
+  const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
+  const uint32_t sS = base + L::kSOff;
+  const uint32_t sP1 = base + L::kPOff, sP2 = sP1 + kPBytes;
+  auto sQ = [&](int s) { return base + (uint32_t)(L::kRingOff + s * 2 * kBlkBytes); };
+  auto sDO = [&](int s) { return sQ(s) + (uint32_t)kBlkBytes; };
+  const int stride = (int)gridDim.x;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
+    }
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(a_full, 1);
+    mbar_init(s_read, 128);
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(o_full, 1);
+    mbar_init(&o_empty[0], 128);
+    mbar_init(&o_empty[1], 128);
+    mbar_init(s_full, 1);
+    mbar_init(sb_full, 128);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ copies
+    if (lane == 0) {
+      // key blocks: Q and dO rows [t0, t0 + 64) of head h, in cursor order
+      prefetch_tmap(&map_q);
+      prefetch_tmap(&map_do);
+      const uint64_t pol = policy_evict_first();
+      Cursor c;
+      cursor_init(p, c);
+      int issued = 0;
+      for (; c.valid; cursor_next(p, c)) {
+        const int s = c.i % kRing;
+        if (c.i >= kRing &&
+            !mbar_wait(&ring_empty[s], ((c.i / kRing) - 1) & 1, p.status, abort_flag))
+          break;
+        const int halves = c.nb / p.G;
+        const int h = c.blk / halves, j = c.blk % halves;
+        const int b = c.bg / p.Hkv, g = c.bg % p.Hkv;
+        const int qh = b * p.Hq + g * p.G + h;
+        const int t0 = c.cs * kChunk + j * kKeyBlk;
+        mbar_arrive_expect_tx(&ring_full[s], 2 * kBlkBytes);
+        uint8_t* q_dst = sm + (sQ(s) - base);
+        uint8_t* do_dst = sm + (sDO(s) - base);
+        tma_load_3d(q_dst, &map_q, &ring_full[s], 0, t0, qh, pol);
+        tma_load_3d(q_dst + kBlkHalf, &map_q, &ring_full[s], 64, t0, qh, pol);
+        tma_load_3d(do_dst, &map_do, &ring_full[s], 0, t0, qh, pol);
+        tma_load_3d(do_dst + kBlkHalf, &map_do, &ring_full[s], 64, t0, qh, pol);
+        issued = c.i + 1;
+      }
+      if (*abort_flag) {  // let copies already issued land before the block exits
+        for (int k = (issued > kRing ? issued - kRing : 0); k < issued; ++k)
+          mbar_wait_drain(&ring_full[k % kRing], (k / kRing) & 1);
+      }
+    } else if (lane == 1) {
+      // K_c, V_c per chunk; L2 prefetch of the next chunk's Q, dO (every head
+      // of the group), K, V, and of the next item's entering state
+      prefetch_tmap(&map_k);
+      prefetch_tmap(&map_v);
+      const uint64_t pol = policy_evict_first();
+      auto prefetch_chunk = [&](int bg, int cs) {
+        const int64_t t0 = (int64_t)cs * kChunk;
+        const uint32_t bytes = (uint32_t)(std::min<int64_t>(kChunk, p.N - t0) * kHeadDim * 2);
+        const int b = bg / p.Hkv, g = bg % p.Hkv;
+        for (int h = 0; h < p.G; ++h) {
+          const size_t off = ((size_t)(b * p.Hq + g * p.G + h) * p.N + t0) * kHeadDim;
+          prefetch_l2_bulk(p.q + off, bytes);
+          prefetch_l2_bulk(p.dO + off, bytes);
+        }
+        const size_t off = ((size_t)bg * p.N + t0) * kHeadDim;
+        prefetch_l2_bulk(p.k + off, bytes);
+        prefetch_l2_bulk(p.v + off, bytes);
+      };
+      int gc = 0;
+      bool go = true;
+      for (int it = blockIdx.x; it < p.items && go; it += stride) {
+        int bg, tb, te;
+        span_of(p, it, bg, tb, te);
+        const int nx = it + stride < p.items ? it + stride : -1;
+        if (p.ws && nx >= 0)
+          prefetch_l2_bulk(p.ws + (size_t)nx * kDD, (uint32_t)(kDD * sizeof(float)));
+        for (int n = 0; n < te - tb; ++n, ++gc) {
+          const int cs = te - 1 - n;
+          if (n + 1 < te - tb) {
+            prefetch_chunk(bg, cs - 1);
+          } else if (nx >= 0) {
+            int bg2, tb2, te2;
+            span_of(p, nx, bg2, tb2, te2);
+            prefetch_chunk(bg2, te2 - 1);
+          }
+          if (gc >= 1 && !mbar_wait(kv_empty, (gc - 1) & 1, p.status, abort_flag)) {
+            go = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kv_full, 2 * kChunkBytes);
+          uint8_t* k_dst = sm + (sK - base);
+          uint8_t* v_dst = sm + (sV - base);
+          tma_load_3d(k_dst, &map_k, kv_full, 0, cs * kChunk, bg, pol);
+          tma_load_3d(k_dst + kHalf, &map_k, kv_full, 64, cs * kChunk, bg, pol);
+          tma_load_3d(v_dst, &map_v, kv_full, 0, cs * kChunk, bg, pol);
+          tma_load_3d(v_dst + kHalf, &map_v, kv_full, 64, cs * kChunk, bg, pol);
+        }
+      }
+      if (*abort_flag && gc > 0) mbar_wait_drain(kv_full, (gc - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // Tensor pipe order: S(0) S(1) | PV(0) D(0) S(2) | PV(1) D(1) S(3) | ...
+    // so the scores of block i+1 are masked while block i's products run.
+    // K_c and V_c sit in one slot: their copy for the next chunk starts once
+    // the chunk's last S and its K_c D, V_c D^T are issued, and a next chunk's
+    // first S is held back until that point.
+    if (elect_one()) {
+      Cursor a, c;  // a: next block to score; c: next block to multiply
+      cursor_init(p, a);
+      cursor_init(p, c);
+      int inter_gc = -1;   // last chunk whose K_c D, V_c D^T are issued
+      int kv_pending = -1; // chunk whose last S is issued before its K_c D
+      auto issue_s = [&](const Cursor& x) -> bool {
+        if (x.blk == 0 && !mbar_wait(kv_full, x.gc & 1, p.status, abort_flag)) return false;
+        const int s = x.i % kRing;
+        if (!mbar_wait(&ring_full[s], (x.i / kRing) & 1, p.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qa = sQ(s), doa = sDO(s);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // S1 = K_c Q^T, S2 = V_c dO^T (all K-major)
+          const uint32_t koff = (uint32_t)((kk & 3) * 32);
+          const uint32_t ch = (uint32_t)(kk >> 2);
+          mma_ss(tmem + kColS1, smem_desc_sw128(sK + ch * kHalf + koff, 16, 1024),
+                 smem_desc_sw128(qa + ch * kBlkHalf + koff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kColS2, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
+                 smem_desc_sw128(doa + ch * kBlkHalf + koff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(a_full);
+        if (x.blk == x.nb - 1) {
+          if (inter_gc >= x.gc)
+            mma_commit(kv_empty);
+          else
+            kv_pending = x.gc;
+        }
+        return true;
+      };
+      // score blocks up to c + 1 (the S tiles are free once the block before
+      // was read out); a chunk's first block waits for the K/V slot rule
+      auto score_ahead = [&](bool must) -> bool {
+        while (a.valid && a.i <= c.i + 1) {
+          if (a.blk == 0 && inter_gc < a.gc - 1 && !(must && a.i == c.i)) break;
+          if (a.i > 0 && !mbar_wait(s_read, (a.i - 1) & 1, p.status, abort_flag)) return false;
+          if (!issue_s(a)) return false;
+          cursor_next(p, a);
+        }
+        return true;
+      };
+      bool ok = score_ahead(true);
+      while (ok && c.valid) {
+        if (a.valid && a.i == c.i && !score_ahead(true)) break;
+        const int k = c.i;
+        const bool first = c.blk == 0, last = c.blk == c.nb - 1;
+        if (!mbar_wait(p_full, k & 1, p.status, abort_flag)) break;
+        if (first && c.gc >= 1 &&
+            (!mbar_wait(&o_empty[0], (c.gc - 1) & 1, p.status, abort_flag) ||
+             !mbar_wait(&o_empty[1], (c.gc - 1) & 1, p.status, abort_flag)))
+          break;
+        tc_fence_after();
+        const int s = k % kRing;
+        const uint32_t qa = sQ(s), doa = sDO(s);
+#pragma unroll
+        for (int kk = 0; kk < kKeyBlk / 16; ++kk) {  // dv += P1 dO, dk += P2 Q
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          mma_ss(tmem + kColDv, smem_desc_sw128(sP1 + kk * 32, 16, 1024),
+                 smem_desc_sw128(doa + kk * 2048, kBlkHalf, 1024), IDESC_PV, acc);
+          mma_ss(tmem + kColDk, smem_desc_sw128(sP2 + kk * 32, 16, 1024),
+                 smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024), IDESC_PV, acc);
+        }
+        if (first) {  // dv += K_c D, dk += V_c D^T from the bf16 copy of D_c
+          if (!mbar_wait(sb_full, c.gc & 1, p.status, abort_flag)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (uint32_t)((kk & 3) * 32);
+            const uint32_t ch = (uint32_t)(kk >> 2);
+            mma_ss(tmem + kColDv, smem_desc_sw128(sK + ch * kHalf + koff, 16, 1024),
+                   smem_desc_sw128(sS + kk * 2048, kHalf, 1024), IDESC_KD, 1u);
+            mma_ss(tmem + kColDk, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
+                   smem_desc_sw128(sS + ch * kHalf + koff, 16, 1024), IDESC_VDT, 1u);
+          }
+          inter_gc = c.gc;
+          if (kv_pending == c.gc) {
+            mma_commit(kv_empty);
+            kv_pending = -1;
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < kKeyBlk / 16; ++kk)  // D += Q^T dO (both MN-major)
+          mma_ss(tmem + kColS, smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024),
+                 smem_desc_sw128(doa + kk * 2048, kBlkHalf, 1024), IDESC_D, 1u);
+        mma_commit(p_free);
+        mma_commit(&ring_empty[s]);
+        if (last) {
+          mma_commit(o_full);
+          mma_commit(s_full);
+        }
+        cursor_next(p, c);
+        if (!score_ahead(false)) break;
+      }
+      mma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ masks, state
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // TMEM lane = chunk row = state row
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+
+    // entering state of item it -> D in tensor memory and its bf16 copy
+    auto load_state = [&](int it) {
+      const float4* src =
+          p.ws ? reinterpret_cast<const float4*>(p.ws + (size_t)it * kDD + (size_t)r * kHeadDim)
+               : nullptr;
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        uint32_t v[32];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (src) f = src[blk * 8 + m];  // plain loads: dS0 may be written in place
+          v[4 * m + 0] = __float_as_uint(f.x);
+          v[4 * m + 1] = __float_as_uint(f.y);
+          v[4 * m + 2] = __float_as_uint(f.z);
+          v[4 * m + 3] = __float_as_uint(f.w);
+        }
+        tmem_st32(tmem + lane_base + kColS + blk * 32, v);
+        store_row32_sw128(sS, r, blk, v);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(sb_full);
+    };
+
+    // after chunk gcd's state update: the bf16 copy for the next chunk, or at
+    // an item's end dS0 out (span 0) and the next item's entering state in
+    auto state_step = [&](int gcd, bool item_end, int done_it, int next_it) -> bool {
+      if (!warp_wait(s_full, gcd & 1, p.status, abort_flag)) return false;
+      tc_fence_after();
+      if (!item_end) {
+#pragma unroll 1
+        for (int blk = 0; blk < 4; blk += 2) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_base + kColS + blk * 32, v0);
+          tmem_ld32(tmem + lane_base + kColS + (blk + 1) * 32, v1);
+          tmem_wait_ld();
+          store_row32_sw128(sS, r, blk, v0);
+          store_row32_sw128(sS, r, blk + 1, v1);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(sb_full);
+        return true;
+      }
+      if (p.s_out && done_it % p.nspan == 0) {
+        float4* dst = reinterpret_cast<float4*>(p.s_out + (size_t)(done_it / p.nspan) * kDD +
+                                                (size_t)r * kHeadDim);
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + kColS + blk * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            dst[blk * 8 + m] = make_float4(__uint_as_float(v[4 * m]), __uint_as_float(v[4 * m + 1]),
+                                           __uint_as_float(v[4 * m + 2]),
+                                           __uint_as_float(v[4 * m + 3]));
+        }
+      }
+      tc_fence_before();
+      if (next_it >= 0) load_state(next_it);
+      return true;
+    };
+
+    // scores of block c -> masked bf16 P tiles in smem
+    auto mask_block = [&](const Cursor& c) -> bool {
+      const int k = c.i;
+      const int halves = c.nb / p.G;
+      const int j = c.blk % halves;
+      if (!warp_wait(a_full, k & 1, p.status, abort_flag)) return false;
+      tc_fence_after();
+      // key column u of the block is token 64 j + u of the chunk; row r keeps
+      // u >= r - 64 j.  Rows 64..127 keep nothing of the first half.
+      const int rel = r - kKeyBlk * j;
+      const bool none = j == 0 && quarter >= 2;
+      uint32_t p1[32], p2[32];
+      if (!none) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          uint32_t x0[32], x1[32];
+          const uint32_t col = t == 0 ? kColS1 : kColS2;
+          tmem_ld32(tmem + lane_base + col, x0);
+          tmem_ld32(tmem + lane_base + col + 32, x1);
+          tmem_wait_ld();
+          uint32_t* pk = t == 0 ? p1 : p2;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const int u = 2 * m;
+            pk[m] = pack_bf16x2(u >= rel ? __uint_as_float(x0[u]) : 0.f,
+                                u + 1 >= rel ? __uint_as_float(x0[u + 1]) : 0.f);
+            pk[16 + m] = pack_bf16x2(u + 32 >= rel ? __uint_as_float(x1[u]) : 0.f,
+                                     u + 33 >= rel ? __uint_as_float(x1[u + 1]) : 0.f);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < 32; ++m) p1[m] = p2[m] = 0u;
+      }
+      tc_fence_before();
+      mbar_arrive(s_read);
+      if (k >= 1 && !warp_wait(p_free, (k - 1) & 1, p.status, abort_flag)) return false;
+      store_p_row(sP1, r, p1);
+      store_p_row(sP2, r, p2);
+      fence_proxy_async_smem();
+      mbar_arrive(p_full);
+      return true;
+    };
+
+    griddep_wait();  // entering states come from the kernel before
+    load_state(blockIdx.x);
+    Cursor c;
+    cursor_init(p, c);
+    int prev_it = -1, prev_gc = -1;
+    for (; c.valid && ok; cursor_next(p, c)) {
+      if (!mask_block(c)) { ok = false; break; }
+      // the chunk before ended: its state step, after this block's mask
+      if (c.blk == 0 && prev_gc >= 0) {
+        const bool item_end = c.it != prev_it;
+        if (!state_step(prev_gc, item_end, prev_it, item_end ? c.it : -1)) { ok = false; break; }
+      }
+      prev_it = c.it;
+      prev_gc = c.gc;
+    }
+    if (ok && prev_gc >= 0) state_step(prev_gc, true, prev_it, -1);
+  } else {
+    // ------------------------------------------------------------ dv, dk out
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    int gc = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < p.items && ok; it += stride) {
+      int bg, tb, te;
+      span_of(p, it, bg, tb, te);
+      for (int n = 0; n < te - tb; ++n, ++gc) {
+        const int cs = te - 1 - n;
+        if (!warp_wait(o_full, gc & 1, p.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const int64_t row = (int64_t)cs * kChunk + r;
+        const bool valid = row < p.N;
+#pragma unroll 1
+        for (int t = 0; t < 2; ++t) {
+          __nv_bfloat16* out = (t == 0 ? p.dv : p.dk) + ((size_t)bg * p.N + row) * kHeadDim;
+          const uint32_t col = t == 0 ? kColDv : kColDk;
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t x0[32], x1[32];
+            tmem_ld32(tmem + lane_base + col + hh * 64, x0);
+            tmem_ld32(tmem + lane_base + col + hh * 64 + 32, x1);
+            tmem_wait_ld();
+            if (hh == 1) {
+              tc_fence_before();
+              mbar_arrive(&o_empty[t]);
+            }
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(out + hh * 64);
+#pragma unroll
+              for (int m = 0; m < 4; ++m)
+                dst[m] = make_uint4(
+                    pack_bf16x2(__uint_as_float(x0[8 * m]), __uint_as_float(x0[8 * m + 1])),
+                    pack_bf16x2(__uint_as_float(x0[8 * m + 2]), __uint_as_float(x0[8 * m + 3])),
+                    pack_bf16x2(__uint_as_float(x0[8 * m + 4]), __uint_as_float(x0[8 * m + 5])),
+                    pack_bf16x2(__uint_as_float(x0[8 * m + 6]), __uint_as_float(x0[8 * m + 7])));
+#pragma unroll
+              for (int m = 0; m < 4; ++m)
+                dst[4 + m] = make_uint4(
+                    pack_bf16x2(__uint_as_float(x1[8 * m]), __uint_as_float(x1[8 * m + 1])),
+                    pack_bf16x2(__uint_as_float(x1[8 * m + 2]), __uint_as_float(x1[8 * m + 3])),
+                    pack_bf16x2(__uint_as_float(x1[8 * m + 4]), __uint_as_float(x1[8 * m + 5])),
+                    pack_bf16x2(__uint_as_float(x1[8 * m + 6]), __uint_as_float(x1[8 * m + 7])));
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ent[bg][j] = dSf[bg] (nullable: 0) + sum over the group's heads h and the
+// spans j' > j of wsh[b*Hq + g*G + h][j'] (span 0 of wsh is not read): the
+// state entering span j of the group's backwards walk.
+__global__ void __launch_bounds__(256)
+    group_scan_kernel(const float4* __restrict__ wsh, const float4* __restrict__ dSf,
+                      float4* __restrict__ ent, int Hq, int Hkv, int G, int nspan, int n4) {
+  griddep_launch_dependents();  // the walk may start its copies
+  griddep_wait();               // the span states are complete
+  const int bg = blockIdx.y;
+  const int b = bg / Hkv, g = bg % Hkv;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n4) return;
+  float4 run = dSf ? dSf[(size_t)bg * n4 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = nspan - 1; j >= 0; --j) {
+    ent[((size_t)bg * nspan + j) * n4 + e] = run;
+    if (j == 0) break;
+    for (int h = 0; h < G; ++h) {
+      const float4 x = wsh[((size_t)(b * Hq + g * G + h) * nspan + j) * n4 + e];
+      run.x += x.x;
+      run.y += x.y;
+      run.z += x.z;
+      run.w += x.w;
+    }
+  }
+}
+
+}  // namespace
+
+int walk_spans(int units, int tiles, int sms, int G) {
+  // cost in chunk steps of one CTA: rounds x chunks per item, plus the span
+  // pass over Q and dO (2G key tiles per chunk against the walk's 2G + 4)
+  // spread over the SMs, plus a fixed cost for its two extra launches
+  const double r_span = (2.0 * G) / (2.0 * G + 4.0);
+  int best = 1;
+  double best_cost = 1e300;
+  for (int ns = 1; ns <= std::min(tiles, 256); ++ns) {
+    const int64_t items = (int64_t)units * ns;
+    const int64_t rounds = (items + sms - 1) / sms;
+    const int per = (tiles + ns - 1) / ns;
+    double cost = (double)(rounds * per);
+    if (ns > 1) cost += (double)(ns - 1) / ns * units * (double)tiles * r_span / sms + 1.0;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = ns;
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_group_scan(const float* wsh, const float* dSf, float* ent, int B, int Hq,
+                              int Hkv, int nspan, cudaStream_t stream) {
+  const int n4 = kHeadDim * kHeadDim / 4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((n4 + 255) / 256), (unsigned)(B * Hkv));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, group_scan_kernel, reinterpret_cast<const float4*>(wsh),
+                            reinterpret_cast<const float4*>(dSf), reinterpret_cast<float4*>(ent),
+                            Hq, Hkv, Hq / Hkv, nspan, n4);
+}
+
+cudaError_t launch_bwd_walk(const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                            const la_bf16* dO, la_bf16* dk, la_bf16* dv, const float* ws,
+                            float* s_out, unsigned* status, int B, int Hq, int Hkv, int64_t N,
+                            int nspan, int num_ctas, cudaStream_t stream, bool dependent) {
+  const int tiles = (int)((N + kChunk - 1) / kChunk);
+  const int64_t items = (int64_t)B * Hkv * nspan;
+  if (N <= 0 || nspan < 1 || nspan > tiles || items > 0x7fffffff || num_ctas <= 0)
+    return cudaErrorInvalidValue;
+  CUtensorMap map_q, map_do, map_k, map_v;
+  if (!make_tmap_bf16(&map_q, q, N, (int64_t)B * Hq, kKeyBlk) ||
+      !make_tmap_bf16(&map_do, dO, N, (int64_t)B * Hq, kKeyBlk) ||
+      !make_tmap_bf16(&map_k, k, N, (int64_t)B * Hkv, kChunk) ||
+      !make_tmap_bf16(&map_v, v, N, (int64_t)B * Hkv, kChunk))
+    return cudaErrorInvalidValue;
+  WalkParams p;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  p.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  p.dO = reinterpret_cast<const __nv_bfloat16*>(dO);
+  p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  p.ws = ws;
+  p.s_out = s_out;
+  p.status = status;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.nspan = nspan;
+  p.tiles_total = tiles;
+  p.items = (int)items;
+  cudaError_t e = cudaFuncSetAttribute(bwd_walk_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       WalkLayout::kBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min<int64_t>(items, num_ctas));
+  cfg.blockDim = dim3(320);
+  cfg.dynamicSmemBytes = WalkLayout::kBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, bwd_walk_kernel, map_q, map_do, map_k, map_v, p);
+}
+
+}  // namespace la

@@ -42,10 +42,12 @@ bool make_tmap_state(CUtensorMap* map, const void* base, int64_t units);
 // for the final state).  parts: each span
 // cut into `parts` sub-spans computed by separate CTAs (more CTAs when there
 // are few sequences and spans); ws then holds nspan * parts states per
-// sequence, in order.
+// sequence, in order.  first (parts == 1 only): spans before it are neither
+// computed nor written (a backwards walk never needs span 0's sum).
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
-                               cudaStream_t stream, bool skip_last = false, int parts = 1);
+                               cudaStream_t stream, bool skip_last = false, int parts = 1,
+                               int first = 0);
 // Persistent chunk loop: min(B*Hkv*nspan, num_ctas) CTAs walk the items (one
 // span of one (batch, kv head) sequence each, every query head of the group)
 // round-robin.  ws: entering state of item bg * nspan + j (nullptr: zero);
@@ -106,6 +108,22 @@ cudaError_t launch_decode_steps(float* S, const void* q, const void* k, const vo
 cudaError_t launch_forward_simt_f32(const float* q, const float* k, const float* v, float* o,
                                     const float* S_in, float* S_out, int B, int Hq, int Hkv,
                                     int64_t N, int d, int chunk, cudaStream_t stream);
+// Spans per kv group for the backward's dk/dv walk (each at least one
+// 128-token chunk): the makespan of the walk plus the span pass it needs.
+int walk_spans(int units, int tiles, int sms, int G);
+// ent[bg][j] <- dSf[bg] (nullable: 0) + sum over the group's query heads and
+// the spans after j of wsh[b*Hq + h][j'] (per-head span states of Q^T dO,
+// span 0 not read); launched as a programmatic dependent of the span pass.
+cudaError_t launch_group_scan(const float* wsh, const float* dSf, float* ent, int B, int Hq,
+                              int Hkv, int nspan, cudaStream_t stream);
+// dk, dv [B*Hkv, N, 128] of the backward in one anti-causal walk per (kv
+// group, span): ws holds the entering state of item bg * nspan + j (nullable:
+// zero; may be s_out when nspan == 1), s_out (nullable) receives dS0 from the
+// items of span 0.  1 <= nspan <= ceil(N / 128).
+cudaError_t launch_bwd_walk(const la_bf16* q, const la_bf16* k, const la_bf16* v,
+                            const la_bf16* dO, la_bf16* dk, la_bf16* dv, const float* ws,
+                            float* s_out, unsigned* status, int B, int Hq, int Hkv, int64_t N,
+                            int nspan, int num_ctas, cudaStream_t stream, bool dependent);
 cudaError_t launch_selftest_wait(unsigned* status, int64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace la

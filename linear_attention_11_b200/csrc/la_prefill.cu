@@ -29,7 +29,8 @@ struct SpanParams {
   float* ws;
   unsigned* status;
   int nspan, tiles_total;
-  int nrun;  // spans computed per (batch, kv head): the first nrun of the nspan
+  int nrun;   // spans computed per (batch, kv head): nrun of the nspan from `first` on
+  int first;
 };
 
 template <int T, int STAGES>
@@ -58,7 +59,7 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
 
   griddep_launch_dependents();  // the scan may be scheduled; it waits for this grid
-  const int j = blockIdx.x % p.nrun;
+  const int j = p.first + (int)(blockIdx.x % p.nrun);
   const int bg = blockIdx.x / p.nrun;
   const int tile_begin = (int)(((int64_t)j * p.tiles_total) / p.nspan);
   const int tile_end = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
@@ -173,12 +174,12 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
                                const CUtensorMap& v, float* ws, unsigned* status,
-                               cudaStream_t stream, bool skip_last, int parts) {
-  if (parts < 1) return cudaErrorInvalidValue;
-  const int nparts = g.nspan * parts;                        // sub-spans per sequence
-  const int nrun = (g.nspan - (skip_last ? 1 : 0)) * parts;  // of them computed
+                               cudaStream_t stream, bool skip_last, int parts, int first) {
+  if (parts < 1 || first < 0 || (first > 0 && parts != 1)) return cudaErrorInvalidValue;
+  const int nparts = g.nspan * parts;                                // sub-spans per sequence
+  const int nrun = (g.nspan - (skip_last ? 1 : 0)) * parts - first;  // of them computed
   if (nrun <= 0) return cudaSuccess;
-  SpanParams p{ws, status, nparts, g.tiles_total, nrun};
+  SpanParams p{ws, status, nparts, g.tiles_total, nrun, first};
   const dim3 grid((unsigned)(g.B * g.Hkv * nrun));
   cudaError_t e;
   if (g.tile == 64) {

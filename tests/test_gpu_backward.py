@@ -46,6 +46,8 @@ SMALL = [
     (1, 4, 1, 64, 64, False),
     (1, 3, 1, 385, 128, True),
     (1, 2, 1, 1, 64, True),
+    (64, 4, 4, 200, 64, True),   # one span per group, CTAs with two groups
+    (3, 8, 1, 2000, 128, True),  # eight query heads per group, many spans
 ]
 
 
