@@ -28,10 +28,11 @@
 // the later spans' sums, from group_scan_kernel) is read at the item start,
 // and the item of span 0 writes dS0 at its end.
 // Roles (320 threads): warp 0 lane 0 streams key blocks (Q and dO of one head
-// half-chunk) through a three-stage ring, lane 1 the K/V tiles of each chunk
-// and L2 prefetches of the next chunk; warp 1 owns the tensor memory and
-// issues the MMAs, scores two blocks ahead; warps 2-5 mask the scores and
-// convert the state; warps 6-9 write dv and dk rows out.
+// half-chunk) through a three-stage ring and prefetches the blocks six ahead
+// into L2, lane 1 the K/V tiles of each chunk (and the next chunk's into L2);
+// warp 1 owns the tensor memory and
+// issues the MMAs, scores two blocks ahead; warps 2-5 mask S1, convert the
+// state and write dv rows out; warps 6-9 mask S2 and write dk rows out.
 // TMEM: dv at column 0, dk at 128, S1 at 256, S2 at 320, D at 384.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -48,6 +49,7 @@ namespace {
 constexpr int kChunk = 128;                         // tokens per chunk
 constexpr int kKeyBlk = 64;                         // tokens per key block
 constexpr int kRing = 3;                            // key-block stages
+constexpr int kPrefetch = 6;                        // key blocks prefetched into L2 ahead
 constexpr int kChunkBytes = kChunk * kHeadDim * 2;  // 32 KB: K_c or V_c
 constexpr int kBlkBytes = kKeyBlk * kHeadDim * 2;   // 16 KB: Q or dO of one block
 constexpr int kBlkHalf = kKeyBlk * 128;             // 8 KB: 64 columns of a key block
@@ -191,8 +193,8 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
     mbar_init(a_full, 1);
-    mbar_init(s_read, 128);
-    mbar_init(p_full, 128);
+    mbar_init(s_read, 256);
+    mbar_init(p_full, 256);
     mbar_init(p_free, 1);
     mbar_init(o_full, 1);
     mbar_init(&o_empty[0], 128);
@@ -219,10 +221,28 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&map_q);
       prefetch_tmap(&map_do);
       const uint64_t pol = policy_evict_first();
-      Cursor c;
+      // each block's rows are also prefetched into L2 kPrefetch blocks before
+      // its copy, so the copies hit L2 while little data waits there
+      auto prefetch_block = [&](const Cursor& x) {
+        const int halves = x.nb / p.G;
+        const int h = x.blk / halves, j = x.blk % halves;
+        const int b = x.bg / p.Hkv, g = x.bg % p.Hkv;
+        const int64_t t0 = (int64_t)x.cs * kChunk + j * kKeyBlk;
+        const uint32_t bytes = (uint32_t)(std::min<int64_t>(kKeyBlk, p.N - t0) * kHeadDim * 2);
+        const size_t off = ((size_t)(b * p.Hq + g * p.G + h) * p.N + t0) * kHeadDim;
+        prefetch_l2_bulk(p.q + off, bytes);
+        prefetch_l2_bulk(p.dO + off, bytes);
+      };
+      Cursor c, pf;
       cursor_init(p, c);
+      cursor_init(p, pf);
+      for (int n = 0; n < kPrefetch && pf.valid; ++n, cursor_next(p, pf)) prefetch_block(pf);
       int issued = 0;
       for (; c.valid; cursor_next(p, c)) {
+        if (pf.valid) {
+          prefetch_block(pf);
+          cursor_next(p, pf);
+        }
         const int s = c.i % kRing;
         if (c.i >= kRing &&
             !mbar_wait(&ring_empty[s], ((c.i / kRing) - 1) & 1, p.status, abort_flag))
@@ -246,20 +266,14 @@ __global__ void __launch_bounds__(320, 1)
           mbar_wait_drain(&ring_full[k % kRing], (k / kRing) & 1);
       }
     } else if (lane == 1) {
-      // K_c, V_c per chunk; L2 prefetch of the next chunk's Q, dO (every head
-      // of the group), K, V, and of the next item's entering state
+      // K_c, V_c per chunk; L2 prefetch of the next chunk's K, V and of the
+      // next item's entering state
       prefetch_tmap(&map_k);
       prefetch_tmap(&map_v);
       const uint64_t pol = policy_evict_first();
       auto prefetch_chunk = [&](int bg, int cs) {
         const int64_t t0 = (int64_t)cs * kChunk;
         const uint32_t bytes = (uint32_t)(std::min<int64_t>(kChunk, p.N - t0) * kHeadDim * 2);
-        const int b = bg / p.Hkv, g = bg % p.Hkv;
-        for (int h = 0; h < p.G; ++h) {
-          const size_t off = ((size_t)(b * p.Hq + g * p.G + h) * p.N + t0) * kHeadDim;
-          prefetch_l2_bulk(p.q + off, bytes);
-          prefetch_l2_bulk(p.dO + off, bytes);
-        }
         const size_t off = ((size_t)bg * p.N + t0) * kHeadDim;
         prefetch_l2_bulk(p.k + off, bytes);
         prefetch_l2_bulk(p.v + off, bytes);
@@ -351,32 +365,44 @@ __global__ void __launch_bounds__(320, 1)
         const int k = c.i;
         const bool first = c.blk == 0, last = c.blk == c.nb - 1;
         if (!mbar_wait(p_full, k & 1, p.status, abort_flag)) break;
-        if (first && c.gc >= 1 &&
-            (!mbar_wait(&o_empty[0], (c.gc - 1) & 1, p.status, abort_flag) ||
-             !mbar_wait(&o_empty[1], (c.gc - 1) & 1, p.status, abort_flag)))
-          break;
         tc_fence_after();
         const int s = k % kRing;
         const uint32_t qa = sQ(s), doa = sDO(s);
+        // dk += P2 Q (a chunk's first block starts dk once it has been read
+        // out), then V_c D^T; dv += P1 dO, then K_c D
+        if (first && c.gc >= 1 && !mbar_wait(&o_empty[1], (c.gc - 1) & 1, p.status, abort_flag))
+          break;
+        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kKeyBlk / 16; ++kk) {  // dv += P1 dO, dk += P2 Q
-          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-          mma_ss(tmem + kColDv, smem_desc_sw128(sP1 + kk * 32, 16, 1024),
-                 smem_desc_sw128(doa + kk * 2048, kBlkHalf, 1024), IDESC_PV, acc);
+        for (int kk = 0; kk < kKeyBlk / 16; ++kk)
           mma_ss(tmem + kColDk, smem_desc_sw128(sP2 + kk * 32, 16, 1024),
-                 smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024), IDESC_PV, acc);
-        }
-        if (first) {  // dv += K_c D, dk += V_c D^T from the bf16 copy of D_c
+                 smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024), IDESC_PV,
+                 (first && kk == 0) ? 0u : 1u);
+        if (first) {
           if (!mbar_wait(sb_full, c.gc & 1, p.status, abort_flag)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t koff = (uint32_t)((kk & 3) * 32);
             const uint32_t ch = (uint32_t)(kk >> 2);
-            mma_ss(tmem + kColDv, smem_desc_sw128(sK + ch * kHalf + koff, 16, 1024),
-                   smem_desc_sw128(sS + kk * 2048, kHalf, 1024), IDESC_KD, 1u);
             mma_ss(tmem + kColDk, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
                    smem_desc_sw128(sS + ch * kHalf + koff, 16, 1024), IDESC_VDT, 1u);
+          }
+          if (c.gc >= 1 && !mbar_wait(&o_empty[0], (c.gc - 1) & 1, p.status, abort_flag)) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < kKeyBlk / 16; ++kk)
+          mma_ss(tmem + kColDv, smem_desc_sw128(sP1 + kk * 32, 16, 1024),
+                 smem_desc_sw128(doa + kk * 2048, kBlkHalf, 1024), IDESC_PV,
+                 (first && kk == 0) ? 0u : 1u);
+        if (first) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (uint32_t)((kk & 3) * 32);
+            const uint32_t ch = (uint32_t)(kk >> 2);
+            mma_ss(tmem + kColDv, smem_desc_sw128(sK + ch * kHalf + koff, 16, 1024),
+                   smem_desc_sw128(sS + kk * 2048, kHalf, 1024), IDESC_KD, 1u);
           }
           inter_gc = c.gc;
           if (kv_pending == c.gc) {
@@ -384,11 +410,11 @@ __global__ void __launch_bounds__(320, 1)
             kv_pending = -1;
           }
         }
+        mma_commit(p_free);  // the next block's P may be stored during D's update
 #pragma unroll
         for (int kk = 0; kk < kKeyBlk / 16; ++kk)  // D += Q^T dO (both MN-major)
           mma_ss(tmem + kColS, smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024),
                  smem_desc_sw128(doa + kk * 2048, kBlkHalf, 1024), IDESC_D, 1u);
-        mma_commit(p_free);
         mma_commit(&ring_empty[s]);
         if (last) {
           mma_commit(o_full);
@@ -401,11 +427,19 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait_drain(mma_done, 0);
     }
     __syncwarp();
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ masks, state
+  } else {
+    // ------------------------------------------------------------ math warpgroups
+    // Warps 2-5 mask S1 into P1, convert the state and write dv; warps 6-9
+    // mask S2 into P2 and write dk.  Each thread owns TMEM lane r = chunk row r.
+    const bool wg1 = warp < 6;
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // TMEM lane = chunk row = state row
+    const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t col_s = wg1 ? kColS1 : kColS2;
+    const uint32_t col_o = wg1 ? kColDv : kColDk;
+    const uint32_t sP = wg1 ? sP1 : sP2;
+    __nv_bfloat16* const out_base = wg1 ? p.dv : p.dk;
+    uint64_t* const my_empty = &o_empty[wg1 ? 0 : 1];
     bool ok = true;
 
     // entering state of item it -> D in tensor memory and its bf16 copy
@@ -434,8 +468,9 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(sb_full);
     };
 
-    // after chunk gcd's state update: the bf16 copy for the next chunk, or at
-    // an item's end dS0 out (span 0) and the next item's entering state in
+    // (warps 2-5) after chunk gcd's state update: the bf16 copy for the next
+    // chunk, or at an item's end dS0 out (span 0) and the next item's
+    // entering state in
     auto state_step = [&](int gcd, bool item_end, int done_it, int next_it) -> bool {
       if (!warp_wait(s_full, gcd & 1, p.status, abort_flag)) return false;
       tc_fence_after();
@@ -474,7 +509,7 @@ __global__ void __launch_bounds__(320, 1)
       return true;
     };
 
-    // scores of block c -> masked bf16 P tiles in smem
+    // this warpgroup's score tile of block c -> masked bf16 P tile in smem
     auto mask_block = [&](const Cursor& c) -> bool {
       const int k = c.i;
       const int halves = c.nb / p.G;
@@ -485,105 +520,100 @@ __global__ void __launch_bounds__(320, 1)
       // u >= r - 64 j.  Rows 64..127 keep nothing of the first half.
       const int rel = r - kKeyBlk * j;
       const bool none = j == 0 && quarter >= 2;
-      uint32_t p1[32], p2[32];
+      uint32_t pk[32];
       if (!none) {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tmem + lane_base + col_s, x0);
+        tmem_ld32(tmem + lane_base + col_s + 32, x1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_read);  // the score columns may be overwritten
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          uint32_t x0[32], x1[32];
-          const uint32_t col = t == 0 ? kColS1 : kColS2;
-          tmem_ld32(tmem + lane_base + col, x0);
-          tmem_ld32(tmem + lane_base + col + 32, x1);
-          tmem_wait_ld();
-          uint32_t* pk = t == 0 ? p1 : p2;
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const int u = 2 * m;
-            pk[m] = pack_bf16x2(u >= rel ? __uint_as_float(x0[u]) : 0.f,
-                                u + 1 >= rel ? __uint_as_float(x0[u + 1]) : 0.f);
-            pk[16 + m] = pack_bf16x2(u + 32 >= rel ? __uint_as_float(x1[u]) : 0.f,
-                                     u + 33 >= rel ? __uint_as_float(x1[u + 1]) : 0.f);
-          }
+        for (int m = 0; m < 16; ++m) {
+          const int u = 2 * m;
+          pk[m] = pack_bf16x2(u >= rel ? __uint_as_float(x0[u]) : 0.f,
+                              u + 1 >= rel ? __uint_as_float(x0[u + 1]) : 0.f);
+          pk[16 + m] = pack_bf16x2(u + 32 >= rel ? __uint_as_float(x1[u]) : 0.f,
+                                   u + 33 >= rel ? __uint_as_float(x1[u + 1]) : 0.f);
         }
       } else {
+        mbar_arrive(s_read);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) p1[m] = p2[m] = 0u;
+        for (int m = 0; m < 32; ++m) pk[m] = 0u;
       }
-      tc_fence_before();
-      mbar_arrive(s_read);
       if (k >= 1 && !warp_wait(p_free, (k - 1) & 1, p.status, abort_flag)) return false;
-      store_p_row(sP1, r, p1);
-      store_p_row(sP2, r, p2);
+      store_p_row(sP, r, pk);
       fence_proxy_async_smem();
       mbar_arrive(p_full);
       return true;
     };
 
-    griddep_wait();  // entering states come from the kernel before
-    load_state(blockIdx.x);
+    // this warpgroup's accumulator of chunk gcd (rows of chunk cs of group
+    // bg) -> bf16 rows in global memory, released once read out
+    auto write_out = [&](int gcd, int bg, int cs) -> bool {
+      if (!warp_wait(o_full, gcd & 1, p.status, abort_flag)) return false;
+      tc_fence_after();
+      const int64_t row = (int64_t)cs * kChunk + r;
+      const bool valid = row < p.N;
+      uint4* dst = reinterpret_cast<uint4*>(out_base + ((size_t)bg * p.N + (valid ? row : 0)) *
+                                                           kHeadDim);
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tmem + lane_base + col_o + hh * 64, x0);
+        tmem_ld32(tmem + lane_base + col_o + hh * 64 + 32, x1);
+        tmem_wait_ld();
+        if (hh == 1) {
+          tc_fence_before();
+          mbar_arrive(my_empty);
+        }
+        if (valid) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            dst[hh * 8 + m] = make_uint4(
+                pack_bf16x2(__uint_as_float(x0[8 * m]), __uint_as_float(x0[8 * m + 1])),
+                pack_bf16x2(__uint_as_float(x0[8 * m + 2]), __uint_as_float(x0[8 * m + 3])),
+                pack_bf16x2(__uint_as_float(x0[8 * m + 4]), __uint_as_float(x0[8 * m + 5])),
+                pack_bf16x2(__uint_as_float(x0[8 * m + 6]), __uint_as_float(x0[8 * m + 7])));
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            dst[hh * 8 + 4 + m] = make_uint4(
+                pack_bf16x2(__uint_as_float(x1[8 * m]), __uint_as_float(x1[8 * m + 1])),
+                pack_bf16x2(__uint_as_float(x1[8 * m + 2]), __uint_as_float(x1[8 * m + 3])),
+                pack_bf16x2(__uint_as_float(x1[8 * m + 4]), __uint_as_float(x1[8 * m + 5])),
+                pack_bf16x2(__uint_as_float(x1[8 * m + 6]), __uint_as_float(x1[8 * m + 7])));
+        }
+      }
+      return true;
+    };
+
+    if (wg1) {
+      griddep_wait();  // entering states come from the kernel before
+      load_state(blockIdx.x);
+    }
     Cursor c;
     cursor_init(p, c);
-    int prev_it = -1, prev_gc = -1;
+    int prev_it = -1, prev_gc = -1, prev_bg = 0, prev_cs = 0;
     for (; c.valid && ok; cursor_next(p, c)) {
       if (!mask_block(c)) { ok = false; break; }
-      // the chunk before ended: its state step, after this block's mask
+      // the chunk before ended: its state step and output, after this
+      // block's mask (which the next MMAs need first)
       if (c.blk == 0 && prev_gc >= 0) {
         const bool item_end = c.it != prev_it;
-        if (!state_step(prev_gc, item_end, prev_it, item_end ? c.it : -1)) { ok = false; break; }
+        if (wg1 && !state_step(prev_gc, item_end, prev_it, item_end ? c.it : -1)) {
+          ok = false;
+          break;
+        }
+        if (!write_out(prev_gc, prev_bg, prev_cs)) { ok = false; break; }
       }
       prev_it = c.it;
       prev_gc = c.gc;
+      prev_bg = c.bg;
+      prev_cs = c.cs;
     }
-    if (ok && prev_gc >= 0) state_step(prev_gc, true, prev_it, -1);
-  } else {
-    // ------------------------------------------------------------ dv, dk out
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    int gc = 0;
-    bool ok = true;
-    for (int it = blockIdx.x; it < p.items && ok; it += stride) {
-      int bg, tb, te;
-      span_of(p, it, bg, tb, te);
-      for (int n = 0; n < te - tb; ++n, ++gc) {
-        const int cs = te - 1 - n;
-        if (!warp_wait(o_full, gc & 1, p.status, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const int64_t row = (int64_t)cs * kChunk + r;
-        const bool valid = row < p.N;
-#pragma unroll 1
-        for (int t = 0; t < 2; ++t) {
-          __nv_bfloat16* out = (t == 0 ? p.dv : p.dk) + ((size_t)bg * p.N + row) * kHeadDim;
-          const uint32_t col = t == 0 ? kColDv : kColDk;
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t x0[32], x1[32];
-            tmem_ld32(tmem + lane_base + col + hh * 64, x0);
-            tmem_ld32(tmem + lane_base + col + hh * 64 + 32, x1);
-            tmem_wait_ld();
-            if (hh == 1) {
-              tc_fence_before();
-              mbar_arrive(&o_empty[t]);
-            }
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(out + hh * 64);
-#pragma unroll
-              for (int m = 0; m < 4; ++m)
-                dst[m] = make_uint4(
-                    pack_bf16x2(__uint_as_float(x0[8 * m]), __uint_as_float(x0[8 * m + 1])),
-                    pack_bf16x2(__uint_as_float(x0[8 * m + 2]), __uint_as_float(x0[8 * m + 3])),
-                    pack_bf16x2(__uint_as_float(x0[8 * m + 4]), __uint_as_float(x0[8 * m + 5])),
-                    pack_bf16x2(__uint_as_float(x0[8 * m + 6]), __uint_as_float(x0[8 * m + 7])));
-#pragma unroll
-              for (int m = 0; m < 4; ++m)
-                dst[4 + m] = make_uint4(
-                    pack_bf16x2(__uint_as_float(x1[8 * m]), __uint_as_float(x1[8 * m + 1])),
-                    pack_bf16x2(__uint_as_float(x1[8 * m + 2]), __uint_as_float(x1[8 * m + 3])),
-                    pack_bf16x2(__uint_as_float(x1[8 * m + 4]), __uint_as_float(x1[8 * m + 5])),
-                    pack_bf16x2(__uint_as_float(x1[8 * m + 6]), __uint_as_float(x1[8 * m + 7])));
-            }
-          }
-        }
-      }
+    if (ok && prev_gc >= 0) {
+      if (wg1) ok = state_step(prev_gc, true, prev_it, -1);
+      if (ok) write_out(prev_gc, prev_bg, prev_cs);
     }
   }
 
