@@ -60,8 +60,9 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
 // where they are a large share of the bytes (see stage_states_pays).
 // qdiv: query rows of head h come from head h / qdiv of the query tensor map;
 // reverse: anti-causal walk (sum over s >= t), each span from its end, tile
-// 128 only (the backward); transpose_in (reverse only): entering states read
-// transposed (not with s_out == ws).
+// 128 only (per-head walks; la_backward takes dk and dv from the grouped walk
+// of la_backward_walk.cu instead); transpose_in (reverse only): entering
+// states read transposed (not with s_out == ws).
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
                                    cudaStream_t stream, bool dependent, bool stage_states,

@@ -58,9 +58,9 @@ struct PersistParams {
 // memory by bulk tensor copies (map_s over the states, [units, 128, 128]),
 // loaded an item ahead by a third copy lane; without it the math warps read
 // and write them row by row.  kDedO: a dedicated output staging tile (else
-// the output goes through the Q slot).  kRev: the anti-causal passes of the
-// backward (sum over s >= t, spans walked from their end, entering states
-// optionally read transposed).
+// the output goes through the Q slot).  kRev: anti-causal per-head passes
+// (sum over s >= t, spans walked from their end, entering states optionally
+// read transposed); la_backward now uses the grouped walk instead.
 template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kRev>
 __global__ void __launch_bounds__(320, 1)
     prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
