@@ -74,3 +74,29 @@ def test_selftest_and_status_reject_bad_arguments(la):
     lib = _raw(la)
     assert lib.la_selftest_wait(0, None) == 1
     assert lib.la_device_status(None, 0) == 1
+
+
+def test_backward_rejects_null_and_misaligned_pointers(la):
+    lib = _raw(la)
+    p, m = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 8)
+    shape = (1, 2, 2, 16, 128, 64, None)
+    assert lib.la_backward(None, p, p, p, None, None, p, p, p, None, *shape) == 1  # q
+    assert lib.la_backward(p, p, p, None, None, None, p, p, p, None, *shape) == 1  # dO
+    assert lib.la_backward(p, p, p, p, None, None, p, p, None, None, *shape) == 1  # dv
+    assert lib.la_backward(p, p, p, m, None, None, p, p, p, None, *shape) == 1     # dO misaligned
+    assert lib.la_backward(p, p, p, p, None, m, p, p, p, None, *shape) == 1        # dSf misaligned
+    assert lib.la_backward(p, p, p, p, None, None, p, p, p, m, *shape) == 1        # dS0 misaligned
+
+
+def test_state_prefix_rejects_bad_arguments(la):
+    lib = _raw(la)
+    per = 1 * 2 * 128 * 128 * 4                  # bytes of one segment's states
+    states, S = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 3 * per)
+    assert lib.la_state_prefix(states, None, S, 3, 3, 1, 2, 128, None) == 1   # seg >= nseg
+    assert lib.la_state_prefix(states, None, S, 3, -1, 1, 2, 128, None) == 1  # seg < 0
+    assert lib.la_state_prefix(states, None, S, 0, 0, 1, 2, 128, None) == 1   # nseg < 1
+    assert lib.la_state_prefix(None, None, S, 3, 1, 1, 2, 128, None) == 1    # states null
+    inside = ctypes.c_void_p((1 << 20) + per)                                  # S within states
+    assert lib.la_state_prefix(states, None, inside, 3, 1, 1, 2, 128, None) == 1
+    odd = ctypes.c_void_p((1 << 20) + 3 * per + 4)                             # misaligned S
+    assert lib.la_state_prefix(states, None, odd, 3, 1, 1, 2, 128, None) == 1
