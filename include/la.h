@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
   LA_OK = 0,
   LA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, Hq % Hkv != 0, misalignment, overlap */
-  LA_ERR_UNSUPPORTED = 2, /* head dim or chunk size this build does not implement */
+  LA_ERR_UNSUPPORTED = 2, /* head dim or chunk size the library does not implement */
   LA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   LA_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired (see la_device_status) */
   LA_ERR_WORKSPACE = 5    /* workspace pointer missing, misaligned or too small */
