@@ -379,10 +379,20 @@ def run_ours(args, w):
                          stream)
         tb /= reps
         bbytes = elt * (3 * B * Hq * N * d + 4 * B * Hkv * N * d)  # q, dO, dq + k, v, dk, dv
+        # chunk-form FLOPs: the dq pass as the forward; the dk, dv walk per
+        # query-head token 2 scores + 2 products over 128-row chunks (8*128*d)
+        # and the state update (2 d^2), per kv token K_c D and V_c D^T (4 d^2)
+        bflops = (B * Hq * N * (4 * chunk * d + 4 * d * d)
+                  + B * Hq * N * (8 * 128 * d + 2 * d * d) + B * Hkv * N * 4 * d * d)
+        t_hbm = bbytes / (pk["hbm_gbs"] * 1e9)
+        t_tc = bflops / (pk["bf16_tflops"] * 1e12)
         backward = {"ms_per_step": tb * 1e3, "mtok_s": world * B * N / tb / 1e6,
                     "algorithmic_gb_s": bbytes / tb / 1e9,
                     "frac_of_hbm_roofline": bbytes / tb / 1e9 / pk["hbm_gbs"],
-                    "bytes": bbytes, "clocks": bclk,
+                    "tflops_chunk_form": bflops / tb / 1e12,
+                    "bound": "tensor" if t_tc > t_hbm else "hbm",
+                    "frac_of_roofline": max(t_hbm, t_tc) / tb,
+                    "bytes": bbytes, "flops": bflops, "clocks": bclk,
                     "passes": "dq causal (grouped) + one anti-causal dk, dv walk per kv group"}
         del dOd
 
