@@ -111,9 +111,41 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _dims(q, k):
+def _on_device(t) -> bool:
+    return t.is_cuda
+
+
+def _need(fn, name, t, dtype=None, device=True):
+    """Reject what the library would misread: host memory where device memory
+    is expected (or the reverse), another element type, or a strided view."""
+    if t is None:
+        return
+    if _on_device(t) != device:
+        raise ValueError(f"{fn}: {name} must be a {'CUDA' if device else 'host'} tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{fn}: {name} must be {dtype}, not {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{fn}: {name} must be contiguous")
+
+
+def _qkv(fn, q, k, v, o=None, dtype=torch.bfloat16, device=True):
+    """q, o [B,Hq,N,d] and k, v [B,Hkv,N,d] of one dtype -> (B, Hq, Hkv, N, d)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _need(fn, name, t, dtype, device)
+    if (q.dim() != 4 or k.dim() != 4 or k.shape != v.shape or k.shape[0] != q.shape[0]
+            or k.shape[2:] != q.shape[2:] or (o is not None and o.shape != q.shape)):
+        raise ValueError(f"{fn}: expected q, o [B,Hq,N,d] and k, v [B,Hkv,N,d]; got q "
+                         f"{tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}"
+                         + ("" if o is None else f", o {tuple(o.shape)}"))
     B, Hq, N, d = q.shape
     return B, Hq, k.shape[1], N, d
+
+
+def _state(fn, name, S, B, Hkv, d):
+    """S [B,Hkv,d,d] fp32 on the device (or None)."""
+    _need(fn, name, S, torch.float32)
+    if S is not None and tuple(S.shape) != (B, Hkv, d, d):
+        raise ValueError(f"{fn}: {name} must be [{B},{Hkv},{d},{d}], not {tuple(S.shape)}")
 
 
 def la_status_string(code: int) -> str:
@@ -122,9 +154,9 @@ def la_status_string(code: int) -> str:
 
 def la_forward(q, k, v, o=None, chunk: int = 64, stream=None):
     """O for q [B,Hq,N,d], k, v [B,Hkv,N,d] (bf16, CUDA); zero initial state."""
+    B, Hq, Hkv, N, d = _qkv("la_forward", q, k, v, o)
     if o is None:
         o = torch.empty_like(q)
-    B, Hq, Hkv, N, d = _dims(q, k)
     _check("la_forward", load_library().la_forward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, N, d, chunk, _stream(stream)))
     return o
@@ -132,9 +164,10 @@ def la_forward(q, k, v, o=None, chunk: int = 64, stream=None):
 
 def la_forward_state(q, k, v, S=None, o=None, chunk: int = 64, stream=None):
     """As la_forward; S [B,Hkv,d,d] fp32 (in: initial state, out: final state)."""
+    B, Hq, Hkv, N, d = _qkv("la_forward_state", q, k, v, o)
+    _state("la_forward_state", "S", S, B, Hkv, d)
     if o is None:
         o = torch.empty_like(q)
-    B, Hq, Hkv, N, d = _dims(q, k)
     _check("la_forward_state", load_library().la_forward_state(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, _stream(stream)))
     return o
@@ -145,7 +178,9 @@ def la_forward_workspace_bytes(B, Hq, Hkv, N, d, chunk) -> int:
 
 
 def la_forward_ws(q, k, v, o, S, workspace, chunk: int = 64, stream=None):
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _qkv("la_forward_ws", q, k, v, o)
+    _state("la_forward_ws", "S", S, B, Hkv, d)
+    _need("la_forward_ws", "workspace", workspace)
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("la_forward_ws", load_library().la_forward_ws(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk,
@@ -156,9 +191,10 @@ def la_forward_ws(q, k, v, o, S, workspace, chunk: int = 64, stream=None):
 def la_forward_noalloc(q, k, v, S=None, o=None, chunk: int = 64, stream=None):
     """As la_forward_state, with the library's fixed device scratch instead of
     an allocation (for callers that cannot allocate device memory)."""
+    B, Hq, Hkv, N, d = _qkv("la_forward_noalloc", q, k, v, o)
+    _state("la_forward_noalloc", "S", S, B, Hkv, d)
     if o is None:
         o = torch.empty_like(q)
-    B, Hq, Hkv, N, d = _dims(q, k)
     _check("la_forward_noalloc", load_library().la_forward_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, _stream(stream)))
     return o
@@ -167,9 +203,10 @@ def la_forward_noalloc(q, k, v, S=None, o=None, chunk: int = 64, stream=None):
 def la_forward_host(q, k, v, o=None, S=None, chunk: int = 64, piece: int = 0, stream=None):
     """Prefill from and to pinned host tensors (q, k, v, o on the CPU, pinned);
     S, if given, is a CUDA tensor.  Asynchronous on `stream`."""
+    B, Hq, Hkv, N, d = _qkv("la_forward_host", q, k, v, o, device=False)
+    _state("la_forward_host", "S", S, B, Hkv, d)
     if o is None:
         o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    B, Hq, Hkv, N, d = _dims(q, k)
     _check("la_forward_host", load_library().la_forward_host(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, piece,
         _stream(stream)))
@@ -183,7 +220,9 @@ def la_prefill_fused_workspace_bytes(B, Hq, Hkv, N, d, chunk, nspan=0) -> int:
 def la_prefill_fused(q, k, v, o, S, workspace, chunk: int = 64, nspan: int = 0,
                      lookahead: int = 0, stream=None):
     """The single-pass prefill with an explicit span count and lookahead (0 = automatic)."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _qkv("la_prefill_fused", q, k, v, o)
+    _state("la_prefill_fused", "S", S, B, Hkv, d)
+    _need("la_prefill_fused", "workspace", workspace)
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("la_prefill_fused", load_library().la_prefill_fused(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, nspan, lookahead,
@@ -199,18 +238,22 @@ def la_prefill_plan(B, Hq, Hkv, N, d, chunk) -> la_plan:
 
 
 def la_prefill_span_states(k, v, plan: la_plan, ws, stream=None):
-    B, Hkv, N, d = k.shape
+    B, _, Hkv, N, d = _qkv("la_prefill_span_states", k, k, v)
+    _need("la_prefill_span_states", "ws", ws)
     _check("la_prefill_span_states", load_library().la_prefill_span_states(
         _ptr(k), _ptr(v), B, Hkv, N, d, ctypes.byref(plan), _ptr(ws), _stream(stream)))
 
 
 def la_prefill_scan(ws, S, plan: la_plan, B, Hkv, d, stream=None):
+    _need("la_prefill_scan", "ws", ws)
+    _state("la_prefill_scan", "S", S, B, Hkv, d)
     _check("la_prefill_scan", load_library().la_prefill_scan(
         _ptr(ws), _ptr(S), B, Hkv, d, ctypes.byref(plan), _stream(stream)))
 
 
 def la_prefill_main(q, k, v, o, ws, plan: la_plan, stream=None):
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _qkv("la_prefill_main", q, k, v, o)
+    _need("la_prefill_main", "ws", ws)
     _check("la_prefill_main", load_library().la_prefill_main(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ws), B, Hq, Hkv, N, d, ctypes.byref(plan),
         _stream(stream)))
@@ -218,7 +261,8 @@ def la_prefill_main(q, k, v, o, ws, plan: la_plan, stream=None):
 
 def la_segment_state(k, v, S=None, chunk: int = 64, stream=None):
     """K^T V of one segment's k, v [B,Hkv,N,d] (bf16, CUDA) -> S [B,Hkv,d,d] fp32."""
-    B, Hkv, N, d = k.shape
+    B, _, Hkv, N, d = _qkv("la_segment_state", k, k, v)
+    _state("la_segment_state", "S", S, B, Hkv, d)
     if S is None:
         S = torch.empty(B, Hkv, d, d, dtype=torch.float32, device=k.device)
     _check("la_segment_state", load_library().la_segment_state(
@@ -228,7 +272,13 @@ def la_segment_state(k, v, S=None, chunk: int = 64, stream=None):
 
 def la_state_prefix(states, seg: int, S0=None, S=None, stream=None):
     """S0 (or 0) + sum of states[:seg]; states [nseg,B,Hkv,d,d] fp32 (CUDA)."""
+    _need("la_state_prefix", "states", states, torch.float32)
+    if states.dim() != 5 or states.shape[3] != states.shape[4]:
+        raise ValueError(f"la_state_prefix: states must be [nseg,B,Hkv,d,d], not "
+                         f"{tuple(states.shape)}")
     nseg, B, Hkv, d, _ = states.shape
+    _state("la_state_prefix", "S0", S0, B, Hkv, d)
+    _state("la_state_prefix", "S", S, B, Hkv, d)
     if S is None:
         S = torch.empty(B, Hkv, d, d, dtype=torch.float32, device=states.device)
     _check("la_state_prefix", load_library().la_state_prefix(
@@ -240,7 +290,9 @@ def la_backward(q, k, v, dO, S0=None, dSf=None, want_dS0: bool = False, chunk: i
                 stream=None):
     """Gradients (dq, dk, dv, dS0 or None) of the prefill for output gradient dO
     and final-state gradient dSf (CUDA tensors; S0 the forward's initial state)."""
-    B, Hq, Hkv, N, d = _dims(q, k)
+    B, Hq, Hkv, N, d = _qkv("la_backward", q, k, v, dO)
+    _state("la_backward", "S0", S0, B, Hkv, d)
+    _state("la_backward", "dSf", dSf, B, Hkv, d)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dS0 = torch.empty(B, Hkv, d, d, dtype=torch.float32, device=q.device) if want_dS0 else None
     _check("la_backward", load_library().la_backward(
@@ -250,9 +302,10 @@ def la_backward(q, k, v, dO, S0=None, dSf=None, want_dS0: bool = False, chunk: i
 
 
 def la_forward_f32(q, k, v, o=None, S=None, chunk: int = 64, stream=None):
+    B, Hq, Hkv, N, d = _qkv("la_forward_f32", q, k, v, o, dtype=torch.float32)
+    _state("la_forward_f32", "S", S, B, Hkv, d)
     if o is None:
         o = torch.empty_like(q)
-    B, Hq, Hkv, N, d = _dims(q, k)
     _check("la_forward_f32", load_library().la_forward_f32(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, _stream(stream)))
     return o
@@ -260,9 +313,18 @@ def la_forward_f32(q, k, v, o=None, S=None, chunk: int = 64, stream=None):
 
 def la_decode_step(S, q, k, v, o=None, stream=None):
     """One decode step: S [B,Hkv,d,d] fp32 updated in place; returns o [B,Hq,d]."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _need("la_decode_step", name, t, torch.bfloat16)
+    if (q.dim() != 3 or k.shape != v.shape or k.dim() != 3 or k.shape[0] != q.shape[0]
+            or k.shape[2] != q.shape[2] or (o is not None and o.shape != q.shape)):
+        raise ValueError(f"la_decode_step: expected q, o [B,Hq,d] and k, v [B,Hkv,d]; got q "
+                         f"{tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    B, Hq, d = q.shape
+    _state("la_decode_step", "S", S, B, k.shape[1], d)
+    if S is None:
+        raise ValueError("la_decode_step: S is required")
     if o is None:
         o = torch.empty_like(q)
-    B, Hq, d = q.shape
     _check("la_decode_step", load_library().la_decode_step(
         _ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, k.shape[1], d, _stream(stream)))
     return o
@@ -270,9 +332,12 @@ def la_decode_step(S, q, k, v, o=None, stream=None):
 
 def la_decode_steps(S, q, k, v, o=None, stream=None):
     """Several decode steps: q [B,Hq,steps,d], k, v [B,Hkv,steps,d]; S updated in place."""
+    B, Hq, Hkv, steps, d = _qkv("la_decode_steps", q, k, v, o)
+    _state("la_decode_steps", "S", S, B, Hkv, d)
+    if S is None:
+        raise ValueError("la_decode_steps: S is required")
     if o is None:
         o = torch.empty_like(q)
-    B, Hq, steps, d = q.shape
     _check("la_decode_steps", load_library().la_decode_steps(
         _ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, k.shape[1], d, steps, _stream(stream)))
     return o
