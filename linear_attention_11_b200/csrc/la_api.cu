@@ -67,6 +67,24 @@ la_status check_shape(int B, int Hq, int Hkv, int64_t N, int d) {
 
 constexpr double kQBytesHost = 128.0 * 128 * 2;  // one 128-row bf16 tile (Q or O)
 
+}  // namespace
+
+bool keep_pool_memory() {
+  static std::once_flag once[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::call_once(once[dev], [dev]() {
+    cudaMemPool_t pool;
+    if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+      uint64_t keep = ~0ull;
+      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+  });
+  return true;
+}
+
+namespace {
+
 la_status plan_impl(int B, int Hq, int Hkv, int64_t N, int d, int chunk, int sms, la_plan* out) {
   la_status st = check_shape(B, Hq, Hkv, N, d);
   if (st != LA_OK) return st;
@@ -501,18 +519,7 @@ LA_EXPORT la_status la_forward_state(const la_bf16* q, const la_bf16* k, const l
   // Stream-ordered workspace from the device's default memory pool, kept
   // cached by the pool between calls (release threshold raised once).
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  {
-    static std::once_flag once[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LA_ERR_CUDA;
-    std::call_once(once[dev], [dev]() {
-      cudaMemPool_t pool;
-      if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
-        uint64_t keep = ~0ull;
-        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-      }
-    });
-  }
+  if (!keep_pool_memory()) return LA_ERR_CUDA;
   const size_t bytes = la_forward_workspace_bytes(B, Hq, Hkv, N, d, chunk);
   if (bytes == 0) return LA_ERR_CUDA;
   void* ws = nullptr;

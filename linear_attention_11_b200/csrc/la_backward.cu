@@ -101,6 +101,7 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
   const size_t ent_bytes = nspan_w > 1 ? round((size_t)B * Hkv * nspan_w * dd * 4) : 0;
   const size_t total = sq_bytes + wsq + wsh + ent_bytes;
   char* pool = nullptr;
+  if (!keep_pool_memory()) return LA_ERR_CUDA;
   if (cudaMallocAsync(reinterpret_cast<void**>(&pool), total, s) != cudaSuccess) return LA_ERR_CUDA;
   char* cur = pool;
   auto take = [&](size_t n) { char* p = cur; cur += n; return p; };

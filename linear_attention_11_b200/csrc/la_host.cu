@@ -90,6 +90,7 @@ LA_EXPORT la_status la_forward_host(const la_bf16* q, const la_bf16* k, const la
   const size_t set_bytes = round(qbytes) * 2 + round(kbytes) * 2;
   const size_t total = 2 * set_bytes + round(ws_bytes) + (S ? 0 : round(sbytes));
   char* pool = nullptr;
+  if (!la::keep_pool_memory()) return LA_ERR_CUDA;
   if (cudaMallocAsync(reinterpret_cast<void**>(&pool), total, s) != cudaSuccess) return LA_ERR_CUDA;
   float* carry = S;
   if (!carry) {

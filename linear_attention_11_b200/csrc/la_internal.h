@@ -30,6 +30,11 @@ struct PrefillMaps {
 
 // Device address of the status word on the current device (nullptr on failure).
 unsigned* device_status_ptr();
+// Raises the release threshold of the current device's default memory pool
+// once, so stream-ordered workspaces stay mapped between calls instead of
+// being returned at every synchronisation (la_shutdown trims the pool).
+// False if the current device cannot be queried.
+bool keep_pool_memory();
 
 // Builds a 3-D bf16 tensor map; returns false on failure.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, int64_t heads,
