@@ -1,0 +1,375 @@
+"""The synchronisation of the backward's dk/dv walk (bwd_walk_kernel in
+linear_attention_11_b200/csrc/la_backward_walk.cu), modelled on the CPU.
+
+Every role of one CTA (key-block copies, K/V copies, MMA issue, the two math
+warpgroups) is written out as the sequence of waits, arrivals, copies and
+MMAs it performs in the kernel, over the same cursor of (item, chunk, key
+block).  MMAs and commits execute in issue order in a tensor-pipe queue at
+random times; bulk copies land at random times in any order; a randomised
+scheduler interleaves the roles.  Checked for many shapes and interleavings:
+
+  - progress: some role can always move until every role has finished (a
+    deadlock here would be a kernel timeout on the GPU);
+  - parity: a wait for phase k of a barrier only starts, or stays blocked,
+    while at most k + 1 phases have completed (a parity wait cannot tell
+    phase k from phase k + 2);
+  - data: every operand an MMA reads (ring slot, K/V slot, P tile, bf16
+    state copy) holds the version it was issued for when the MMA executes,
+    and no copy, P store or state conversion overwrites a version a queued
+    MMA still needs; score tiles are read by both mask warpgroups before the
+    next scores land; the state D is reloaded or converted before the next
+    chunk's updates; dk, dv are read out before the next chunk starts them;
+  - coverage: every (group, chunk, key block) is multiplied exactly once and
+    every chunk's dk, dv are written exactly once.
+
+The model mirrors the kernel as written; a change to the kernel's
+synchronisation must be made here too.
+"""
+import random
+
+import pytest
+
+RING = 3
+CHUNK, KEYBLK = 128, 64
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count = name, count
+        self.done = 0      # completed phases
+        self.pending = 0   # arrivals in the current phase
+
+    def arrive(self):
+        self.pending += 1
+        assert self.pending <= self.count, f"{self.name}: too many arrivals"
+        if self.pending == self.count:
+            self.pending = 0
+            self.done += 1
+
+
+class Model:
+    def __init__(self, B, Hq, Hkv, N, nspan, grid, cta, seed):
+        self.G, self.Hkv, self.N, self.nspan = Hq // Hkv, Hkv, N, nspan
+        self.tiles = (N + CHUNK - 1) // CHUNK
+        self.items = B * Hkv * nspan
+        self.grid, self.cta = grid, cta
+        self.rng = random.Random(seed)
+        mk = Barrier
+        self.ring_full = [mk(f"ring_full{s}", 1) for s in range(RING)]
+        self.ring_empty = [mk(f"ring_empty{s}", 1) for s in range(RING)]
+        self.kv_full, self.kv_empty = mk("kv_full", 1), mk("kv_empty", 1)
+        self.a_full, self.s_read = mk("a_full", 1), mk("s_read", 2)
+        self.p_full, self.p_free = mk("p_full", 2), mk("p_free", 1)
+        self.o_full = mk("o_full", 1)
+        self.o_empty = [mk("o_empty0", 1), mk("o_empty1", 1)]
+        self.s_full, self.sb_full = mk("s_full", 1), mk("sb_full", 1)
+        self.waiting = {}      # role -> (barrier, phase)
+        self.tensor = []       # queued MMAs and commits, executed in order
+        self.copies = []       # (barrier, resource, version), landing in any order
+        # resource versions
+        self.ver = {("ring", s): None for s in range(RING)}
+        self.ver.update({"kv": None, "P1": None, "P2": None, "sS": 0, "S": None})
+        self.d_ready = 0              # D holds what chunk d_ready's updates need
+        self.d_done = -1              # last chunk whose every update of D has executed
+        self.scores_read = {1: -1, 2: -1}  # last block whose scores each warpgroup read
+        self.acc = {1: None, 2: None}      # chunk of the last product into dv (1), dk (2)
+        self.acc_read = {1: -1, 2: -1}     # last chunk each warpgroup wrote out
+        self.multiplied, self.written = [], []
+
+    # ----------------------------------------------------------- cursor
+    def span_of(self, it):
+        j = it % self.nspan
+        return it // self.nspan, j * self.tiles // self.nspan, (j + 1) * self.tiles // self.nspan
+
+    def halves(self, cs):
+        return 2 if self.N - cs * CHUNK > KEYBLK else 1
+
+    def blocks(self):
+        """Blocks in the order every role walks them."""
+        i = gc = 0
+        for it in range(self.cta, self.items, self.grid):
+            bg, tb, te = self.span_of(it)
+            for n in range(te - tb):
+                cs = te - 1 - n
+                nb = self.G * self.halves(cs)
+                for blk in range(nb):
+                    yield dict(it=it, bg=bg, n=n, cs=cs, blk=blk, nb=nb, gc=gc, i=i)
+                    i += 1
+                gc += 1
+
+    # ----------------------------------------------------------- primitives
+    def wait(self, role, bar, phase):
+        assert bar.done <= phase + 1, (
+            f"{role}: waits for phase {phase} of {bar.name} after {bar.done} completed")
+        self.waiting[role] = (bar, phase)
+        while bar.done <= phase:
+            yield
+        del self.waiting[role]
+
+    def mma(self, name, reads=(), run=None):
+        self.tensor.append(("mma", name, tuple(reads), run))
+
+    def commit(self, bar):
+        self.tensor.append(("commit", bar))
+
+    def queued_reads(self, res):
+        return [v for e in self.tensor if e[0] == "mma" for r, v in e[2] if r == res]
+
+    def overwrite(self, res, version, who):
+        stale = [v for v in self.queued_reads(res) if v != version]
+        assert not stale, f"{who}: overwrites {res} while queued MMAs still need {stale}"
+        self.ver[res] = version
+
+    def execute(self):
+        e = self.tensor.pop(0)
+        if e[0] == "commit":
+            e[1].arrive()
+            return
+        _, name, reads, run = e
+        for res, v in reads:
+            assert self.ver[res] == v, f"{name}: reads {res} = {self.ver[res]}, issued for {v}"
+        if run:
+            run()
+
+    # ----------------------------------------------------------- roles
+    def producer_ring(self):
+        for x in self.blocks():
+            s = x["i"] % RING
+            if x["i"] >= RING:
+                yield from self.wait("ring", self.ring_empty[s], x["i"] // RING - 1)
+            self.copies.append((self.ring_full[s], ("ring", s), x["i"]))
+            yield
+
+    def producer_kv(self):
+        gc = 0
+        for it in range(self.cta, self.items, self.grid):
+            _, tb, te = self.span_of(it)
+            for _n in range(te - tb):
+                if gc >= 1:
+                    yield from self.wait("kv", self.kv_empty, gc - 1)
+                self.copies.append((self.kv_full, "kv", gc))
+                gc += 1
+                yield
+
+    def mma_role(self):
+        seq = list(self.blocks())
+        st = {"inter_gc": -1, "kv_pending": -1, "a": 0}
+
+        def scores(i):
+            def run():
+                for wg in (1, 2):
+                    assert self.scores_read[wg] >= i - 1, (
+                        f"S({i}) lands before warpgroup {wg} read S({i - 1})")
+                self.ver["S"] = i
+            return run
+
+        def product(wg, gc, first):
+            def run():
+                if first:
+                    assert self.acc_read[wg] >= gc - 1, (
+                        f"chunk {gc} starts accumulator {wg} before chunk {gc - 1} was read out")
+                self.acc[wg] = gc
+            return run
+
+        def update(gc, last):
+            def run():
+                assert self.d_ready >= gc, f"update of chunk {gc} before D was ready for it"
+                if last:
+                    self.d_done = gc
+            return run
+
+        def issue_s(x):
+            if x["blk"] == 0:
+                yield from self.wait("mma", self.kv_full, x["gc"])
+            s = x["i"] % RING
+            yield from self.wait("mma", self.ring_full[s], x["i"] // RING)
+            self.mma(f"S({x['i']})", [(("ring", s), x["i"]), ("kv", x["gc"])], scores(x["i"]))
+            self.commit(self.a_full)
+            if x["blk"] == x["nb"] - 1:
+                if st["inter_gc"] >= x["gc"]:
+                    self.commit(self.kv_empty)
+                else:
+                    st["kv_pending"] = x["gc"]
+
+        def score_ahead(c_i, must):
+            while st["a"] < len(seq) and st["a"] <= c_i + 1:
+                x = seq[st["a"]]
+                if x["blk"] == 0 and st["inter_gc"] < x["gc"] - 1 and not (must and x["i"] == c_i):
+                    break
+                if x["i"] > 0:
+                    yield from self.wait("mma", self.s_read, x["i"] - 1)
+                yield from issue_s(x)
+                st["a"] += 1
+
+        yield from score_ahead(0, True)
+        for c in seq:
+            k, gc, s = c["i"], c["gc"], c["i"] % RING
+            if st["a"] == k:
+                yield from score_ahead(k, True)
+            first, last = c["blk"] == 0, c["blk"] == c["nb"] - 1
+            yield from self.wait("mma", self.p_full, k)
+            if first and gc >= 1:
+                yield from self.wait("mma", self.o_empty[1], gc - 1)
+            self.mma(f"dk+=P2Q({k})", [(("ring", s), k), ("P2", k)], product(2, gc, first))
+            if first:
+                yield from self.wait("mma", self.sb_full, gc)
+                self.mma(f"dk+=VD^T({gc})", [("kv", gc), ("sS", gc)], product(2, gc, False))
+                if gc >= 1:
+                    yield from self.wait("mma", self.o_empty[0], gc - 1)
+            self.mma(f"dv+=P1dO({k})", [(("ring", s), k), ("P1", k)], product(1, gc, first))
+            if first:
+                self.mma(f"dv+=KD({gc})", [("kv", gc), ("sS", gc)], product(1, gc, False))
+                st["inter_gc"] = gc
+                if st["kv_pending"] == gc:
+                    self.commit(self.kv_empty)
+                    st["kv_pending"] = -1
+            self.commit(self.p_free)
+            self.mma(f"D+=QdO({k})", [(("ring", s), k)], update(gc, last))
+            self.commit(self.ring_empty[s])
+            if last:
+                self.commit(self.o_full)
+                self.commit(self.s_full)
+            self.multiplied.append((c["bg"], c["cs"], c["blk"]))
+            yield
+            yield from score_ahead(k + 1, False)
+
+    def warpgroup(self, wg):
+        role = f"wg{wg}"
+        prev = None
+
+        def write_out(p):
+            yield from self.wait(role, self.o_full, p["gc"])
+            assert self.acc[wg] == p["gc"], f"{role}: reads chunk {p['gc']}, holds {self.acc[wg]}"
+            self.acc_read[wg] = p["gc"]
+            self.o_empty[wg - 1].arrive()
+            self.written.append((role, p["bg"], p["cs"]))
+
+        def state_ready(gc):
+            # D after chunk gc - 1 is read (converted, or the final state at
+            # an item's end); the bf16 copy (and at an item start D itself)
+            # now serve chunk gc
+            if gc > 0:
+                assert self.d_done == gc - 1, f"{role}: reads D for chunk {gc} after chunk {self.d_done}"
+            self.overwrite("sS", gc, role)
+            self.d_ready = gc
+            self.sb_full.arrive()
+
+        if wg == 1:
+            state_ready(0)
+        for c in self.blocks():
+            k = c["i"]
+            yield from self.wait(role, self.a_full, k)
+            assert self.ver["S"] == k, f"{role}: scores of block {k} replaced by {self.ver['S']}"
+            self.scores_read[wg] = k
+            self.s_read.arrive()
+            if k >= 1:
+                yield from self.wait(role, self.p_free, k - 1)
+            self.overwrite(f"P{wg}", k, role)
+            self.p_full.arrive()
+            yield
+            if c["blk"] == 0 and prev is not None:
+                if wg == 1:
+                    yield from self.wait(role, self.s_full, prev["gc"])
+                    state_ready(c["gc"])
+                yield from write_out(prev)
+            prev = c
+        if prev is not None:
+            if wg == 1:
+                yield from self.wait(role, self.s_full, prev["gc"])
+                assert self.d_done == prev["gc"], f"{role}: final state read early"
+            yield from write_out(prev)
+
+    # ----------------------------------------------------------- scheduler
+    def run(self):
+        live = {"ring": self.producer_ring(), "kv": self.producer_kv(), "mma": self.mma_role(),
+                "wg1": self.warpgroup(1), "wg2": self.warpgroup(2)}
+        idle = 0
+        while live or self.tensor or self.copies:
+            moved = False
+            choice = self.rng.random()
+            if self.tensor and choice < 0.3:
+                self.execute()
+                moved = True
+            elif self.copies and choice < 0.5:
+                bar, res, v = self.copies.pop(self.rng.randrange(len(self.copies)))
+                self.overwrite(res, v, f"copy into {res}")
+                bar.arrive()
+                moved = True
+            elif live:
+                name = self.rng.choice(list(live))
+                before = self.waiting.get(name)
+                try:
+                    next(live[name])
+                except StopIteration:
+                    del live[name]
+                    moved = True
+                else:
+                    moved = before is None or self.waiting.get(name) != before
+            for role, (bar, phase) in self.waiting.items():
+                assert bar.done <= phase + 1, (
+                    f"{role}: blocked on phase {phase} of {bar.name}, {bar.done} completed")
+            idle = 0 if moved else idle + 1
+            if idle > 5000:
+                blocked = {r: (b.name, p, b.done) for r, (b, p) in self.waiting.items()}
+                raise AssertionError(f"no progress: {blocked}, live {sorted(live)}")
+        return self
+
+
+def _walk_spans(units, tiles, sms, G):
+    """The host planner's span choice (walk_spans in la_backward_walk.cu)."""
+    r_span = (2.0 * G) / (2.0 * G + 4.0)
+    best, best_cost = 1, float("inf")
+    for ns in range(1, min(tiles, 256) + 1):
+        rounds = -(-units * ns // sms)
+        cost = rounds * -(-tiles // ns)
+        if ns > 1:
+            cost += (ns - 1) / ns * units * tiles * r_span / sms + 1.0
+        if cost < best_cost - 1e-9:
+            best, best_cost = ns, cost
+    return best
+
+
+SHAPES = [
+    # B, Hq, Hkv, N, nspan, grid
+    (1, 1, 1, 1, 1, 1),         # one token: one chunk with one key block
+    (1, 1, 1, 129, 2, 2),       # G = 1, a one-block chunk at an item start
+    (1, 1, 1, 300, 1, 1),       # G = 1, one-block chunk after two full ones
+    (1, 1, 1, 64, 1, 1),        # exactly one half chunk
+    (1, 3, 1, 385, 2, 1),       # both spans on one CTA, ragged last chunk
+    (2, 4, 2, 777, 3, 5),       # several items per CTA, G = 4
+    (1, 16, 1, 500, 2, 1),      # G = 16
+    (4, 8, 8, 200, 1, 3),       # many groups, one span each
+    (1, 8, 1, 2000, 4, 3),      # many spans of a long sequence
+    (3, 2, 1, 129, 2, 4),       # G = 2 with one-block chunks, items over CTAs
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,nspan,grid", SHAPES)
+def test_walk_protocol(B, Hq, Hkv, N, nspan, grid):
+    items = B * Hkv * nspan
+    grid = min(grid, items)
+    tiles = (N + CHUNK - 1) // CHUNK
+    assert 1 <= nspan <= tiles
+    multiplied, written = [], []
+    for cta in range(grid):
+        for seed in range(10):
+            m = Model(B, Hq, Hkv, N, nspan, grid, cta, seed=1000 * cta + seed).run()
+            if seed == 0:
+                multiplied += m.multiplied
+                written += m.written
+    G = Hq // Hkv
+    want = [(bg, cs, blk) for bg in range(B * Hkv) for cs in range(tiles)
+            for blk in range(G * (2 if N - cs * CHUNK > KEYBLK else 1))]
+    assert sorted(multiplied) == sorted(want)
+    chunks = sorted((bg, cs) for bg in range(B * Hkv) for cs in range(tiles))
+    for role in ("wg1", "wg2"):
+        assert sorted((bg, cs) for r, bg, cs in written if r == role) == chunks
+
+
+def test_planner_spans_fit_the_chunks():
+    """The span counts the host planner can pick leave every span a chunk."""
+    for units in (1, 3, 32, 200):
+        for tiles in (1, 2, 9, 256, 8192):
+            for G in (1, 4, 16):
+                ns = _walk_spans(units, tiles, 148, G)
+                assert 1 <= ns <= tiles
