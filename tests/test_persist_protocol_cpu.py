@@ -1,0 +1,394 @@
+"""The synchronisation of the prefill's persistent chunk-loop kernel
+(prefill_persist_kernel in linear_attention_11_b200/csrc/la_prefill_persist.cu),
+modelled on the CPU, for the three forward configurations the launcher
+instantiates: 64-token tiles with a dedicated output tile, 64-token tiles with
+staged states (output through the Q slot), and 128-token tiles.
+
+Each role of one CTA (Q copies, K/V copies, staged-state copies, MMA issue,
+the mask warpgroup, the output warpgroup; both warpgroups convert the state)
+is written out as its sequence of barrier waits, arrivals, copies and MMAs
+over the same items, chunk steps and head subsets as the kernel.  MMAs and
+commits execute in issue order at random times, copies land at random times,
+and a randomised scheduler interleaves the roles.  Checked: progress; that
+no parity wait can see its barrier two phases ahead; that every operand an
+MMA reads (Q slot, K/V slot, bf16 state copy, score/output buffer, P buffer)
+holds the version it was issued for when it executes and that nothing
+overwrites a version a queued MMA or a pending store still needs; that the
+state is read after its update and reloaded before the next one; and that
+every tile is written out once.  A change to the kernel's synchronisation
+must be made here too.
+"""
+import random
+
+import pytest
+
+from test_walk_protocol_cpu import Barrier
+
+
+class Model:
+    def __init__(self, T, QST, KVST, dedo, staged, G, units, nspan, tiles, grid, cta, s_out,
+                 seed):
+        self.T, self.QST, self.KVST, self.dedo, self.staged = T, QST, KVST, dedo, staged
+        self.nsub = G // (128 // T)
+        self.nspan, self.tiles, self.items = nspan, tiles, units * nspan
+        self.grid, self.cta, self.s_out = grid, cta, s_out
+        self.lookahead = KVST >= 3
+        self.rng = random.Random(seed)
+        mk = Barrier
+        self.q_full = [mk(f"q_full{s}", 1) for s in range(QST)]
+        self.q_empty = [mk(f"q_empty{s}", 1 if dedo else 2) for s in range(QST)]
+        self.kv_full = [mk(f"kv_full{s}", 1) for s in range(KVST)]
+        self.kv_empty = [mk(f"kv_empty{s}", 1) for s in range(KVST)]
+        self.a_full, self.p_full = mk("a_full", 1), mk("p_full", 1)
+        self.o_full = [mk("o_full0", 1), mk("o_full1", 1)]
+        self.o_empty = [mk("o_empty0", 1), mk("o_empty1", 1)]
+        self.s_full, self.sb_full = mk("s_full", 1), mk("sb_full", 2)
+        self.store_ready, self.ostage_free = mk("store_ready", 1), mk("ostage_free", 1)
+        self.st_full, self.st_empty, self.stage_done = (mk("st_full", 1), mk("st_empty", 1),
+                                                       mk("stage_done", 2))
+        self.waiting, self.tensor, self.copies = {}, [], []
+        self.ver = {("q", s): None for s in range(QST)}
+        self.ver.update({("kv", s): None for s in range(KVST)})
+        self.ver.update({("obuf", 0): None, ("obuf", 1): None, ("p", 0): None, ("p", 1): None,
+                         "sS": 0, "ostage": None, ("staging", 0): None, ("staging", 1): None})
+        self.stage_need = {0: None, 1: None}  # what each half of the staging tile still owes
+        self.obuf_need = {0: None, 1: None}   # scores or output a buffer still owes a reader
+        self.state_chunk = None   # the chunk step after which the state in TMEM is final
+        self.state_ready = 0      # the chunk step whose update may run next
+        self.stored = []
+
+    # ----------------------------------------------------------- schedule
+    def next_item(self, it):
+        return it + self.grid if it + self.grid < self.items else -1
+
+    def steps(self):
+        """(k, it, n, hs, i, gc, last_hs, item_end, has_next) as every role walks them."""
+        i = gc = 0
+        for k, it in enumerate(range(self.cta, self.items, self.grid)):
+            j = it % self.nspan
+            tb, te = j * self.tiles // self.nspan, (j + 1) * self.tiles // self.nspan
+            last_item = self.next_item(it) < 0
+            for n in range(te - tb):
+                for hs in range(self.nsub):
+                    last_hs = hs == self.nsub - 1
+                    item_end = last_hs and n == te - tb - 1
+                    yield dict(k=k, it=it, n=n, hs=hs, i=i, gc=gc, last_hs=last_hs,
+                               item_end=item_end, has_next=not (last_item and item_end))
+                    i += 1
+                gc += 1
+
+    # ----------------------------------------------------------- primitives
+    def wait(self, role, bar, phase):
+        assert bar.done <= phase + 1, (
+            f"{role}: waits for phase {phase} of {bar.name} after {bar.done} completed")
+        self.waiting[role] = (bar, phase)
+        while bar.done <= phase:
+            yield
+        del self.waiting[role]
+
+    def mma(self, name, reads, run=None):
+        self.tensor.append(("mma", name, tuple(reads), run))
+
+    def commit(self, bar):
+        self.tensor.append(("commit", bar))
+
+    def overwrite(self, res, version, who):
+        stale = [v for e in self.tensor if e[0] == "mma" for r, v in e[2]
+                 if r == res and v != version]
+        assert not stale, f"{who}: overwrites {res} while queued MMAs still need {stale}"
+        self.ver[res] = version
+
+    def expect(self, res, version, who):
+        assert self.ver[res] == version, f"{who}: {res} holds {self.ver[res]}, wants {version}"
+
+    def land(self, res, v):
+        if res != "staging":
+            self.overwrite(res, v, f"copy into {res}")
+            return
+        for h in (0, 1):
+            assert self.stage_need[h] is None, (
+                f"state copy {v[1]} overwrites {self.stage_need[h]} of half {h}")
+            self.ver[("staging", h)] = v
+            self.stage_need[h] = v
+
+    def execute(self):
+        e = self.tensor.pop(0)
+        if e[0] == "commit":
+            e[1].arrive()
+            return
+        _, name, reads, run = e
+        for res, v in reads:
+            self.expect(res, v, name)
+        if run:
+            run()
+
+    # ----------------------------------------------------------- copy lanes
+    def q_lane(self):
+        for x in self.steps():
+            i, s = x["i"], x["i"] % self.QST
+            if i >= self.QST:
+                yield from self.wait("q", self.q_empty[s], i // self.QST - 1)
+            self.copies.append((self.q_full[s], ("q", s), ("Q", i)))
+            yield
+
+    def kv_lane(self):
+        for x in self.steps():
+            if not x["last_hs"]:
+                continue
+            gc, s = x["gc"], x["gc"] % self.KVST
+            if gc >= self.KVST:
+                yield from self.wait("kv", self.kv_empty[s], gc // self.KVST - 1)
+            self.copies.append((self.kv_full[s], ("kv", s), gc))
+            yield
+
+    def stage_lane(self):
+        for k, _it in enumerate(range(self.cta, self.items, self.grid)):
+            if k >= 1:
+                yield from self.wait("st", self.st_empty, k - 1)
+            self.copies.append((self.st_full, "staging", ("in", k)))  # both halves
+            yield
+
+    # ----------------------------------------------------------- MMA
+    def mma_role(self):
+        seq = list(self.steps())
+        first_gc = {}
+        for x in seq:
+            first_gc.setdefault(x["gc"], x["i"])
+
+        def qk(i, gci):
+            ob = i & 1
+            yield from self.wait("mma", self.q_full[i % self.QST], i // self.QST)
+            yield from self.wait("mma", self.kv_full[gci % self.KVST], gci // self.KVST)
+            if i >= 2:
+                yield from self.wait("mma", self.o_empty[ob], (i >> 1) - 1)
+
+            def run():
+                assert self.obuf_need[ob] is None, (
+                    f"QK({i}) overwrites {self.obuf_need[ob]} before it was read")
+                self.ver[("obuf", ob)] = ("A", i)
+                self.obuf_need[ob] = ("A", i)
+            self.mma(f"QK({i})", [(("q", i % self.QST), ("Q", i)),
+                                  (("kv", gci % self.KVST), gci)], run)
+            self.commit(self.a_full)
+
+        def kv(gci):
+            def run():
+                assert self.state_ready >= gci, f"KV({gci}) before the state was ready"
+                self.state_chunk = gci
+            self.mma(f"KV({gci})", [(("kv", gci % self.KVST), gci)], run)
+            self.commit(self.s_full)
+            self.commit(self.kv_empty[gci % self.KVST])
+
+        yield from qk(0, 0)
+        for x in seq:
+            i, gc, ob = x["i"], x["gc"], x["i"] & 1
+            yield from self.wait("mma", self.p_full, i)
+            if x["hs"] == 0:
+                yield from self.wait("mma", self.sb_full, gc)
+
+            def qs_run(ob=ob, i=i):
+                assert self.obuf_need[ob] is None, f"QS({i}) overwrites unread scores"
+                self.ver[("obuf", ob)] = ("O", i)
+
+            def pv_run(ob=ob, i=i):
+                self.obuf_need[ob] = ("O", i)
+            self.mma(f"QS({i})", [(("q", i % self.QST), ("Q", i)), ("sS", gc),
+                                  (("obuf", ob), ("A", i))], qs_run)
+            self.mma(f"PV({i})", [(("p", ob), i), (("kv", gc % self.KVST), gc),
+                                  (("obuf", ob), ("O", i))], pv_run)
+            self.commit(self.o_full[ob])
+            self.commit(self.q_empty[i % self.QST])
+            qk_first = self.lookahead and not x["item_end"]
+            if not x["last_hs"]:
+                yield from qk(i + 1, gc)
+            else:
+                if qk_first:
+                    yield from qk(i + 1, gc + 1)
+                kv(gc)
+                if not qk_first and x["has_next"]:
+                    yield from qk(i + 1, gc + 1)
+            yield
+
+    # ----------------------------------------------------------- warpgroups
+    def state_in(self, role, gc):
+        """A new state version (the next chunk's bf16 copy, or an item's
+        entering state) for chunk step gc."""
+        self.overwrite("sS", gc, role)
+        self.state_ready = gc
+        self.sb_full.arrive()
+
+    def stage_swap(self, role, have_in, have_out, k, gc):
+        h = 0 if role == "mask" else 1  # each warpgroup swaps its own columns
+        if have_in:
+            self.expect(("staging", h), ("in", k), role)
+            self.stage_need[h] = None
+        if have_out:
+            assert self.state_chunk == gc - 1, f"{role}: final state of {gc - 1} read early"
+            self.ver[("staging", h)] = ("out", k - 1)
+            self.stage_need[h] = ("out", k - 1)
+        if have_in:
+            self.state_in(role, gc)
+        self.stage_done.arrive()
+
+    def state_step(self, role, x, nx):
+        gc, k = x["gc"], x["k"]
+        yield from self.wait(role, self.s_full, gc)
+        assert self.state_chunk == gc, f"{role}: state of chunk step {gc} read early"
+        if x["item_end"] and self.staged:
+            if nx >= 0:
+                yield from self.wait(role, self.st_full, k + 1)
+            self.stage_swap(role, nx >= 0, self.s_out, k + 1, gc + 1)
+        elif not x["item_end"]:
+            self.state_in(role, gc + 1)
+        elif nx >= 0:
+            self.state_in(role, gc + 1)
+
+    def first_state(self, role):
+        # both warpgroups bring in half of the CTA's first entering state
+        if self.staged:
+            yield from self.wait(role, self.st_full, 0)
+            self.stage_swap(role, True, False, 0, 0)
+        else:
+            self.state_in(role, 0)
+
+    def mask_role(self):
+        role = "mask"
+        yield from self.first_state(role)
+
+        def mask_tile(i):
+            ob = i & 1
+            yield from self.wait(role, self.a_full, i)
+            self.expect(("obuf", ob), ("A", i), f"mask({i})")
+            self.obuf_need[ob] = None
+            self.overwrite(("p", ob), i, f"mask({i})")
+            self.p_full.arrive()
+
+        yield from mask_tile(0)
+        for x in self.steps():
+            nx = self.next_item(x["it"])
+            step_first = x["last_hs"] and (not self.lookahead or x["item_end"])
+            for ph in (0, 1):
+                do_step = x["last_hs"] and ph == (0 if step_first else 1)
+                do_mask = x["has_next"] and ph == (1 if step_first else 0)
+                if do_mask:
+                    yield from mask_tile(x["i"] + 1)
+                if do_step:
+                    yield from self.state_step(role, x, nx)
+            yield
+
+    def out_role(self):
+        role = "out"
+        yield from self.first_state(role)
+        if self.staged:
+            yield from self.wait(role, self.stage_done, 0)
+            self.st_empty.arrive()
+        for x in self.steps():
+            i, ob, k = x["i"], x["i"] & 1, x["k"]
+            nx = self.next_item(x["it"])
+            if x["last_hs"]:
+                yield from self.state_step(role, x, nx)
+            if self.staged and x["item_end"]:
+                yield from self.wait(role, self.stage_done, k + 1)
+                if self.s_out:
+                    for h in (0, 1):
+                        self.expect(("staging", h), ("out", k), "final-state store")
+                        self.stage_need[h] = None
+                self.st_empty.arrive()
+            yield from self.wait(role, self.o_full[ob], i >> 1)
+            if self.dedo and i > 0:
+                yield from self.wait(role, self.ostage_free, i - 1)
+            self.expect(("obuf", ob), ("O", i), f"epilogue({i})")
+            self.obuf_need[ob] = None
+            stage = "ostage" if self.dedo else ("q", i % self.QST)
+            self.overwrite(stage, ("out", i), f"epilogue({i})")
+            self.o_empty[ob].arrive()
+            self.store_ready.arrive()
+            yield from self.wait(role, self.store_ready, i)
+            self.expect(stage, ("out", i), f"store({i})")   # the store reads the tile
+            self.stored.append((x["it"], x["n"], x["hs"]))
+            (self.ostage_free if self.dedo else self.q_empty[i % self.QST]).arrive()
+            yield
+
+    # ----------------------------------------------------------- scheduler
+    def run(self):
+        live = {"q": self.q_lane(), "kv": self.kv_lane(), "mma": self.mma_role(),
+                "mask": self.mask_role(), "out": self.out_role()}
+        if self.staged:
+            live["st"] = self.stage_lane()
+        idle = 0
+        # random speeds per run, so that some runs leave a role or a queue
+        # nearly frozen while the others race ahead
+        speed = {name: self.rng.choice((0.02, 0.3, 1.0, 1.0, 4.0)) for name in live}
+        p_tensor = self.rng.choice((0.05, 0.3, 0.6))
+        p_copy = self.rng.choice((0.05, 0.3, 0.6))
+        while live or self.tensor or self.copies:
+            moved = False
+            choice = self.rng.random()
+            if self.tensor and choice < p_tensor:
+                self.execute()
+                moved = True
+            elif self.copies and choice < p_tensor + p_copy * (1 - p_tensor):
+                bar, res, v = self.copies.pop(self.rng.randrange(len(self.copies)))
+                self.land(res, v)
+                bar.arrive()
+                moved = True
+            elif live:
+                names = list(live)
+                name = self.rng.choices(names, weights=[speed[n] for n in names])[0]
+                before = self.waiting.get(name)
+                try:
+                    next(live[name])
+                except StopIteration:
+                    del live[name]
+                    moved = True
+                else:
+                    moved = before is None or self.waiting.get(name) != before
+            for role, (bar, phase) in self.waiting.items():
+                assert bar.done <= phase + 1, (
+                    f"{role}: blocked on phase {phase} of {bar.name}, {bar.done} completed")
+            idle = 0 if moved else idle + 1
+            if idle > 20000:
+                blocked = {r: (b.name, p, b.done) for r, (b, p) in self.waiting.items()}
+                raise AssertionError(f"no progress: {blocked}, live {sorted(live)}")
+        return self
+
+
+CONFIGS = {
+    "t64_dedicated_out": dict(T=64, QST=3, KVST=2, dedo=True, staged=False),
+    "t64_staged": dict(T=64, QST=2, KVST=2, dedo=False, staged=True),
+    "t128": dict(T=128, QST=2, KVST=2, dedo=False, staged=False),
+}
+
+SHAPES = [
+    # G, units, nspan, tiles, grid, s_out
+    (2, 1, 1, 1, 1, True),
+    (2, 3, 1, 1, 2, True),      # one-tile items, several per CTA (the staged case)
+    (4, 2, 1, 4, 1, False),
+    (4, 1, 3, 7, 2, False),     # spans of unequal length
+    (8, 5, 1, 2, 3, True),
+    (2, 2, 4, 9, 3, False),
+]
+
+
+@pytest.mark.parametrize("config", sorted(CONFIGS))
+@pytest.mark.parametrize("G,units,nspan,tiles,grid,s_out", SHAPES)
+def test_persist_protocol(config, G, units, nspan, tiles, grid, s_out):
+    cfg = CONFIGS[config]
+    if cfg["staged"] and nspan != 1:
+        pytest.skip("states are staged with one span per sequence only")
+    items = units * nspan
+    grid = min(grid, items)
+    stored = []
+    for cta in range(grid):
+        for seed in range(8):
+            m = Model(G=G, units=units, nspan=nspan, tiles=tiles, grid=grid, cta=cta,
+                      s_out=s_out, seed=100 * cta + seed, **cfg).run()
+            if seed == 0:
+                stored += [(it, n, hs) for it, n, hs in m.stored]
+    nsub = G // (128 // cfg["T"])
+    want = []
+    for it in range(items):
+        j = it % nspan
+        steps = (j + 1) * tiles // nspan - j * tiles // nspan
+        want += [(it, n, hs) for n in range(steps) for hs in range(nsub)]
+    assert sorted(stored) == sorted(want)

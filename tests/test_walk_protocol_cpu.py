@@ -120,6 +120,9 @@ class Model:
         assert not stale, f"{who}: overwrites {res} while queued MMAs still need {stale}"
         self.ver[res] = version
 
+    def land(self, res, v):
+        self.overwrite(res, v, f"copy into {res}")
+
     def execute(self):
         e = self.tensor.pop(0)
         if e[0] == "commit":
@@ -284,19 +287,25 @@ class Model:
         live = {"ring": self.producer_ring(), "kv": self.producer_kv(), "mma": self.mma_role(),
                 "wg1": self.warpgroup(1), "wg2": self.warpgroup(2)}
         idle = 0
+        # random speeds per run, so that some runs leave a role or a queue
+        # nearly frozen while the others race ahead
+        speed = {name: self.rng.choice((0.02, 0.3, 1.0, 1.0, 4.0)) for name in live}
+        p_tensor = self.rng.choice((0.05, 0.3, 0.6))
+        p_copy = self.rng.choice((0.05, 0.3, 0.6))
         while live or self.tensor or self.copies:
             moved = False
             choice = self.rng.random()
-            if self.tensor and choice < 0.3:
+            if self.tensor and choice < p_tensor:
                 self.execute()
                 moved = True
-            elif self.copies and choice < 0.5:
+            elif self.copies and choice < p_tensor + p_copy * (1 - p_tensor):
                 bar, res, v = self.copies.pop(self.rng.randrange(len(self.copies)))
-                self.overwrite(res, v, f"copy into {res}")
+                self.land(res, v)
                 bar.arrive()
                 moved = True
             elif live:
-                name = self.rng.choice(list(live))
+                names = list(live)
+                name = self.rng.choices(names, weights=[speed[n] for n in names])[0]
                 before = self.waiting.get(name)
                 try:
                     next(live[name])
@@ -309,7 +318,7 @@ class Model:
                 assert bar.done <= phase + 1, (
                     f"{role}: blocked on phase {phase} of {bar.name}, {bar.done} completed")
             idle = 0 if moved else idle + 1
-            if idle > 5000:
+            if idle > 20000:
                 blocked = {r: (b.name, p, b.done) for r, (b, p) in self.waiting.items()}
                 raise AssertionError(f"no progress: {blocked}, live {sorted(live)}")
         return self
