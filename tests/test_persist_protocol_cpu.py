@@ -357,6 +357,9 @@ CONFIGS = {
     "t64_dedicated_out": dict(T=64, QST=3, KVST=2, dedo=True, staged=False),
     "t64_staged": dict(T=64, QST=2, KVST=2, dedo=False, staged=True),
     "t128": dict(T=128, QST=2, KVST=2, dedo=False, staged=False),
+    # a third K/V slot (scores of the next step before the state update):
+    # supported by the kernel, not chosen by the launcher at present
+    "t64_kv_lookahead": dict(T=64, QST=3, KVST=3, dedo=True, staged=False),
 }
 
 SHAPES = [
