@@ -16,6 +16,9 @@ v ~ N(0,1), seed 2).  Its inputs (2.7 GB) exceed L2, so no flush is needed.
   roofline   the main chunk-loop kernel: algorithmic Q+K+V+O bytes / its
              CUDA-event duration, against the measured HBM copy bandwidth
   decode     the decode step on B=256, Hq=64/Hkv=16, d=128, 64 steps: GB/s
+  workloads  the suite's other prefill workloads (mha B4 H16 N8K chunk 64, gqa
+             at chunk 128, long B1 H8 N1M chunk 128): step time, Mtok/s and
+             fraction of roofline of the step and of the chunk-loop kernel
   cpu_baseline  the fp64 CPU oracle (recurrent form) on a bounded sample
 
 Multi-GPU (torchrun): every rank runs its own copy of the workload (independent
@@ -62,6 +65,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads of the suite (mha 8K, gqa chunk 128, long 1M)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=None)
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override N (smaller case of the same workload, for profiling)")
@@ -173,27 +178,24 @@ def kernel_source_sha256():
 
 
 def traffic_from_profile():
-    """DRAM bytes per launch of the chunk-loop kernel from the committed ncu
-    summary, if the kernel source is unchanged since the capture; else None."""
-    path = os.path.join(ROOT, "profiles", "prefill_persist_traffic_gqa_b1_h128kv32.md")
+    """DRAM bytes per launch of the chunk-loop kernel on the benchmark workload
+    from the committed ncu figure (profiles/prefill_persist_traffic.json), if
+    the kernel source is unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "prefill_persist_traffic.json")
     try:
-        fields = {}
-        for line in open(path):
-            if ":" in line:
-                k, v = line.split(":", 1)
-                fields[k.strip()] = v.strip()
-        sha = kernel_source_sha256()
-        if fields.get("kernel-source-sha256") == sha:
-            return int(fields["traffic-bytes-per-launch"])
-    except (OSError, ValueError, KeyError):
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("kernel_source_sha256") == kernel_source_sha256():
+            return int(rec["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError, TypeError):
         pass
     return None
 
 
 # ------------------------------------------------------------------ CPU oracle
-def cpu_baseline(w, sample_tokens=None, target_s=10.0):
+def cpu_baseline(w, tokens=None, target_s=10.0):
     """The fp64 oracle (recurrent form), as it stands, on a sequence of n tokens
-    drawn with the workload's recipe, all heads.  Without sample_tokens, n is
+    drawn with the workload's recipe, all heads.  Without tokens, n is
     grown from a 256-token probe to about target_s seconds of work.
     Returns (tokens/s, sample description, threads used, seconds)."""
     import numpy as np
@@ -201,14 +203,7 @@ def cpu_baseline(w, sample_tokens=None, target_s=10.0):
     import oracle
     cores = oracle.threads()
     units = w.B * w.Hkv
-    if sample_tokens is None:
-        q, k, v = synth.prefill_inputs(w, N=256)
-        t0 = time.perf_counter()
-        oracle.recurrent(q, k, v, o_dtype=np.float32)
-        dt0 = time.perf_counter() - t0
-        n = int(min(w.N, max(256, 256 * target_s / max(dt0, 1e-3))))
-    else:
-        n = sample_tokens
+    n = sample_tokens(w, target_s) if tokens is None else tokens
     q, k, v = synth.prefill_inputs(w, N=n)
     t0 = time.perf_counter()
     oracle.recurrent(q, k, v, o_dtype=np.float32)
@@ -216,6 +211,51 @@ def cpu_baseline(w, sample_tokens=None, target_s=10.0):
     sample = (f"{n} of {w.N} tokens drawn with the workload recipe, B={w.B}, all {w.Hq} query "
               f"heads; {units} independent (batch, kv head) units over {min(cores, units)} threads")
     return w.B * n / dt, sample, min(cores, units), dt
+
+
+def bench_workload(la, w, chunk, steps, dev, stream, pk):
+    """One more workload of the suite on this GPU: the whole prefill step
+    (la_forward, every stage) and its chunk-loop kernel alone, each timed
+    with CUDA events, against the HBM roofline of its Q, K, V, O bytes."""
+    q, k, v = synth.prefill_inputs(w)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    del q, k, v
+    o = torch.empty_like(qd)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+
+    def step():
+        la.la_forward(qd, kd, vd, o=o, chunk=chunk, stream=stream)
+
+    for _ in range(3):
+        step()
+    t, clk = timed(step, steps, stream)
+    t /= steps
+    plan = la.api.la_prefill_plan(B, Hq, Hkv, N, d, chunk)
+    ws = torch.empty(max(1, plan.workspace_bytes // 4), dtype=torch.float32, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(max(3, min(steps, 10)))]
+    for i in range(len(ev) + 2):
+        la.api.la_prefill_span_states(kd, vd, plan, ws, stream=stream)
+        la.api.la_prefill_scan(ws, None, plan, B, Hkv, d, stream=stream)
+        if i >= 2:
+            ev[i - 2][0].record(stream)
+        la.api.la_prefill_main(qd, kd, vd, o, ws, plan, stream=stream)
+        if i >= 2:
+            ev[i - 2][1].record(stream)
+    torch.cuda.synchronize()
+    t_main = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
+    alg = 2 * (2 * B * Hq * N * d + 2 * B * Hkv * N * d)
+    flops = B * Hq * N * (4 * chunk * d + 4 * d * d)
+    t_roof = max(alg / (pk["hbm_gbs"] * 1e9), flops / (pk["bf16_tflops"] * 1e12))
+    del qd, kd, vd, o, ws
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "chunk": chunk, "steps": steps, "ms_per_step": t * 1e3,
+            "mtok_s": B * N / t / 1e6, "algorithmic_bytes": alg,
+            "step_frac_of_roofline": t_roof / t, "chunk_loop_ms": t_main * 1e3,
+            "chunk_loop_frac_of_hbm": alg / t_main / 1e9 / pk["hbm_gbs"],
+            "nspan": plan.nspan, "clocks": clk,
+            "roofline": "slower of Q+K+V+O bytes at the measured HBM peak and the chunk-form "
+                        "FLOPs N(4Cd+4d^2) per query head at the measured bf16 peak (HBM here)"}
 
 
 # ------------------------------------------------------------------ arms
@@ -226,6 +266,19 @@ def bench_config(w, chunk, world):
             "l2": "inputs larger than L2 (no flush)"}
 
 
+def sample_tokens(w, target_s):
+    """Tokens of the workload the oracle covers in about target_s seconds
+    (grown from a 256-token probe, at most the whole sequence)."""
+    import numpy as np
+
+    import oracle
+    q, k, v = synth.prefill_inputs(w, N=256)
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, o_dtype=np.float32)
+    dt0 = time.perf_counter() - t0
+    return int(min(w.N, max(256, 256 * target_s / max(dt0, 1e-3))))
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -234,7 +287,9 @@ def run_reference(args, w):
 
     import oracle
     steps, warm = args.steps, args.warmup
-    n = args.cpu_sample_tokens or 512
+    # the same sample as the in-line cpu_baseline (the whole sequence when it
+    # takes up to ~10 s), shortened only to keep the whole run near 150 s
+    n = args.cpu_sample_tokens or sample_tokens(w, min(10.0, 150.0 / max(1, steps + warm)))
     cores = min(oracle.threads(), w.B * w.Hkv)
     q, k, v = synth.prefill_inputs(w, N=n)
     per = []
@@ -494,6 +549,16 @@ def run_ours(args, w):
             "note": "bf16 operands, fp32 state in tensor memory; outputs within the bf16 "
                     "tolerance of the oracle, not bitwise equal to single steps"}
 
+    # --- the other workloads of the suite (prefill step and chunk loop each)
+    workloads = None
+    if not args.no_workloads:
+        workloads = []
+        for ow, oc in ((synth.MHA_8K, 64), (synth.GQA_32K, 128), (synth.LONG_1M, 128)):
+            if ow is w and oc == chunk:
+                continue
+            reps = max(3, min(args.steps, 10 if ow is synth.LONG_1M else 20))
+            workloads.append(bench_workload(la, ow, oc, reps, dev, stream, pk))
+
     line = {
         "metric": METRIC,
         "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
@@ -509,6 +574,7 @@ def run_ours(args, w):
         "e2e": e2e,
         "backward": backward,
         "decode": decode,
+        "workloads": workloads,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tok_s, sample, cores, dt = cpu_baseline(w, args.cpu_sample_tokens)

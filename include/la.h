@@ -179,7 +179,11 @@ la_status la_prefill_fused(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v,
  *     (batch, kv head), which runs as the single chunk-loop launch and needs
  *     no workspace, so every problem size is accepted.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     (cudaGetSymbolAddress).  With lazy module loading that lookup, like
+ *     the first launch of each kernel, loads the module holding the array
+ *     and so allocates device memory.  Make one warm-up call per device,
+ *     outside any context where allocation is forbidden and before any
+ *     stream capture; calls after it allocate nothing.
  *   - All calls share the array: calls whose work overlaps on the GPU race
  *     and must be serialised by the caller.  Each call writes every entry it
  *     reads, so nothing from an earlier call needs clearing.

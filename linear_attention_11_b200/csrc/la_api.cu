@@ -181,8 +181,8 @@ PrefillGeometry geometry(const la_plan* p, int B, int Hq, int Hkv, int64_t N) {
 
 la_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
-// Pointer checks of a bf16 prefill call: present, 16-byte aligned, o (and S)
-// disjoint from everything else.
+}  // namespace
+
 la_status check_prefill_ptrs(const void* q, const void* k, const void* v, const void* o,
                              const void* S, int B, int Hq, int Hkv, int64_t N, int d) {
   if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
@@ -197,8 +197,6 @@ la_status check_prefill_ptrs(const void* q, const void* k, const void* v, const 
     return LA_ERR_INVALID_ARG;
   return LA_OK;
 }
-
-}  // namespace
 
 unsigned* device_status_ptr() {
   unsigned* st = nullptr;
@@ -339,8 +337,7 @@ la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v,
     e = launch_state_scan(ws, S, B * Hkv, nsub_spans, kHeadDim, stream, 0,
                           final_state ? nsub_spans : nsub_spans - parts);
   if (e == cudaSuccess)
-    e = launch_prefill_persist(g, maps, ws, nullptr, status, sms, stream, true, false, 1, 0, 0,
-                               parts);
+    e = launch_prefill_persist(g, maps, ws, nullptr, status, sms, stream, true, false, parts);
   return from_cuda(e);
 }
 

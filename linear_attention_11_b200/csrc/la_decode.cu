@@ -9,13 +9,15 @@
 // causal mask).
 //
 // The step is a pure sweep over the fp32 states (2 x 4 d^2 bytes per unit,
-// about 1.2 flop/byte): HBM-bound.  One CTA of 256 threads per unit; a warp
-// reads one row of S as 32 contiguous float4 (512 B, fully coalesced), each
-// thread keeps its updated rows in registers for the G dot products, and the
-// per-row-group partial sums are reduced through shared memory.  S is read and
-// written exactly once with streaming cache hints.  The single step runs 512
-// threads per CTA (256 for groups above 16 heads); the multi-step kernel keeps
-// one state column per thread.
+// about 1.2 flop/byte): HBM-bound.  One CTA per unit, 512 threads (256 for
+// groups above 16 query heads); a warp reads one row of S as 32 contiguous
+// float4 (512 B, fully coalesced), each thread keeps its updated rows in
+// registers for the G dot products.  The sum over rows of o_h = q_h S runs
+// across warps (the lanes of a warp hold different columns, which is what
+// makes the row reads coalesced), so the per-row-group partial sums are
+// reduced through shared memory rather than by warp shuffles.  S is read and
+// written exactly once with streaming cache hints.  The multi-step kernel
+// keeps half a state column per thread and does shuffle its dot products.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

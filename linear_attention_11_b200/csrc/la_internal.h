@@ -36,6 +36,12 @@ unsigned* device_status_ptr();
 // False if the current device cannot be queried.
 bool keep_pool_memory();
 
+// Pointer checks of a bf16 prefill call: q, k, v, o present and 16-byte
+// aligned, S (nullable) aligned, o and S disjoint from each other and from
+// q, k, v.  LA_OK or LA_ERR_INVALID_ARG.
+la_status check_prefill_ptrs(const void* q, const void* k, const void* v, const void* o,
+                             const void* S, int B, int Hq, int Hkv, int64_t N, int d);
+
 // Builds a 3-D bf16 tensor map; returns false on failure.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows_per_head, int64_t heads,
                     int box_rows);
@@ -57,21 +63,15 @@ cudaError_t launch_span_states(const PrefillGeometry& g, const CUtensorMap& k,
 // span of one (batch, kv head) sequence each, every query head of the group)
 // round-robin.  ws: entering state of item bg * nspan + j (nullptr: zero);
 // s_out (nullable): final states [B*Hkv, d, d], written by the items of the
-// last spans in walk order; with nspan == 1 it may be ws itself.  ws_stride:
+// last spans; with nspan == 1 it may be ws itself.  ws_stride:
 // entering state of item it at ws[it * ws_stride] (spans cut into parts).  dependent:
 // launched as a programmatic dependent of the previous kernel in the stream.
 // stage_states (honoured at tile 64, nspan == 1, forward, s_out null or ws):
 // states pass through shared memory by bulk tensor copies, for short items
 // where they are a large share of the bytes (see stage_states_pays).
-// qdiv: query rows of head h come from head h / qdiv of the query tensor map;
-// reverse: anti-causal walk (sum over s >= t), each span from its end, tile
-// 128 only (per-head walks; la_backward takes dk and dv from the grouped walk
-// of la_backward_walk.cu instead); transpose_in (reverse only): entering
-// states read transposed (not with s_out == ws).
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
                                    cudaStream_t stream, bool dependent, bool stage_states,
-                                   int qdiv = 1, int reverse = 0, int transpose_in = 0,
                                    int ws_stride = 1);
 // Whether staging the states pays for a one-span plan: the staged layout
 // (two Q slots, output through a Q slot) streams tiles slower, so only items

@@ -5,14 +5,20 @@
 // and rejects foreign allocations, or a hard-real-time path that must not
 // block on the driver's allocator).
 //
-// The workspace that la_forward takes from the stream-ordered pool (span
-// states, or the counters of the single-span launch) lives instead in one
-// file-scope device array of fixed size.  Every GPU that
-// loads this part of the library holds the array until the process exits.
-// Every call uses the same array, so calls whose work overlaps on the GPU
-// (other streams, other host threads) race on it and must be serialised by
-// the caller.  Each call writes every workspace entry before reading it, so
-// nothing left by an earlier call needs clearing.
+// The workspace that la_forward takes from the stream-ordered pool (the span
+// states of the span-parallel scheme; a plan with one span per sequence needs
+// none) lives instead in one file-scope device array of fixed size.  Every
+// GPU that loads this part of the library holds the array until the process
+// exits.  Every call uses the same array, so calls whose work overlaps on the
+// GPU (other streams, other host threads) race on it and must be serialised
+// by the caller.  Each call writes every workspace entry before reading it,
+// so nothing left by an earlier call needs clearing.
+//
+// The first call on a device is not free of allocation: it looks up the
+// array's device address, and with lazy module loading that lookup, like the
+// first launch of each kernel, loads the module and so allocates its device
+// memory (the 32 MiB array among it).  Callers make one warm-up call outside
+// any restricted context; calls after it allocate nothing.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -47,14 +53,6 @@ void* scratch_on_current_device() {
   return g_scratch_ptr[dev];
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-bool overlap(const void* a, size_t na, const void* b, size_t nb) {
-  if (!a || !b) return false;
-  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x < y + nb && y < x + na;
-}
-
 }  // namespace
 
 LA_EXPORT la_status la_forward_noalloc(const la_bf16* q, const la_bf16* k, const la_bf16* v,
@@ -64,15 +62,7 @@ LA_EXPORT la_status la_forward_noalloc(const la_bf16* q, const la_bf16* k, const
   la_plan plan;
   la_status st = la_prefill_plan(B, Hq, Hkv, N, d, chunk, &plan);
   if (st != LA_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (S && !aligned16(S)))
-    return LA_ERR_INVALID_ARG;
-  const size_t qbytes = (size_t)B * Hq * N * d * 2, kbytes = (size_t)B * Hkv * N * d * 2,
-               sbytes = (size_t)B * Hkv * d * d * 4;
-  if (overlap(o, qbytes, q, qbytes) || overlap(o, qbytes, k, kbytes) ||
-      overlap(o, qbytes, v, kbytes) || overlap(o, qbytes, S, sbytes) ||
-      overlap(S, sbytes, q, qbytes) || overlap(S, sbytes, k, kbytes) ||
-      overlap(S, sbytes, v, kbytes))
-    return LA_ERR_INVALID_ARG;
+  if ((st = la::check_prefill_ptrs(q, k, v, o, S, B, Hq, Hkv, N, d)) != LA_OK) return st;
   // Fewer spans if the planned span states exceed the array; a single span
   // needs none (the chunk loop reads and writes the state itself).
   const int64_t per_span = (int64_t)B * Hkv * d * d * (int64_t)sizeof(float);

@@ -1,5 +1,5 @@
-// la_prefill_persist.cu -- the chunk loop of the prefill (and of the
-// backward's anti-causal walks) as a persistent tensor-core kernel.
+// la_prefill_persist.cu -- the chunk loop of the prefill as a persistent
+// tensor-core kernel.
 //
 // Per 128-row tile it computes the causal chunk form of "如何理解MiniMax股价创
 // 历史新高？拆解国产大模型技术底座", section "Lightning Attention：长上下文为什么
@@ -49,8 +49,6 @@ struct PersistParams {
   float* s_out;     // final state of sequence bg at s_out[bg], written by its last span's item
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total, items;
-  int qdiv;          // query rows of head h come from head h / qdiv of the query tensor
-  int transpose_in;  // entering states read transposed (register path, anti-causal walks)
   int ws_stride;     // spans cut into this many sub-spans in the workspace
 };
 
@@ -58,10 +56,8 @@ struct PersistParams {
 // memory by bulk tensor copies (map_s over the states, [units, 128, 128]),
 // loaded an item ahead by a third copy lane; without it the math warps read
 // and write them row by row.  kDedO: a dedicated output staging tile (else
-// the output goes through the Q slot).  kRev: anti-causal per-head passes
-// (sum over s >= t, spans walked from their end, entering states optionally
-// read transposed); la_backward now uses the grouped walk instead.
-template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kRev>
+// the output goes through the Q slot).
+template <int T, int QST, int KVST, bool kDedO, bool kStage>
 __global__ void __launch_bounds__(320, 1)
     prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
                            const __grid_constant__ CUtensorMap map_k,
@@ -118,8 +114,6 @@ __global__ void __launch_bounds__(320, 1)
     te = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
   };
   const int stride = (int)gridDim.x;
-  // n-th chunk step of the span [tb, te): forwards, or from the end in reverse
-  auto chunk_at = [&](int tb, int te, int n) { return kRev ? te - 1 - n : tb + n; };
   auto next_item = [&](int it) { return it + stride < p.items ? it + stride : -1; };
 
   const int warp = threadIdx.x >> 5;
@@ -173,7 +167,7 @@ __global__ void __launch_bounds__(320, 1)
         span_of(it, bg, tb, te);
         const int b = bg / p.Hkv, g = bg % p.Hkv;
         for (int n = 0; n < te - tb && go; ++n) {
-          const int cs = chunk_at(tb, te, n);
+          const int cs = tb + n;
           for (int hs = 0; hs < p.nsub; ++hs, ++i) {
             const int s = i % QST;
             if (i >= QST && !mbar_wait(&q_empty[s], ((i / QST) - 1) & 1, p.status, abort_flag)) {
@@ -184,7 +178,7 @@ __global__ void __launch_bounds__(320, 1)
             uint8_t* q_dst = sm + (sQ(i) - base);
 #pragma unroll
             for (int hh = 0; hh < HPT; ++hh) {
-              const int qh = (b * p.Hq + g * p.G + hs * HPT + hh) / p.qdiv;
+              const int qh = b * p.Hq + g * p.G + hs * HPT + hh;
               tma_load_3d(q_dst + hh * T * 128, &map_q, &q_full[s], 0, cs * T, qh, pol_q);
               tma_load_3d(q_dst + kHalf + hh * T * 128, &map_q, &q_full[s], 64, cs * T, qh,
                           pol_q);
@@ -208,7 +202,7 @@ __global__ void __launch_bounds__(320, 1)
         if (!staged && p.ws && nx >= 0)  // next item's entering state, read at this item's end
           prefetch_l2_bulk(p.ws + (size_t)nx * p.ws_stride * kDD, (uint32_t)(kDD * sizeof(float)));
         for (int n = 0; n < te - tb; ++n, ++gc) {
-          const int cs = chunk_at(tb, te, n);
+          const int cs = tb + n;
           const int s = gc % KVST;
           if (gc >= KVST && !mbar_wait(&kv_empty[s], ((gc / KVST) - 1) & 1, p.status, abort_flag)) {
             go = false;
@@ -289,7 +283,6 @@ __global__ void __launch_bounds__(320, 1)
         span_of(it, bg, tb, te);
         const bool last_item = next_item(it) < 0;
         for (int n = 0; n < te - tb && ok; ++n) {
-          const int cs = chunk_at(tb, te, n);
           for (int hs = 0; hs < p.nsub && ok; ++hs) {
             const uint32_t ob = (uint32_t)(i & 1);
             const uint32_t ocol = ob * 128;
@@ -343,7 +336,6 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int t_in = r % T;
     const int diag_blk = t_in / 32;
-    constexpr bool reverse = kRev;
     const int blk0 = wg1 ? 0 : 2;  // state column blocks this warpgroup handles
     const bool store_thread = (warp == 6 && lane == 0);
     bool ok = true;
@@ -354,25 +346,18 @@ __global__ void __launch_bounds__(320, 1)
       const float* st = p.ws ? p.ws + (size_t)it * p.ws_stride * kDD : nullptr;
       const float4* src =
           st ? reinterpret_cast<const float4*>(st + (size_t)r * kHeadDim) : nullptr;
-      const float* col = st ? st + r : nullptr;  // column r (transposed)
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb) {
         const int blk = blk0 + bb;
         uint32_t v[32];
-        if (kRev && p.transpose_in && col) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)  // read-only here: s_out is never ws with transpose_in
-            v[e] = __float_as_uint(__ldg(col + (size_t)(blk * 32 + e) * kHeadDim));
-        } else {
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (src) f = src[blk * 8 + m];  // plain loads: the state may be updated in place
-            v[4 * m + 0] = __float_as_uint(f.x);
-            v[4 * m + 1] = __float_as_uint(f.y);
-            v[4 * m + 2] = __float_as_uint(f.z);
-            v[4 * m + 3] = __float_as_uint(f.w);
-          }
+        for (int m = 0; m < 8; ++m) {
+          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (src) f = src[blk * 8 + m];  // plain loads: the state may be updated in place
+          v[4 * m + 0] = __float_as_uint(f.x);
+          v[4 * m + 1] = __float_as_uint(f.y);
+          v[4 * m + 2] = __float_as_uint(f.z);
+          v[4 * m + 3] = __float_as_uint(f.w);
         }
         tmem_st32(tmem + lane_base + kColS + blk * 32, v);
         store_row32_sw128(sS, r, blk, v);
@@ -419,7 +404,16 @@ __global__ void __launch_bounds__(320, 1)
       if (!warp_wait(s_full, gc & 1, p.status, abort_flag)) return false;
       tc_fence_after();
       if (item_end && staged) {
-        if (nx >= 0 && !warp_wait(st_full, (k + 1) & 1, p.status, abort_flag)) return false;
+        if (nx >= 0) {
+          // the next entering state has landed (its copy was issued only after
+          // the tile's previous final state had been read by its store)
+          if (!warp_wait(st_full, (k + 1) & 1, p.status, abort_flag)) return false;
+        } else if (p.s_out) {
+          // the CTA's last item: nothing comes in to order the reuse of the
+          // tile, so wait until the store of the previous final state (or the
+          // first hand-over) has released it before writing this one
+          if (!warp_wait(st_empty, k & 1, p.status, abort_flag)) return false;
+        }
         stage_swap(nx >= 0, p.s_out != nullptr);
         return true;
       }
@@ -436,9 +430,8 @@ __global__ void __launch_bounds__(320, 1)
         return true;
       }
       // the final state of sequence bg is complete at the end of its last span
-      // in walk order (span 0 in reverse)
       const int jspan = ((int)blockIdx.x + k * stride) % p.nspan;
-      if (p.s_out && jspan == (reverse ? 0 : p.nspan - 1)) {
+      if (p.s_out && jspan == p.nspan - 1) {
         uint32_t v0[32], v1[32];
         tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
         tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
@@ -484,7 +477,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int bb = 0; bb < 2; ++bb) {
             const int blk = 2 * h + bb;
-            need[bb] = T == 64 || (reverse ? blk >= diag_blk : blk <= diag_blk);
+            need[bb] = T == 64 || blk <= diag_blk;
             if (need[bb]) tmem_ld32(tmem + lane_base + ocol + blk * 32, a[bb]);
           }
           tmem_wait_ld();
@@ -495,8 +488,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
               const int s0 = blk * 32 + 2 * m;
-              const bool keep0 = need[bb] && (reverse ? s0 >= t_in : s0 <= t_in);
-              const bool keep1 = need[bb] && (reverse ? s0 + 1 >= t_in : s0 + 1 <= t_in);
+              const bool keep0 = need[bb] && s0 <= t_in;
+              const bool keep1 = need[bb] && s0 + 1 <= t_in;
               const float f0 = keep0 ? __uint_as_float(a[bb][2 * m]) : 0.0f;
               const float f1 = keep1 ? __uint_as_float(a[bb][2 * m + 1]) : 0.0f;
               pk[m] = pack_bf16x2(f0, f1);
@@ -516,7 +509,6 @@ __global__ void __launch_bounds__(320, 1)
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
         for (int n = 0; n < te - tb && ok; ++n) {
-          const int cs = chunk_at(tb, te, n);
           for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
             const bool last_hs = hs == p.nsub - 1;
             const bool item_end = last_hs && n == te - tb - 1;
@@ -565,7 +557,7 @@ __global__ void __launch_bounds__(320, 1)
         const int b = bg / p.Hkv, g = bg % p.Hkv;
         const int nx = next_item(it);
         for (int n = 0; n < te - tb && ok; ++n) {
-          const int cs = chunk_at(tb, te, n);
+          const int cs = tb + n;
           for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
             const bool last_hs = hs == p.nsub - 1;
             const bool item_end = last_hs && n == te - tb - 1;
@@ -637,12 +629,12 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kRev = false>
+template <int T, int QST, int KVST, bool kDedO, bool kStage>
 cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
                            const CUtensorMap& map_s, const PersistParams& p, bool dependent) {
   using L = MainLayout<T, QST, KVST, kDedO, kStage>;
   static_assert(L::kBytes <= 232448, "shared memory");
-  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage, kRev>;
+  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage>;
   cudaError_t e = set_smem(kernel, L::kBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -663,29 +655,23 @@ cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& ma
 cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& maps,
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
                                    cudaStream_t stream, bool dependent, bool stage_states,
-                                   int qdiv, int reverse, int transpose_in, int ws_stride) {
+                                   int ws_stride) {
   if (s_out && s_out == ws && g.nspan != 1) return cudaErrorInvalidValue;
   const int nsub = g.G / g.heads_per_tile;
   const int64_t items = (int64_t)g.B * g.Hkv * g.nspan;
   if (items <= 0 || items > 0x7fffffff || num_ctas <= 0) return cudaErrorInvalidValue;
-  if (qdiv < 1 || ws_stride < 1 || (transpose_in && s_out == ws && s_out))
-    return cudaErrorInvalidValue;
-  PersistParams p{ws,      s_out,         status,     g.Hq, g.Hkv,        g.G,      nsub,
-                  g.nspan, g.tiles_total, (int)items, qdiv, transpose_in, ws_stride};
+  if (ws_stride < 1) return cudaErrorInvalidValue;
+  PersistParams p{ws,      s_out,         status,     g.Hq, g.Hkv, g.G, nsub,
+                  g.nspan, g.tiles_total, (int)items, ws_stride};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
   // Staged states (room for the tile: two Q slots, output through the Q
   // slot); otherwise the smem goes to the rings.
-  if (stage_states && !reverse && !transpose_in && ws_stride == 1 && g.tile == 64 &&
+  if (stage_states && ws_stride == 1 && g.tile == 64 &&
       g.nspan == 1 && ws && (!s_out || s_out == ws)) {
     CUtensorMap map_s;
     if (!make_tmap_state(&map_s, ws, (int64_t)g.B * g.Hkv)) return cudaErrorInvalidValue;
     return launch_persist<64, 2, 2, false, true>(grid, stream, maps, map_s, p, dependent);
   }
-  if (reverse) {  // the backward's anti-causal passes: one query head per tile
-    if (g.tile != 128) return cudaErrorInvalidValue;
-    return launch_persist<128, 2, 2, false, false, true>(grid, stream, maps, maps.q, p, dependent);
-  }
-  if (transpose_in) return cudaErrorInvalidValue;
   if (g.tile == 64) return launch_persist<64, 3, 2, true, false>(grid, stream, maps, maps.q, p, dependent);
   return launch_persist<128, 2, 2, false, false>(grid, stream, maps, maps.q, p, dependent);
 }

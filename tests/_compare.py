@@ -46,3 +46,33 @@ def assert_f32_close(got, ref, what="", tol=F32_REL_L2):
     assert np.all(np.isfinite(as64(got))), f"{what}: non-finite values"
     assert rel <= tol, f"{what}: rel-L2 {rel:.3e} > {tol}"
     return rel
+
+
+class RunningBF16Check:
+    """The bf16 bounds over a tensor compared piece by piece: rel-L2 and
+    max-abs are accumulated over all pieces and checked once, so the bound
+    is the same as for the whole tensor at once."""
+
+    def __init__(self):
+        self.d2 = self.r2 = self.mx = self.scale = 0.0
+        self.finite = True
+        self.count = 0
+
+    def update(self, got, ref):
+        g, r = as64(got), as64(ref)
+        diff = g - r
+        self.finite &= bool(np.all(np.isfinite(g)))
+        self.d2 += float(np.sum(diff * diff))
+        self.r2 += float(np.sum(r * r))
+        if diff.size:
+            self.mx = max(self.mx, float(np.max(np.abs(diff))))
+            self.scale = max(self.scale, float(np.max(np.abs(r))))
+        self.count += diff.size
+
+    def check(self, what=""):
+        rel = float(np.sqrt(self.d2) / max(np.sqrt(self.r2), 1e-300))
+        assert self.finite, f"{what}: non-finite values"
+        assert rel <= BF16_REL_L2, f"{what}: rel-L2 {rel:.3e} > {BF16_REL_L2}"
+        assert self.mx <= BF16_MAX_ABS * self.scale, \
+            f"{what}: max-abs {self.mx:.3e} > {BF16_MAX_ABS} * {self.scale:.3e}"
+        return rel, self.mx

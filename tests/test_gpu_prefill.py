@@ -12,7 +12,8 @@ import torch
 import oracle
 from linear_attention_11_b200 import synth
 
-from _compare import STATE_REL_L2, assert_bf16_close, assert_f32_close, errors
+from _compare import (STATE_REL_L2, RunningBF16Check, assert_bf16_close, assert_f32_close,
+                      errors)
 
 pytestmark = pytest.mark.gpu
 
@@ -177,7 +178,7 @@ def test_argument_errors_on_device(la):
 
 
 # ------------------------------------------------------------------ full size
-def _full(la, w, chunk, rows_only=False):
+def _full(la, w, chunk):
     q, k, v = synth.prefill_inputs(w)
     qd, kd, vd = _cuda(q, k, v)
     S = torch.zeros(w.B, w.Hkv, 128, 128, dtype=torch.float32, device=DEV)
@@ -186,19 +187,8 @@ def _full(la, w, chunk, rows_only=False):
     assert la.la_device_status()[1] == 0
     oc = o.cpu()
     del o, qd, kd, vd
-    if rows_only:
-        rng = np.random.default_rng(0)
-        N = w.N
-        ts = sorted({0, 1, 127, 128, 129, N // 2, N - 129, N - 128, N - 1,
-                     *rng.integers(0, N, 40).tolist()})
-        sel = [(int(rng.integers(0, w.B)), int(rng.integers(0, w.Hq)), t) for t in ts]
-        ref = oracle.rows(q, k, v, sel)
-        got = torch.stack([oc[b, h, t] for b, h, t in sel])
-        assert_bf16_close(got, ref, f"{w.name} sampled rows")
-        ref_S = oracle.state_gemm(k, v)
-    else:
-        ref_o, ref_S = oracle.recurrent(q, k, v, o_dtype=np.float32)
-        assert_bf16_close(oc, ref_o, f"{w.name} chunk {chunk}")
+    ref_o, ref_S = oracle.recurrent(q, k, v, o_dtype=np.float32)
+    assert_bf16_close(oc, ref_o, f"{w.name} chunk {chunk}")
     assert_f32_close(S.cpu(), ref_S, f"{w.name} final state", tol=STATE_REL_L2)
 
 
@@ -211,8 +201,63 @@ def test_full_gqa_32k(la, chunk):
     _full(la, synth.GQA_32K, chunk)
 
 
+def _boundary_rows(la, w, chunk, count, seed=0):
+    """Rows t at every place a GPU schedule changes hands -- the first and
+    last tokens, both sides of chunk boundaries near the start, middle and
+    end, and both sides of every span boundary of the plan -- plus random
+    rows, at least `count` in all."""
+    N = w.N
+    plan = la.api.la_prefill_plan(w.B, w.Hq, w.Hkv, N, w.d, chunk)
+    ts = {0, 1, chunk - 1, chunk, chunk + 1, 2 * chunk - 1, 2 * chunk, N // 2 - 1, N // 2,
+          N - chunk - 1, N - chunk, N - 1}
+    for j in range(1, plan.nspan):
+        b, _ = _span_bounds(plan, j)
+        ts.update({b - 1, b})
+    rng = np.random.default_rng(seed)
+    while len(ts) < count:
+        ts.add(int(rng.integers(0, N)))
+    ts = sorted(t for t in ts if 0 <= t < N)
+    return [(int(rng.integers(0, w.B)), int(rng.integers(0, w.Hq)), t) for t in ts]
+
+
 def test_full_long_1m(la):
-    _full(la, synth.LONG_1M, 128, rows_only=True)
+    """All 8 x 2^20 output rows against the token recurrence (run in pieces of
+    2^17 tokens, each starting from the fp64 state the previous piece ended
+    with, which is the same recurrence), the final state against the
+    recurrence and K^T V, and >= 64 rows at chunk and span boundaries
+    against the masked quadratic sum."""
+    w, chunk = synth.LONG_1M, 128
+    q, k, v = synth.prefill_inputs(w)
+    qd, kd, vd = _cuda(q, k, v)
+    S = torch.zeros(w.B, w.Hkv, 128, 128, dtype=torch.float32, device=DEV)
+    o = la.la_forward_state(qd, kd, vd, S=S, chunk=chunk)
+    torch.cuda.synchronize()
+    assert la.la_device_status()[1] == 0
+    oc = o.cpu()
+    Sc = S.cpu()
+    del o, qd, kd, vd, S
+    torch.cuda.empty_cache()
+
+    piece = 1 << 17
+    run = RunningBF16Check()
+    S64 = None
+    for a in range(0, w.N, piece):
+        b = min(w.N, a + piece)
+        ref_o, S64 = oracle.recurrent(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], S0=S64,
+                                      o_dtype=np.float32)
+        run.update(oc[:, :, a:b], ref_o)
+        del ref_o
+    assert run.count == w.B * w.Hq * w.N * w.d
+    run.check(f"{w.name} chunk {chunk}, all rows vs the recurrence")
+    assert_f32_close(Sc, S64, f"{w.name} final state vs the recurrence", tol=STATE_REL_L2)
+    assert_f32_close(Sc, oracle.state_gemm(k, v), f"{w.name} final state vs K^T V",
+                     tol=STATE_REL_L2)
+
+    sel = _boundary_rows(la, w, chunk, 64)
+    assert len(sel) >= 64
+    ref = oracle.rows(q, k, v, sel)
+    got = torch.stack([oc[b, h, t] for b, h, t in sel])
+    assert_bf16_close(got, ref, f"{w.name} rows at chunk and span boundaries")
 
 
 # ------------------------------------------------------------------ fused kernel

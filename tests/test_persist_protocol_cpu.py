@@ -9,7 +9,10 @@ the mask warpgroup, the output warpgroup; both warpgroups convert the state)
 is written out as its sequence of barrier waits, arrivals, copies and MMAs
 over the same items, chunk steps and head subsets as the kernel.  MMAs and
 commits execute in issue order at random times, copies land at random times,
-and a randomised scheduler interleaves the roles.  Checked: progress; that
+and a randomised scheduler interleaves the roles.  The bulk store of a
+staged final state reads the staging tile at a random later time, and the
+tile is released only then: the other warps do not wait for that store, so
+they may reach the next hand-over first.  Checked: progress; that
 no parity wait can see its barrier two phases ahead; that every operand an
 MMA reads (Q slot, K/V slot, bf16 state copy, score/output buffer, P buffer)
 holds the version it was issued for when it executes and that nothing
@@ -47,6 +50,10 @@ class Model:
         self.st_full, self.st_empty, self.stage_done = (mk("st_full", 1), mk("st_empty", 1),
                                                        mk("stage_done", 2))
         self.waiting, self.tensor, self.copies = {}, [], []
+        # final-state stores in flight: a bulk store reads the staging tile at
+        # some later time, then warp 6 releases the tile (st_empty); the other
+        # warps of both warpgroups do not wait for it
+        self.state_stores = []
         self.ver = {("q", s): None for s in range(QST)}
         self.ver.update({("kv", s): None for s in range(KVST)})
         self.ver.update({("obuf", 0): None, ("obuf", 1): None, ("p", 0): None, ("p", 1): None,
@@ -110,6 +117,13 @@ class Model:
                 f"state copy {v[1]} overwrites {self.stage_need[h]} of half {h}")
             self.ver[("staging", h)] = v
             self.stage_need[h] = v
+
+    def store_state(self):
+        k = self.state_stores.pop(0)
+        for h in (0, 1):
+            self.expect(("staging", h), ("out", k), "final-state store")
+            self.stage_need[h] = None
+        self.st_empty.arrive()
 
     def execute(self):
         e = self.tensor.pop(0)
@@ -224,6 +238,8 @@ class Model:
             self.stage_need[h] = None
         if have_out:
             assert self.state_chunk == gc - 1, f"{role}: final state of {gc - 1} read early"
+            assert self.stage_need[h] is None, (
+                f"{role}: final state {k - 1} overwrites {self.stage_need[h]} of half {h}")
             self.ver[("staging", h)] = ("out", k - 1)
             self.stage_need[h] = ("out", k - 1)
         if have_in:
@@ -237,6 +253,10 @@ class Model:
         if x["item_end"] and self.staged:
             if nx >= 0:
                 yield from self.wait(role, self.st_full, k + 1)
+            elif self.s_out:
+                # no state comes in to order the reuse: wait until the
+                # previous final state's store has read the tile
+                yield from self.wait(role, self.st_empty, k)
             self.stage_swap(role, nx >= 0, self.s_out, k + 1, gc + 1)
         elif not x["item_end"]:
             self.state_in(role, gc + 1)
@@ -290,10 +310,9 @@ class Model:
             if self.staged and x["item_end"]:
                 yield from self.wait(role, self.stage_done, k + 1)
                 if self.s_out:
-                    for h in (0, 1):
-                        self.expect(("staging", h), ("out", k), "final-state store")
-                        self.stage_need[h] = None
-                self.st_empty.arrive()
+                    self.state_stores.append(k)
+                else:
+                    self.st_empty.arrive()
             yield from self.wait(role, self.o_full[ob], i >> 1)
             if self.dedo and i > 0:
                 yield from self.wait(role, self.ostage_free, i - 1)
@@ -321,10 +340,13 @@ class Model:
         speed = {name: self.rng.choice((0.02, 0.3, 1.0, 1.0, 4.0)) for name in live}
         p_tensor = self.rng.choice((0.05, 0.3, 0.6))
         p_copy = self.rng.choice((0.05, 0.3, 0.6))
-        while live or self.tensor or self.copies:
+        while live or self.tensor or self.copies or self.state_stores:
             moved = False
             choice = self.rng.random()
-            if self.tensor and choice < p_tensor:
+            if self.state_stores and self.rng.random() < p_copy:
+                self.store_state()
+                moved = True
+            elif self.tensor and choice < p_tensor:
                 self.execute()
                 moved = True
             elif self.copies and choice < p_tensor + p_copy * (1 - p_tensor):
@@ -366,6 +388,7 @@ SHAPES = [
     # G, units, nspan, tiles, grid, s_out
     (2, 1, 1, 1, 1, True),
     (2, 3, 1, 1, 2, True),      # one-tile items, several per CTA (the staged case)
+    (2, 9, 1, 1, 2, True),      # the same with more items per CTA
     (4, 2, 1, 4, 1, False),
     (4, 1, 3, 7, 2, False),     # spans of unequal length
     (8, 5, 1, 2, 3, True),
@@ -382,8 +405,10 @@ def test_persist_protocol(config, G, units, nspan, tiles, grid, s_out):
     items = units * nspan
     grid = min(grid, items)
     stored = []
+    # short one-span items (the staged case) get more interleavings
+    seeds = 48 if nspan == 1 and tiles <= 2 else 8
     for cta in range(grid):
-        for seed in range(8):
+        for seed in range(seeds):
             m = Model(G=G, units=units, nspan=nspan, tiles=tiles, grid=grid, cta=cta,
                       s_out=s_out, seed=100 * cta + seed, **cfg).run()
             if seed == 0:
@@ -395,3 +420,60 @@ def test_persist_protocol(config, G, units, nspan, tiles, grid, s_out):
         steps = (j + 1) * tiles // nspan - j * tiles // nspan
         want += [(it, n, hs) for n in range(steps) for hs in range(nsub)]
     assert sorted(stored) == sorted(want)
+
+
+# Planted mistakes: each removes or weakens one wait or barrier count of the
+# kernel's protocol, as a plausible slip would, and must fail the model.
+MUTANTS = {
+    "epilogue without o_full": (
+        "            yield from self.wait(role, self.o_full[ob], i >> 1)\n", ""),
+    "QK without o_empty": (
+        "            if i >= 2:\n"
+        "                yield from self.wait(\"mma\", self.o_empty[ob], (i >> 1) - 1)\n", ""),
+    "mask without a_full": ("            yield from self.wait(role, self.a_full, i)\n", ""),
+    "K/V copy without kv_empty": (
+        "            if gc >= self.KVST:\n"
+        "                yield from self.wait(\"kv\", self.kv_empty[s], gc // self.KVST - 1)\n", ""),
+    "Q copy without q_empty": (
+        "            if i >= self.QST:\n"
+        "                yield from self.wait(\"q\", self.q_empty[s], i // self.QST - 1)\n", ""),
+    "state copy without st_empty": (
+        "            if k >= 1:\n"
+        "                yield from self.wait(\"st\", self.st_empty, k - 1)\n", ""),
+    "last final state without st_empty": (
+        "                yield from self.wait(role, self.st_empty, k)\n", "                pass\n"),
+    "state step without s_full": (
+        "        yield from self.wait(role, self.s_full, gc)\n        assert self.state_chunk == gc",
+        "        assert self.state_chunk == gc"),
+    "QS without sb_full": (
+        "            if x[\"hs\"] == 0:\n"
+        "                yield from self.wait(\"mma\", self.sb_full, gc)\n", ""),
+    "q_empty released by the MMA alone": (
+        "self.q_empty = [mk(f\"q_empty{s}\", 1 if dedo else 2) for s in range(QST)]",
+        "self.q_empty = [mk(f\"q_empty{s}\", 1) for s in range(QST)]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_protocol_mistakes(name):
+    import inspect
+    import sys
+    old, new = MUTANTS[name]
+    src = inspect.getsource(sys.modules[__name__])
+    src = src[:src.index("\n# Planted mistakes")]
+    assert src.count(old) == 1, name
+    ns = {"__name__": f"mutant_{abs(hash(name))}"}
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), ns)
+    caught = False
+    for config in sorted(ns["CONFIGS"]):
+        for shape in ns["SHAPES"]:
+            try:
+                ns["test_persist_protocol"](config, *shape)
+            except AssertionError:
+                caught = True
+                break
+            except pytest.skip.Exception:
+                continue
+        if caught:
+            break
+    assert caught, f"planted mistake '{name}' passed the model"
