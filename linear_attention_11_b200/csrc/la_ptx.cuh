@@ -143,6 +143,27 @@ __device__ __forceinline__ bool warp_wait_flag(const unsigned* flag, unsigned* s
   return __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
 }
 
+// Wait until *flag == value (acquire, GPU scope), bounded like mbar_wait;
+// every lane of the warp takes the same outcome.
+__device__ __forceinline__ bool warp_wait_flag_eq(const unsigned* flag, unsigned value,
+                                                  unsigned* status, volatile int* abort) {
+  bool ok = ld_acquire_gpu(flag) == value;
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      if (ld_acquire_gpu(flag) == value) { ok = true; break; }
+      if (*abort) break;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kDevTimeout);
+        *abort = 1;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  return __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
+}
+
 // ---------------------------------------------------------------- dependent launch
 // Programmatic dependent launch: a kernel launched with the programmatic
 // stream-serialization attribute may start before the previous kernel in the
@@ -186,6 +207,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
 // aligned); no completion to wait for.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// The same prefetch with an L2 eviction-priority hint.
+__device__ __forceinline__ void prefetch_l2_bulk_hint(const void* p, uint32_t bytes,
+                                                      uint64_t policy) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(p),
+               "r"(bytes), "l"(policy)
+               : "memory");
 }
 
 // 3-D tiled store shared -> global (bulk-group completion).
