@@ -554,7 +554,7 @@ LA_EXPORT la_status la_prefill_chained(const la_bf16* q, const la_bf16* k, const
       !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
     return LA_ERR_CUDA;
   PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
-  return from_cuda(launch_prefill_chain(g, maps, k, v, S, S, workspace, status, sms,
+  return from_cuda(launch_prefill_chain(g, maps, S, S, workspace, status, sms,
                                         static_cast<cudaStream_t>(stream)));
 }
 

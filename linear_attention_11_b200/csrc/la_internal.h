@@ -81,11 +81,9 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
 // loop.  Items are dealt span index first; the launch is cooperative (items
 // wait on items of other CTAs).  workspace: chain_workspace_bytes(B, Hkv)
 // bytes, 16-byte aligned, contents irrelevant (the flags in it are cleared
-// on the stream before the launch).  s0 may equal s_out.  k, v: the tensors
-// behind maps.k, maps.v (for L2 prefetches of whole spans).
+// on the stream before the launch).  s0 may equal s_out.
 size_t chain_workspace_bytes(int B, int Hkv);
-cudaError_t launch_prefill_chain(const PrefillGeometry& g, const PrefillMaps& maps,
-                                 const la_bf16* k, const la_bf16* v, const float* s0,
+cudaError_t launch_prefill_chain(const PrefillGeometry& g, const PrefillMaps& maps, const float* s0,
                                  float* s_out, void* workspace, unsigned* status, int num_ctas,
                                  cudaStream_t stream);
 // Whether staging the states pays for a one-span plan: the staged layout

@@ -40,7 +40,6 @@
 #include "la_internal.h"
 #include "la_ptx.cuh"
 #include "la_tile.cuh"
-#include <cuda_bf16.h>
 
 namespace la {
 namespace {
@@ -59,9 +58,6 @@ struct PersistParams {
   unsigned* flags;
   const float* s0;  // initial states (nullptr: zero), read by the items of span 0
   int units;        // B * Hkv
-  const __nv_bfloat16* k_rows;  // kChain: k, v as [B * Hkv, n_rows, 128] (L2 prefetch)
-  const __nv_bfloat16* v_rows;
-  int64_t n_rows;
 };
 
 // kStage: entering and final states pass through a 64 KB fp32 tile in shared
@@ -232,19 +228,6 @@ __global__ void __launch_bounds__(320, 1)
           const uint64_t pol = pass == 0 ? pol_keep : pol_kv;
           for (int n = 0; n < te - tb; ++n, ++gc) {
             const int cs = tb + n;
-            if (kChain && pass == 1 && n == (te - tb) / 2 && nx >= 0) {
-              // halfway through this item's chunk loop: the next item's K and V
-              // into L2, so that its first pass over them does not wait on HBM
-              int nbg, ntb, nte;
-              span_of(nx, nbg, ntb, nte);
-              const int64_t r0 = (int64_t)ntb * T;
-              const int64_t r1 = std::min<int64_t>((int64_t)nte * T, p.n_rows);
-              const size_t off = ((size_t)nbg * (size_t)p.n_rows + (size_t)r0) * kHeadDim;
-              const uint32_t bytes =  // (more than L2 holds would be pointless)
-                  (uint32_t)std::min<int64_t>((r1 - r0) * kHeadDim * 2, (int64_t)8 << 20);
-              prefetch_l2_bulk_hint(p.k_rows + off, bytes, pol_keep);
-              prefetch_l2_bulk_hint(p.v_rows + off, bytes, pol_keep);
-            }
             const int s = gc % KVST;
             if (gc >= KVST &&
                 !mbar_wait(&kv_empty[s], ((gc / KVST) - 1) & 1, p.status, abort_flag)) {
@@ -931,7 +914,7 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
   if (ws_stride < 1) return cudaErrorInvalidValue;
   PersistParams p{ws,      s_out,         status,     g.Hq,    g.Hkv,   g.G,     nsub,
                   g.nspan, g.tiles_total, (int)items, ws_stride, nullptr, nullptr, nullptr,
-                  g.B * g.Hkv, nullptr, nullptr, g.N};
+                  g.B * g.Hkv};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
   // Staged states (room for the tile: two Q slots, output through the Q
   // slot); otherwise the smem goes to the rings.
@@ -950,8 +933,7 @@ size_t chain_workspace_bytes(int B, int Hkv) {
   return units * 2 * kHeadDim * kHeadDim * sizeof(float) + ((units * 2 * sizeof(unsigned) + 255) & ~(size_t)255);
 }
 
-cudaError_t launch_prefill_chain(const PrefillGeometry& g, const PrefillMaps& maps,
-                                 const la_bf16* k, const la_bf16* v, const float* s0,
+cudaError_t launch_prefill_chain(const PrefillGeometry& g, const PrefillMaps& maps, const float* s0,
                                  float* s_out, void* workspace, unsigned* status, int num_ctas,
                                  cudaStream_t stream) {
   const int64_t units = (int64_t)g.B * g.Hkv;
@@ -965,8 +947,7 @@ cudaError_t launch_prefill_chain(const PrefillGeometry& g, const PrefillMaps& ma
   if (e != cudaSuccess) return e;
   PersistParams p{nullptr, s_out,         status,     g.Hq,  g.Hkv, g.G, g.G / g.heads_per_tile,
                   g.nspan, g.tiles_total, (int)items, 1,     chain, flags, s0,
-                  (int)units, reinterpret_cast<const __nv_bfloat16*>(k),
-                  reinterpret_cast<const __nv_bfloat16*>(v), g.N};
+                  (int)units};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
   if (g.tile == 64)
     return launch_persist<64, 3, 2, true, false, true>(grid, stream, maps, maps.q, p, false);

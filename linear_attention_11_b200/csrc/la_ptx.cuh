@@ -209,14 +209,6 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// The same prefetch with an L2 eviction-priority hint.
-__device__ __forceinline__ void prefetch_l2_bulk_hint(const void* p, uint32_t bytes,
-                                                      uint64_t policy) {
-  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(p),
-               "r"(bytes), "l"(policy)
-               : "memory");
-}
-
 // 3-D tiled store shared -> global (bulk-group completion).
 __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int c0, int c1,
                                              int c2) {
