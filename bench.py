@@ -401,10 +401,6 @@ def run_ours(args, w):
     wsf = torch.empty(fb, dtype=torch.uint8, device=dev)
     t_fused = ev_mean(lambda: la.api.la_prefill_fused(qd, kd, vd, o, None, wsf, chunk=chunk,
                                                       stream=stream))
-    wsc = torch.empty(la.api.la_prefill_chained_workspace_bytes(B, Hkv), dtype=torch.uint8,
-                      device=dev)
-    t_chained = ev_mean(lambda: la.api.la_prefill_chained(qd, kd, vd, o, None, wsc, chunk=chunk,
-                                                          stream=stream))
     # the same step captured once in a CUDA graph and replayed (launch costs
     # of the host call removed): informational
     gs = torch.cuda.Stream()
@@ -421,14 +417,11 @@ def run_ours(args, w):
         "cuda_graph_replay_ms": 1e3 * t_graph,
         "sequential_chunk_loop_ms": 1e3 * t_seq,
         "single_pass_fused_ms": 1e3 * t_fused,
-        "single_pass_chained_ms": 1e3 * t_chained,
         "note": "sequential = one span per (batch, kv head): one CTA walks every chunk of "
                 "the kv group; "
-                "fused = span states and chunk loops in one persistent kernel; "
-                "chained = each chunk-loop item forms its own span's K^T V first and passes "
-                "its state to the next span's item",
+                "fused = span states and chunk loops in one persistent kernel",
     }
-    del ws1, wsf, wsc
+    del ws1, wsf
 
     # --- backward of the same workload (training): dq, dk, dv from dO
     backward = None

@@ -166,33 +166,6 @@ la_status la_prefill_fused(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v,
                            la_stream stream);
 
 /* ------------------------------------------------------------------------
- * The prefill in one pass over the sequence ("chained spans"), one
- * persistent kernel.  The arithmetic is that of la_forward_state; the
- * schedule is not on the pages (their chunk loop is sequential).  Every
- * (batch, kv head) sequence is cut into `nspan` spans of whole tiles.  The
- * item for span j first streams the span's K and V once to form its K^T V,
- * takes the state entering the span from the item of span j - 1 (S, or zero,
- * for span 0), passes the state after the span on to the item of span j + 1
- * (S receives the final state, if given), then runs the chunk loop of the
- * span, whose second read of K and V finds them in L2.  Items are dealt span
- * index first, so that at any time each sequence has a few consecutive spans
- * in flight; states pass through GPU-scope flags, and every wait is bounded.
- * The launch is cooperative: all CTAs are resident together.
- *   nspan <= 0 picks the span count for the problem and device; otherwise
- *   1 <= nspan <= ceil(N / tile) (tile = la_plan.tile).
- *   workspace: device memory, 256-byte aligned, at least
- *   la_prefill_chained_workspace_bytes(B, Hkv) bytes (two states and two
- *   flags per sequence); the call clears the flags on `stream` first
- *   (cudaMemsetAsync).  S may be read and written in place.
- * Errors as la_forward_ws.
- * ---------------------------------------------------------------------- */
-size_t la_prefill_chained_workspace_bytes(int B, int Hkv);
-la_status la_prefill_chained(const la_bf16 *q, const la_bf16 *k, const la_bf16 *v, la_bf16 *o,
-                             float *S, int B, int Hq, int Hkv, int64_t N, int d, int chunk,
-                             int nspan, void *workspace, size_t workspace_bytes,
-                             la_stream stream);
-
-/* ------------------------------------------------------------------------
  * Prefill without any device allocation.  The pages have no counterpart to
  * this entry point: it exists for callers that cannot allocate device memory
  * at call time (code inside an allocator or memory-pool callback, frameworks

@@ -25,7 +25,6 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_E
 EXPORTS = ("la_status_string", "la_version", "la_forward", "la_forward_state",
            "la_forward_workspace_bytes", "la_forward_ws", "la_forward_noalloc",
            "la_forward_host", "la_prefill_fused_workspace_bytes", "la_prefill_fused",
-           "la_prefill_chained_workspace_bytes", "la_prefill_chained",
            "la_prefill_plan", "la_backward", "la_segment_state", "la_state_prefix",
            "la_prefill_span_states", "la_prefill_scan", "la_prefill_main", "la_forward_f32",
            "la_decode_step", "la_decode_steps", "la_device_status", "la_selftest_wait",
@@ -62,8 +61,6 @@ def _declare(lib):
         "la_forward_host": ([P, P, P, P, P, I, I, I, L, I, I, L, P], I),
         "la_prefill_fused_workspace_bytes": ([I, I, I, L, I, I, I], S),
         "la_prefill_fused": ([P, P, P, P, P, I, I, I, L, I, I, I, I, P, S, P], I),
-        "la_prefill_chained_workspace_bytes": ([I, I], S),
-        "la_prefill_chained": ([P, P, P, P, P, I, I, I, L, I, I, I, P, S, P], I),
         "la_prefill_plan": ([I, I, I, L, I, I, PP], I),
         "la_prefill_span_states": ([P, P, I, I, L, I, PP, P, P], I),
         "la_prefill_scan": ([P, P, I, I, I, PP, P], I),
@@ -229,22 +226,6 @@ def la_prefill_fused(q, k, v, o, S, workspace, chunk: int = 64, nspan: int = 0,
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("la_prefill_fused", load_library().la_prefill_fused(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, nspan, lookahead,
-        _ptr(workspace), nbytes, _stream(stream)))
-    return o
-
-
-def la_prefill_chained_workspace_bytes(B, Hkv) -> int:
-    return int(load_library().la_prefill_chained_workspace_bytes(B, Hkv))
-
-
-def la_prefill_chained(q, k, v, o, S, workspace, chunk: int = 64, nspan: int = 0, stream=None):
-    """The one-pass prefill with chained spans (nspan 0 = automatic)."""
-    B, Hq, Hkv, N, d = _qkv("la_prefill_chained", q, k, v, o)
-    _state("la_prefill_chained", "S", S, B, Hkv, d)
-    _need("la_prefill_chained", "workspace", workspace)
-    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check("la_prefill_chained", load_library().la_prefill_chained(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), B, Hq, Hkv, N, d, chunk, nspan,
         _ptr(workspace), nbytes, _stream(stream)))
     return o
 

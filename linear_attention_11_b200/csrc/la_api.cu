@@ -489,75 +489,6 @@ LA_EXPORT la_status la_prefill_fused(const la_bf16* q, const la_bf16* k, const l
                                         static_cast<cudaStream_t>(stream)));
 }
 
-namespace la {
-namespace {
-
-// Span count of the chained schedule: each CTA holds one span of K and V in
-// L2 between its two passes over it, so a span's K and V times the CTAs in
-// flight should stay well inside the 126 MB L2 next to the streaming Q and
-// O (about 64 MB); among those counts, the fewest rounds x (tiles per item +
-// a per-item cost of about three tiles).
-int chain_nspan(int64_t units, int64_t tiles, int nsub, int T, int sms) {
-  const double budget = 64.0 * 1024 * 1024;
-  const double tile_kv = 2.0 * T * kHeadDim * 2;
-  int64_t best = 0;
-  double best_cost = 1e300;
-  for (int64_t ns = 1; ns <= std::min<int64_t>(tiles, 4096); ++ns) {
-    const int64_t items = units * ns;
-    if (items > 0x7fffffff) break;
-    const int64_t per_tiles = (tiles + ns - 1) / ns;
-    const double in_flight = (double)std::min<int64_t>(items, sms) * per_tiles * tile_kv;
-    if (in_flight > budget) continue;
-    const int64_t rounds = (items + sms - 1) / sms;
-    const double cost = (double)rounds * (double)(per_tiles * nsub + 3);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = ns;
-    }
-  }
-  return (int)(best > 0 ? best : std::min<int64_t>(tiles, 4096));
-}
-
-}  // namespace
-}  // namespace la
-
-LA_EXPORT size_t la_prefill_chained_workspace_bytes(int B, int Hkv) {
-  if (B <= 0 || Hkv <= 0) return 0;
-  return chain_workspace_bytes(B, Hkv);
-}
-
-LA_EXPORT la_status la_prefill_chained(const la_bf16* q, const la_bf16* k, const la_bf16* v,
-                                       la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N,
-                                       int d, int chunk, int nspan, void* workspace,
-                                       size_t workspace_bytes, la_stream stream) {
-  if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
-  la_plan plan;
-  la_status st = la_prefill_plan(B, Hq, Hkv, N, d, chunk, &plan);
-  if (st != LA_OK) return st;
-  if ((st = check_prefill_ptrs(q, k, v, o, S, B, Hq, Hkv, N, d)) != LA_OK) return st;
-  unsigned* status = nullptr;
-  int sms = 0;
-  if (!device_info(&status, &sms)) return LA_ERR_CUDA;
-  if (nspan <= 0)
-    nspan = chain_nspan((int64_t)B * Hkv, plan.tiles_total, (Hq / Hkv) / plan.heads_per_tile,
-                        plan.tile, sms);
-  if (nspan > plan.tiles_total) return LA_ERR_INVALID_ARG;
-  if ((int64_t)B * Hkv * nspan > 0x7fffffff) return LA_ERR_INVALID_ARG;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      workspace_bytes < chain_workspace_bytes(B, Hkv))
-    return LA_ERR_WORKSPACE;
-  plan.nspan = nspan;
-  PrefillMaps maps;
-  if (!make_tmap_bf16(&maps.q, q, N, (int64_t)B * Hq, plan.tile) ||
-      !make_tmap_bf16(&maps.o, o, N, (int64_t)B * Hq, plan.tile) ||
-      !make_tmap_bf16(&maps.k, k, N, (int64_t)B * Hkv, plan.tile) ||
-      !make_tmap_bf16(&maps.v, v, N, (int64_t)B * Hkv, plan.tile))
-    return LA_ERR_CUDA;
-  PrefillGeometry g = geometry(&plan, B, Hq, Hkv, N);
-  return from_cuda(launch_prefill_chain(g, maps, S, S, workspace, status, sms,
-                                        static_cast<cudaStream_t>(stream)));
-}
-
 LA_EXPORT la_status la_forward_ws(const la_bf16* q, const la_bf16* k, const la_bf16* v,
                                   la_bf16* o, float* S, int B, int Hq, int Hkv, int64_t N, int d,
                                   int chunk, void* workspace, size_t workspace_bytes,

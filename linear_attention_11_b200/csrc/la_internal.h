@@ -73,19 +73,6 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
                                    const float* ws, float* s_out, unsigned* status, int num_ctas,
                                    cudaStream_t stream, bool dependent, bool stage_states,
                                    int ws_stride = 1);
-// Chained spans (one pass over the sequence): the persistent chunk-loop
-// kernel in which item (bg, j) -- span j of (batch, kv head) bg -- first
-// forms its span's K^T V, takes the state entering the span from item
-// (bg, j - 1) (s0, nullable, for j = 0), passes the state after it on to item
-// (bg, j + 1) (s_out, nullable, gets the final state), then runs its chunk
-// loop.  Items are dealt span index first; the launch is cooperative (items
-// wait on items of other CTAs).  workspace: chain_workspace_bytes(B, Hkv)
-// bytes, 16-byte aligned, contents irrelevant (the flags in it are cleared
-// on the stream before the launch).  s0 may equal s_out.
-size_t chain_workspace_bytes(int B, int Hkv);
-cudaError_t launch_prefill_chain(const PrefillGeometry& g, const PrefillMaps& maps, const float* s0,
-                                 float* s_out, void* workspace, unsigned* status, int num_ctas,
-                                 cudaStream_t stream);
 // Whether staging the states pays for a one-span plan: the staged layout
 // (two Q slots, output through a Q slot) streams tiles slower, so only items
 // of at most four tiles use it.

@@ -50,27 +50,14 @@ struct PersistParams {
   unsigned* status;
   int Hq, Hkv, G, nsub, nspan, tiles_total, items;
   int ws_stride;     // spans cut into this many sub-spans in the workspace
-  // chained spans (kChain): the state entering span j + 1 of sequence bg,
-  // S0 + K^T V over spans 0..j, passes from item (bg, j) to item (bg, j + 1)
-  // through chain[bg][(j + 1) & 1] (d x d fp32), published by setting
-  // flags[bg][(j + 1) & 1] = j + 1 (zero at launch)
-  float* chain;
-  unsigned* flags;
-  const float* s0;  // initial states (nullptr: zero), read by the items of span 0
-  int units;        // B * Hkv
 };
 
 // kStage: entering and final states pass through a 64 KB fp32 tile in shared
 // memory by bulk tensor copies (map_s over the states, [units, 128, 128]),
 // loaded an item ahead by a third copy lane; without it the math warps read
 // and write them row by row.  kDedO: a dedicated output staging tile (else
-// the output goes through the Q slot).  kChain: chained spans, one pass over
-// the sequence (see launch_prefill_chain): every item first streams its
-// span's K and V once to form the span's K^T V in tensor memory, takes its
-// entering state from the item of the span before, publishes the state
-// after its span for the item of the span after, then runs its chunk loop,
-// which reads K and V again while they are still in L2.
-template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kChain>
+// the output goes through the Q slot).
+template <int T, int QST, int KVST, bool kDedO, bool kStage>
 __global__ void __launch_bounds__(320, 1)
     prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
                            const __grid_constant__ CUtensorMap map_k,
@@ -108,8 +95,6 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* st_full = ostage_free + 1;   // staged entering state of the CTA's k-th item landed
   uint64_t* st_empty = st_full + 1;      // staging tile free again (read, final state stored)
   uint64_t* stage_done = st_empty + 1;   // math warps done with the staging tile
-  uint64_t* span_done = stage_done + 1;  // kChain: the span's K^T V complete in tensor memory
-  uint64_t* publish_bar = span_done + 1; // kChain: every math thread stored its part of a state
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
 
@@ -122,12 +107,9 @@ __global__ void __launch_bounds__(320, 1)
   auto sO = [&](int i) { return kDedicatedO ? base + (uint32_t)L::kOOff : sQ(i); };
 
   // item it: sequence bg = it / nspan, chunk steps [tb, te) of span it % nspan
-  // (chained spans: span it / units of sequence it % units, so the items of
-  // one span index are dealt together and each follows its predecessor by
-  // `units` items)
   auto span_of = [&](int it, int& bg, int& tb, int& te) {
-    const int j = kChain ? it / p.units : it % p.nspan;
-    bg = kChain ? it % p.units : it / p.nspan;
+    const int j = it % p.nspan;
+    bg = it / p.nspan;
     tb = (int)(((int64_t)j * p.tiles_total) / p.nspan);
     te = (int)(((int64_t)(j + 1) * p.tiles_total) / p.nspan);
   };
@@ -160,8 +142,6 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(st_full, 1);
     mbar_init(st_empty, 1);
     mbar_init(stage_done, 256);
-    mbar_init(span_done, 1);
-    mbar_init(publish_bar, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -213,35 +193,28 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&map_k);
       prefetch_tmap(&map_v);
       const uint64_t pol_kv = policy_evict_first();
-      // chained spans: the first pass over a span keeps K and V in L2 for the
-      // chunk loop's pass, which is their last use
-      const uint64_t pol_keep = policy_evict_last();
       int gc = 0;
       bool go = true;
       for (int it = blockIdx.x; it < p.items && go; it += stride) {
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
-        if (!kChain && !staged && p.ws && nx >= 0)  // next item's entering state, read at this item's end
+        if (!staged && p.ws && nx >= 0)  // next item's entering state, read at this item's end
           prefetch_l2_bulk(p.ws + (size_t)nx * p.ws_stride * kDD, (uint32_t)(kDD * sizeof(float)));
-        for (int pass = kChain ? 0 : 1; pass < 2 && go; ++pass) {
-          const uint64_t pol = pass == 0 ? pol_keep : pol_kv;
-          for (int n = 0; n < te - tb; ++n, ++gc) {
-            const int cs = tb + n;
-            const int s = gc % KVST;
-            if (gc >= KVST &&
-                !mbar_wait(&kv_empty[s], ((gc / KVST) - 1) & 1, p.status, abort_flag)) {
-              go = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&kv_full[s], L::kKVBytes);
-            uint8_t* k_dst = sm + (sK(gc) - base);
-            uint8_t* v_dst = sm + (sV(gc) - base);
-            tma_load_3d(k_dst, &map_k, &kv_full[s], 0, cs * T, bg, pol);
-            tma_load_3d(k_dst + T * 128, &map_k, &kv_full[s], 64, cs * T, bg, pol);
-            tma_load_3d(v_dst, &map_v, &kv_full[s], 0, cs * T, bg, pol);
-            tma_load_3d(v_dst + T * 128, &map_v, &kv_full[s], 64, cs * T, bg, pol);
+        for (int n = 0; n < te - tb; ++n, ++gc) {
+          const int cs = tb + n;
+          const int s = gc % KVST;
+          if (gc >= KVST && !mbar_wait(&kv_empty[s], ((gc / KVST) - 1) & 1, p.status, abort_flag)) {
+            go = false;
+            break;
           }
+          mbar_arrive_expect_tx(&kv_full[s], L::kKVBytes);
+          uint8_t* k_dst = sm + (sK(gc) - base);
+          uint8_t* v_dst = sm + (sV(gc) - base);
+          tma_load_3d(k_dst, &map_k, &kv_full[s], 0, cs * T, bg, pol_kv);
+          tma_load_3d(k_dst + T * 128, &map_k, &kv_full[s], 64, cs * T, bg, pol_kv);
+          tma_load_3d(v_dst, &map_v, &kv_full[s], 0, cs * T, bg, pol_kv);
+          tma_load_3d(v_dst + T * 128, &map_v, &kv_full[s], 64, cs * T, bg, pol_kv);
         }
       }
       if (*abort_flag) {
@@ -303,72 +276,6 @@ __global__ void __launch_bounds__(320, 1)
         mma_commit(s_full);
         mma_commit(&kv_empty[gci % KVST]);
       };
-      if constexpr (kChain) {
-        // Per item: the span's K^T V (first pass over its K/V tiles) into the
-        // state columns, then the chunk loop from the entering state the math
-        // warps place there.  The chunk loop's last update is not issued: the
-        // state after the span travels along the chain instead.
-        int i = 0, kt = 0, sv = 0;
-        bool ok = true;
-        for (int it = blockIdx.x; it < p.items && ok; it += stride) {
-          int bg, tb, te;
-          span_of(it, bg, tb, te);
-          const int nt = te - tb;
-          for (int n = 0; n < nt && ok; ++n, ++kt) {
-            const int s = kt % KVST;
-            if (!mbar_wait(&kv_full[s], (kt / KVST) & 1, p.status, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t k_addr = sK(kt), v_addr = sV(kt);
-#pragma unroll
-            for (int kk = 0; kk < T / 16; ++kk) {
-              const uint64_t da = smem_desc_sw128(k_addr + kk * 2048, T * 128, 1024);
-              const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
-              mma_ss(tmem + kColS, da, db, IDESC_KV, (n > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(&kv_empty[s]);
-          }
-          if (!ok) break;
-          mma_commit(span_done);
-          if (!issue_qk(i, kt)) { ok = false; break; }
-          for (int n = 0; n < nt && ok; ++n) {
-            for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
-              const uint32_t ob = (uint32_t)(i & 1);
-              const uint32_t ocol = ob * 128;
-              const uint32_t pcol = 256 + ob * (T / 2);
-              if (!mbar_wait(p_full, i & 1, p.status, abort_flag)) { ok = false; break; }
-              if (hs == 0 && !mbar_wait(sb_full, sv & 1, p.status, abort_flag)) { ok = false; break; }
-              tc_fence_after();
-              const uint32_t q_addr = sQ(i), v_addr = sV(kt);
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {  // O = Q S
-                const uint64_t da =
-                    smem_desc_sw128(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
-                const uint64_t db = smem_desc_sw128(sS + kk * 2048, kHalf, 1024);
-                mma_ss(tmem + ocol, da, db, IDESC_QS, kk > 0 ? 1u : 0u);
-              }
-#pragma unroll
-              for (int kk = 0; kk < T / 16; ++kk) {  // O += P V
-                const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
-                mma_ts(tmem + ocol, tmem + pcol + kk * 8, db, IDESC_PV, 1u);
-              }
-              mma_commit(&o_full[ob]);
-              mma_commit(&q_empty[i % QST]);
-              if (hs < p.nsub - 1) {
-                if (!issue_qk(i + 1, kt)) ok = false;
-              } else {
-                if (n < nt - 1) {
-                  issue_kv(kt);
-                  if (!issue_qk(i + 1, kt + 1)) ok = false;
-                } else {
-                  mma_commit(&kv_empty[kt % KVST]);
-                }
-                ++kt;
-                ++sv;
-              }
-            }
-          }
-        }
-      } else {
       int i = 0, gc = 0;
       bool ok = issue_qk(0, 0);
       for (int it = blockIdx.x; it < p.items && ok; it += stride) {
@@ -417,7 +324,6 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      }  // kChain
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0);
     }
@@ -545,118 +451,10 @@ __global__ void __launch_bounds__(320, 1)
       return true;
     };
 
-    // Chained spans, at the start of item it (the CTA's k-th): this thread's
-    // half of row r of the span's K^T V is in the state columns; P, the state
-    // entering the span, arrives from the item of the span before (the
-    // caller's initial state, or zero, for span 0).  P + K^T V goes on to the
-    // item of the span after (the final state after the last span), and P
-    // replaces K^T V in tensor memory and in the bf16 copy.  16 columns at a
-    // time keep the registers of the incoming and outgoing rows apart.
-    int pubs = 0;
-    auto chain_phase = [&](int it, int k) -> bool {
-      const int j = it / p.units, bg = it % p.units;
-      if (!warp_wait(span_done, k & 1, p.status, abort_flag)) return false;
-      tc_fence_after();
-      const float* src;
-      if (j == 0) {
-        src = p.s0 ? p.s0 + (size_t)bg * kDD : nullptr;
-      } else {
-        if (!warp_wait_flag_eq(p.flags + (size_t)bg * 2 + (j & 1), (unsigned)j, p.status,
-                               abort_flag))
-          return false;
-        src = p.chain + ((size_t)bg * 2 + (j & 1)) * kDD;
-      }
-      const bool last = j == p.nspan - 1;
-      float* dst = last ? (p.s_out ? p.s_out + (size_t)bg * kDD : nullptr)
-                        : p.chain + ((size_t)bg * 2 + ((j + 1) & 1)) * kDD;
-      // this thread's 64 values of P in two halves of 32, each half's loads in
-      // flight at once (written by another CTA in this launch: read at L2, not
-      // through L1)
-      const float4* s4 =
-          src ? reinterpret_cast<const float4*>(src + (size_t)r * kHeadDim + blk0 * 32) : nullptr;
-#pragma unroll 1
-      for (int hb = 0; hb < 2; ++hb) {
-        float4 pin[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-          pin[m] = s4 ? __ldcg(s4 + 8 * hb + m) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int q = 2 * blk0 + 2 * hb + h2;
-          uint32_t kv[16], pj[16];
-          tmem_ld16(tmem + lane_base + kColS + q * 16, kv);
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const float4 f = pin[4 * h2 + m];
-            pj[4 * m + 0] = __float_as_uint(f.x);
-            pj[4 * m + 1] = __float_as_uint(f.y);
-            pj[4 * m + 2] = __float_as_uint(f.z);
-            pj[4 * m + 3] = __float_as_uint(f.w);
-          }
-          tmem_wait_ld();
-          if (dst) {
-            float4* d4 = reinterpret_cast<float4*>(dst + (size_t)r * kHeadDim + q * 16);
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-              __stcg(d4 + m,
-                     make_float4(__uint_as_float(pj[4 * m + 0]) + __uint_as_float(kv[4 * m + 0]),
-                                 __uint_as_float(pj[4 * m + 1]) + __uint_as_float(kv[4 * m + 1]),
-                                 __uint_as_float(pj[4 * m + 2]) + __uint_as_float(kv[4 * m + 2]),
-                                 __uint_as_float(pj[4 * m + 3]) + __uint_as_float(kv[4 * m + 3])));
-          }
-          tmem_st16(tmem + lane_base + kColS + q * 16, pj);
-          store_row16_sw128(sS, r, q, pj);
-        }
-      }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      // every math thread fences its part of the outgoing state and arrives
-      // before it releases the state for the MMAs, so one publication's
-      // arrivals are all in before any thread can reach the next one
-      if (!last) {
-        __threadfence();
-        mbar_arrive(publish_bar);
-      }
-      tc_fence_before();
-      mbar_arrive(sb_full);
-      if (!last) {
-        // warp 6 releases the flag for the item of the next span
-        if (warp == 6) {
-          if (!warp_wait(publish_bar, pubs & 1, p.status, abort_flag)) return false;
-          if (lane == 0) {
-            __threadfence();
-            st_release_gpu(p.flags + (size_t)bg * 2 + ((j + 1) & 1), (unsigned)(j + 1));
-          }
-          __syncwarp();
-        }
-        ++pubs;
-      }
-      return true;
-    };
-
-    // Chained spans, after the update of a chunk step inside an item (the
-    // su-th update of the CTA): the bf16 copy of the updated state.
-    auto chain_state_step = [&](int su) -> bool {
-      if (!warp_wait(s_full, su & 1, p.status, abort_flag)) return false;
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tmem + lane_base + kColS + blk0 * 32, v0);
-      tmem_ld32(tmem + lane_base + kColS + (blk0 + 1) * 32, v1);
-      tmem_wait_ld();
-      store_row32_sw128(sS, r, blk0, v0);
-      store_row32_sw128(sS, r, blk0 + 1, v1);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(sb_full);
-      return true;
-    };
-
     // The kernel may start before the kernel writing the entering states has
     // finished (programmatic dependent launch): wait before the first read.
     griddep_wait();
-    if constexpr (kChain) {
-      ok = chain_phase(blockIdx.x, 0);
-    } else if (staged) {
+    if (staged) {
       ok = warp_wait(st_full, 0, p.status, abort_flag);
       if (ok) stage_swap(true, false);
     } else {
@@ -705,27 +503,6 @@ __global__ void __launch_bounds__(320, 1)
         return true;
       };
       ok = ok && mask_tile(0);
-      if constexpr (kChain) {
-        // MMA order per tile: QS PV, then (inside an item) QK of the next tile
-        // after the state update; at an item's end the next item's span
-        // K^T V, then QK of its first tile
-        int i = 0, su = 0;
-        for (int it = blockIdx.x, k = 0; it < p.items && ok; it += stride, ++k) {
-          int bg, tb, te;
-          span_of(it, bg, tb, te);
-          const int nx = next_item(it);
-          for (int n = 0; n < te - tb && ok; ++n) {
-            for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
-              const bool last_hs = hs == p.nsub - 1;
-              const bool item_end = last_hs && n == te - tb - 1;
-              if (item_end && nx < 0) continue;
-              if (last_hs && !item_end && !chain_state_step(su++)) { ok = false; break; }
-              if (item_end && !chain_phase(nx, k + 1)) { ok = false; break; }
-              if (!mask_tile(i + 1)) { ok = false; break; }
-            }
-          }
-        }
-      } else {
       int i = 0, gc = 0;
       for (int it = blockIdx.x, k = 0; it < p.items && ok; it += stride, ++k) {
         int bg, tb, te;
@@ -751,7 +528,6 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      }  // kChain
     } else {
       // Warp 6, after the math warps are done with the staging tile (use c:
       // 0 = the first entering state, k + 1 = the end of item k): bulk-store
@@ -773,68 +549,7 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
         return true;
       };
-      // output epilogue of tile i (head subset hs of chunk step cs of kv
-      // group g of batch b): TMEM -> bf16 -> staging tile -> bulk store
-      auto epilogue = [&](int i, int b, int g, int hs, int cs) -> bool {
-        const uint32_t ob = (uint32_t)(i & 1);
-        const uint32_t ocol = ob * 128;
-        if (!warp_wait(&o_full[ob], (i >> 1) & 1, p.status, abort_flag)) return false;
-        if (kDedicatedO && i > 0 && !warp_wait(ostage_free, (i - 1) & 1, p.status, abort_flag))
-          return false;
-        tc_fence_after();
-        const uint32_t stage_o = sO(i);
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tmem + lane_base + ocol + (2 * bb) * 32, v0);
-          tmem_ld32(tmem + lane_base + ocol + (2 * bb + 1) * 32, v1);
-          tmem_wait_ld();
-          store_row32_sw128(stage_o, r, 2 * bb, v0);
-          store_row32_sw128(stage_o, r, 2 * bb + 1, v1);
-        }
-        tc_fence_before();
-        mbar_arrive(&o_empty[ob]);
-        fence_proxy_async_smem();
-        mbar_arrive(store_ready);
-        if (warp == 6 && !warp_wait(store_ready, i & 1, p.status, abort_flag)) return false;
-        if (store_thread) {
-          const uint8_t* src = sm + (stage_o - base);
-#pragma unroll
-          for (int hh = 0; hh < HPT; ++hh) {
-            const int oh = b * p.Hq + g * p.G + hs * HPT + hh;
-            tma_store_3d(&map_o, src + hh * T * 128, 0, cs * T, oh);
-            tma_store_3d(&map_o, src + kHalf + hh * T * 128, 64, cs * T, oh);
-          }
-          bulk_commit_group();
-          bulk_wait_group_read<0>();  // the store has read the staging tile
-          if (kDedicatedO)
-            mbar_arrive(ostage_free);
-          else
-            mbar_arrive(&q_empty[i % QST]);
-        }
-        return true;
-      };
       if (staged && ok && warp == 6) ok = stage_release(0, 0, false);
-      if constexpr (kChain) {
-        // the output of an item's last tile goes out before the next item's
-        // hand-over, which may wait for another CTA
-        int i = 0, su = 0;
-        for (int it = blockIdx.x, k = 0; it < p.items && ok; it += stride, ++k) {
-          int bg, tb, te;
-          span_of(it, bg, tb, te);
-          const int b = bg / p.Hkv, g = bg % p.Hkv;
-          const int nx = next_item(it);
-          for (int n = 0; n < te - tb && ok; ++n) {
-            for (int hs = 0; hs < p.nsub && ok; ++hs, ++i) {
-              const bool last_hs = hs == p.nsub - 1;
-              const bool item_end = last_hs && n == te - tb - 1;
-              if (last_hs && !item_end && !chain_state_step(su++)) { ok = false; break; }
-              if (!epilogue(i, b, g, hs, tb + n)) { ok = false; break; }
-              if (item_end && nx >= 0 && !chain_phase(nx, k + 1)) { ok = false; break; }
-            }
-          }
-        }
-      } else {
       int i = 0, gc = 0;
       for (int it = blockIdx.x, k = 0; it < p.items && ok; it += stride, ++k) {
         int bg, tb, te;
@@ -852,11 +567,51 @@ __global__ void __launch_bounds__(320, 1)
               break;
             }
             if (last_hs) ++gc;
-            if (!epilogue(i, b, g, hs, cs)) { ok = false; break; }
+            // output epilogue: TMEM -> bf16 -> staging tile -> bulk store
+            const uint32_t ob = (uint32_t)(i & 1);
+            const uint32_t ocol = ob * 128;
+            if (!warp_wait(&o_full[ob], (i >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+            if (kDedicatedO && i > 0 &&
+                !warp_wait(ostage_free, (i - 1) & 1, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t stage_o = sO(i);
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+              uint32_t v0[32], v1[32];
+              tmem_ld32(tmem + lane_base + ocol + (2 * bb) * 32, v0);
+              tmem_ld32(tmem + lane_base + ocol + (2 * bb + 1) * 32, v1);
+              tmem_wait_ld();
+              store_row32_sw128(stage_o, r, 2 * bb, v0);
+              store_row32_sw128(stage_o, r, 2 * bb + 1, v1);
+            }
+            tc_fence_before();
+            mbar_arrive(&o_empty[ob]);
+            fence_proxy_async_smem();
+            mbar_arrive(store_ready);
+            if (warp == 6) {
+              if (!warp_wait(store_ready, i & 1, p.status, abort_flag)) { ok = false; break; }
+            }
+            if (store_thread) {
+              const uint8_t* src = sm + (stage_o - base);
+#pragma unroll
+              for (int hh = 0; hh < HPT; ++hh) {
+                const int oh = b * p.Hq + g * p.G + hs * HPT + hh;
+                tma_store_3d(&map_o, src + hh * T * 128, 0, cs * T, oh);
+                tma_store_3d(&map_o, src + kHalf + hh * T * 128, 64, cs * T, oh);
+              }
+              bulk_commit_group();
+              bulk_wait_group_read<0>();  // the store has read the staging tile
+              if (kDedicatedO)
+                mbar_arrive(ostage_free);
+              else
+                mbar_arrive(&q_empty[i % QST]);
+            }
           }
         }
       }
-      }  // kChain
       if (store_thread) bulk_wait_group<0>();
     }
   }
@@ -874,12 +629,12 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kChain = false>
+template <int T, int QST, int KVST, bool kDedO, bool kStage>
 cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
                            const CUtensorMap& map_s, const PersistParams& p, bool dependent) {
   using L = MainLayout<T, QST, KVST, kDedO, kStage>;
   static_assert(L::kBytes <= 232448, "shared memory");
-  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage, kChain>;
+  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage>;
   cudaError_t e = set_smem(kernel, L::kBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -888,16 +643,10 @@ cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& ma
   cfg.dynamicSmemBytes = L::kBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  if (kChain) {
-    // items wait for items of other CTAs: all CTAs must be resident at once
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-  } else {
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-  }
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = (kChain || dependent) ? 1 : 0;
+  cfg.numAttrs = dependent ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, maps.q, maps.k, maps.v, maps.o, map_s, p);
 }
 
@@ -912,9 +661,8 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
   const int64_t items = (int64_t)g.B * g.Hkv * g.nspan;
   if (items <= 0 || items > 0x7fffffff || num_ctas <= 0) return cudaErrorInvalidValue;
   if (ws_stride < 1) return cudaErrorInvalidValue;
-  PersistParams p{ws,      s_out,         status,     g.Hq,    g.Hkv,   g.G,     nsub,
-                  g.nspan, g.tiles_total, (int)items, ws_stride, nullptr, nullptr, nullptr,
-                  g.B * g.Hkv};
+  PersistParams p{ws,      s_out,         status,     g.Hq, g.Hkv, g.G, nsub,
+                  g.nspan, g.tiles_total, (int)items, ws_stride};
   const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
   // Staged states (room for the tile: two Q slots, output through the Q
   // slot); otherwise the smem goes to the rings.
@@ -926,32 +674,6 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
   }
   if (g.tile == 64) return launch_persist<64, 3, 2, true, false>(grid, stream, maps, maps.q, p, dependent);
   return launch_persist<128, 2, 2, false, false>(grid, stream, maps, maps.q, p, dependent);
-}
-
-size_t chain_workspace_bytes(int B, int Hkv) {
-  const size_t units = (size_t)B * Hkv;
-  return units * 2 * kHeadDim * kHeadDim * sizeof(float) + ((units * 2 * sizeof(unsigned) + 255) & ~(size_t)255);
-}
-
-cudaError_t launch_prefill_chain(const PrefillGeometry& g, const PrefillMaps& maps, const float* s0,
-                                 float* s_out, void* workspace, unsigned* status, int num_ctas,
-                                 cudaStream_t stream) {
-  const int64_t units = (int64_t)g.B * g.Hkv;
-  const int64_t items = units * g.nspan;
-  if (items <= 0 || items > 0x7fffffff || num_ctas <= 0 || !workspace) return cudaErrorInvalidValue;
-  if (g.nspan < 1 || g.nspan > g.tiles_total) return cudaErrorInvalidValue;
-  float* chain = static_cast<float*>(workspace);
-  unsigned* flags =
-      reinterpret_cast<unsigned*>(chain + (size_t)units * 2 * kHeadDim * kHeadDim);
-  cudaError_t e = cudaMemsetAsync(flags, 0, (size_t)units * 2 * sizeof(unsigned), stream);
-  if (e != cudaSuccess) return e;
-  PersistParams p{nullptr, s_out,         status,     g.Hq,  g.Hkv, g.G, g.G / g.heads_per_tile,
-                  g.nspan, g.tiles_total, (int)items, 1,     chain, flags, s0,
-                  (int)units};
-  const dim3 grid((unsigned)std::min<int64_t>(items, num_ctas));
-  if (g.tile == 64)
-    return launch_persist<64, 3, 2, true, false, true>(grid, stream, maps, maps.q, p, false);
-  return launch_persist<128, 2, 2, false, false, true>(grid, stream, maps, maps.q, p, false);
 }
 
 }  // namespace la

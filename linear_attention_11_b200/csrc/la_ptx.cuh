@@ -143,27 +143,6 @@ __device__ __forceinline__ bool warp_wait_flag(const unsigned* flag, unsigned* s
   return __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
 }
 
-// Wait until *flag == value (acquire, GPU scope), bounded like mbar_wait;
-// every lane of the warp takes the same outcome.
-__device__ __forceinline__ bool warp_wait_flag_eq(const unsigned* flag, unsigned value,
-                                                  unsigned* status, volatile int* abort) {
-  bool ok = ld_acquire_gpu(flag) == value;
-  if (!ok) {
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-      if (ld_acquire_gpu(flag) == value) { ok = true; break; }
-      if (*abort) break;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(status, kDevTimeout);
-        *abort = 1;
-        break;
-      }
-      __nanosleep(64);
-    }
-  }
-  return __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
-}
-
 // ---------------------------------------------------------------- dependent launch
 // Programmatic dependent launch: a kernel launched with the programmatic
 // stream-serialization attribute may start before the previous kernel in the

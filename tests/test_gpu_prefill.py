@@ -301,73 +301,6 @@ def test_fused_rejects_bad_span_count(la):
     assert e.value.code == 5
 
 
-# ------------------------------------------------------------------ chained spans
-@pytest.mark.parametrize("Hq,Hkv,chunk", [(4, 2, 64), (2, 2, 64), (4, 1, 128), (6, 3, 64),
-                                          (8, 1, 64), (3, 3, 128)])
-@pytest.mark.parametrize("nspan", [1, 2, 3, 7, 0, -1])
-def test_chained_span_counts(la, Hq, Hkv, chunk, nspan):
-    """The one-pass prefill with chained spans for span counts 1, 2, 3, 7,
-    automatic (0) and one span per tile (-1), with an initial state read and
-    the final state written in place; two calls on one workspace."""
-    B, N = 2, 1100
-    q, k, v = _qkv(B, Hq, Hkv, N, seed=500 + Hq * 10 + Hkv + chunk)
-    S0 = torch.randn(B, Hkv, 128, 128, generator=torch.Generator().manual_seed(8)) / 128
-    ref_o, ref_S = oracle.recurrent(q, k, v, S0=S0.double().numpy())
-    qd, kd, vd = _cuda(q, k, v)
-    if nspan == -1:
-        nspan = la.api.la_prefill_plan(B, Hq, Hkv, N, 128, chunk).tiles_total
-    ws = torch.empty(la.api.la_prefill_chained_workspace_bytes(B, Hkv), dtype=torch.uint8,
-                     device=DEV)
-    for call in range(2):
-        S = S0.to(DEV)
-        o = torch.full_like(qd, float("nan"))
-        la.api.la_prefill_chained(qd, kd, vd, o, S, ws, chunk=chunk, nspan=nspan)
-        torch.cuda.synchronize()
-        assert_bf16_close(o.cpu(), ref_o, f"O nspan={nspan} call {call}")
-        assert_f32_close(S.cpu(), ref_S, f"final state nspan={nspan} call {call}",
-                         tol=STATE_REL_L2)
-    assert la.la_device_status()[1] == 0
-
-
-@pytest.mark.parametrize("B,Hq,Hkv,N,chunk,nspan", [(1, 4, 1, 1, 64, 1), (3, 8, 2, 65, 64, 0),
-                                                     (1, 2, 1, 300, 128, 3),
-                                                     (200, 4, 2, 64, 64, 1),
-                                                     (40, 8, 4, 777, 64, 0)])
-def test_chained_ragged_and_many_sequences(la, B, Hq, Hkv, N, chunk, nspan):
-    """Ragged last tiles, a one-token sequence, more sequences than CTAs (the
-    items of a span index then cover several rounds), without an initial
-    state and without a final state."""
-    q, k, v = _qkv(B, Hq, Hkv, N, seed=600 + N + B)
-    ref_o, ref_S = oracle.recurrent(q, k, v)
-    qd, kd, vd = _cuda(q, k, v)
-    ws = torch.empty(la.api.la_prefill_chained_workspace_bytes(B, Hkv), dtype=torch.uint8,
-                     device=DEV)
-    o = la.api.la_prefill_chained(qd, kd, vd, torch.empty_like(qd), None, ws, chunk=chunk,
-                                  nspan=nspan)
-    S = torch.zeros(B, Hkv, 128, 128, device=DEV)
-    o2 = la.api.la_prefill_chained(qd, kd, vd, torch.empty_like(qd), S, ws, chunk=chunk,
-                                   nspan=nspan)
-    torch.cuda.synchronize()
-    assert_bf16_close(o.cpu(), ref_o, "O without a state")
-    assert torch.equal(o, o2)
-    assert_f32_close(S.cpu(), ref_S, "final state", tol=STATE_REL_L2)
-    assert la.la_device_status()[1] == 0
-
-
-def test_chained_rejects_bad_arguments(la):
-    q, k, v = _cuda(*_qkv(1, 2, 2, 256, seed=9))
-    tiles = la.api.la_prefill_plan(1, 2, 2, 256, 128, 64).tiles_total
-    ws = torch.empty(la.api.la_prefill_chained_workspace_bytes(1, 2), dtype=torch.uint8,
-                     device=DEV)
-    with pytest.raises(la.LAError) as e:
-        la.api.la_prefill_chained(q, k, v, torch.empty_like(q), None, ws, chunk=64,
-                                  nspan=tiles + 1)
-    assert e.value.code == 1
-    with pytest.raises(la.LAError) as e:
-        la.api.la_prefill_chained(q, k, v, torch.empty_like(q), None, ws[:64], chunk=64, nspan=1)
-    assert e.value.code == 5
-
-
 # ------------------------------------------------------------------ host buffers
 @pytest.mark.parametrize("N,piece,with_state", [(1000, 0, False), (1000, 128, True), (777, 300, True),
                                                 (64, 0, False)])
