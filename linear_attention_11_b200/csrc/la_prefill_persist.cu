@@ -7,8 +7,8 @@
 // grouped kv heads as in "MiniMax-01与Lightning Attention", section 1.1.
 // Tile: 128 rows = HPT query heads x T tokens (T = 64, HPT = 2, or T = 128,
 // HPT = 1), d = 128:
-//   A  = Q_c K_c^T      tcgen05 M=128 N=T  K=128 (SS) -> TMEM
-//   P  = bf16(tril(A))  TMEM -> registers -> TMEM (diagonal kept)
+//   A  = Q_c K_c^T      tcgen05 M=128 N=T  K=128 (SS) -> TMEM score buffer
+//   P  = bf16(tril(A))  TMEM -> registers -> TMEM, over its own scores
 //   O  = Q_c bf16(S)    tcgen05 M=128 N=128 K=128 (SS)
 //   O += P V_c          tcgen05 M=128 N=128 K=T (A from TMEM)
 //   S += K_c^T V_c      tcgen05 M=128 N=128 K=T (SS, both MN-major)
@@ -31,7 +31,11 @@
 // the L2 prefetch), lane 2 staged states; warp 1 owns the tensor memory and
 // issues the MMAs; warps 2-5 mask score tiles, warps 6-9 store output tiles;
 // both warpgroups handle half of the state columns.  TMEM: O buffers at
-// columns 0 and 128 (score tiles first), P at 256, state at 384.
+// columns 0 and 128, score buffers from 256 (two of 64 columns at T = 64, one
+// of 128 at T = 128; each tile's P is written over the first half of its
+// scores), state at 384.  With the scores apart from the output, Q S of a
+// tile is issued before its mask is done, and at T = 64 the next tile's
+// scores go ahead of P V, so the tensor pipe does not wait for the mask.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -71,7 +75,7 @@ __global__ void __launch_bounds__(320, 1)
   constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, 0, 1);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
   constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, 1, 1);
-  constexpr bool kLookahead = KVST >= 3;
+  constexpr int NSC = T == 64 ? 2 : 1;  // score buffers
   constexpr int kDD = kHeadDim * kHeadDim;
 
   extern __shared__ uint8_t smem_raw[];
@@ -83,9 +87,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* q_empty = q_full + QST;
   uint64_t* kv_full = q_empty + QST;
   uint64_t* kv_empty = kv_full + KVST;
-  uint64_t* a_full = kv_empty + KVST;
-  uint64_t* p_full = a_full + 1;
-  uint64_t* o_full = p_full + 1;    // two: tile i completes o_full[i & 1]
+  uint64_t* a_full = kv_empty + KVST;  // two: tile i's scores complete a_full[i % NSC]
+  uint64_t* p_full = a_full + 2;       // two: tile i's P complete p_full[i % NSC]
+  uint64_t* o_full = p_full + 2;    // two: tile i completes o_full[i & 1]
   uint64_t* o_empty = o_full + 2;   // two
   uint64_t* s_full = o_empty + 2;   // one completion per chunk step (state update)
   uint64_t* sb_full = s_full + 1;   // one completion per state version (bf16 copy ready)
@@ -105,6 +109,8 @@ __global__ void __launch_bounds__(320, 1)
   auto sK = [&](int c) { return base + (uint32_t)(L::kKVOff + (c % KVST) * L::kKVBytes); };
   auto sV = [&](int c) { return sK(c) + (uint32_t)L::kKBytes; };
   auto sO = [&](int i) { return kDedicatedO ? base + (uint32_t)L::kOOff : sQ(i); };
+  // TMEM column of tile i's score buffer (its P over the first T / 2 columns)
+  auto scol = [&](int i) { return (uint32_t)(256 + (i % NSC) * T); };
 
   // item it: sequence bg = it / nspan, chunk steps [tb, te) of span it % nspan
   auto span_of = [&](int it, int& bg, int& tb, int& te) {
@@ -128,8 +134,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(a_full, 1);
-    mbar_init(p_full, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&a_full[b], 1);
+      mbar_init(&p_full[b], 128);
+    }
     mbar_init(&o_full[0], 1);
     mbar_init(&o_full[1], 1);
     mbar_init(&o_empty[0], 128);
@@ -241,18 +249,20 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per tile i (chunk step gc, head subset hs): QS(i) PV(i); then, inside a
-    // chunk step, QK(i+1); after the last head subset, QK(i+1) and the state
-    // update KV(gc) (update first without a third K/V slot, so the next tile's
-    // copy is not waited for).  Every item ends with its update, so the state in
-    // tensor memory is final there.
+    // Per tile i (chunk step gc, head subset hs): QS(i) into output buffer
+    // i & 1 (once the epilogue of tile i - 2 has read it; at a chunk step's
+    // first tile, once the state copy of the step is in), then P V(i) once
+    // the mask has written P(i); after the last head subset of a chunk step
+    // the state update KV(gc).  The scores of tile i + 1 go into their own
+    // buffer: at T = 64 (two score buffers) right after QS(i), ahead of P V(i),
+    // so the next mask overlaps P V and the update; at T = 128 (one buffer,
+    // whose P(i) P V(i) still reads) after P V(i), so the next mask overlaps
+    // QS(i + 1).  At an item's end the update goes first, so the state
+    // hand-over to the next item does not wait for that item's first tiles.
     if (elect_one()) {
       auto issue_qk = [&](int i, int gci) -> bool {
-        const uint32_t ob = (uint32_t)(i & 1);
         if (!mbar_wait(&q_full[i % QST], (i / QST) & 1, p.status, abort_flag)) return false;
         if (!mbar_wait(&kv_full[gci % KVST], (gci / KVST) & 1, p.status, abort_flag)) return false;
-        if (i >= 2 && !mbar_wait(&o_empty[ob], ((i >> 1) - 1) & 1, p.status, abort_flag))
-          return false;
         tc_fence_after();
         const uint32_t q_addr = sQ(i), k_addr = sK(gci);
 #pragma unroll
@@ -260,9 +270,9 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t koff = (uint32_t)((kk & 3) * 32);
           const uint64_t da = smem_desc_sw128(q_addr + (kk >> 2) * kHalf + koff, 16, 1024);
           const uint64_t db = smem_desc_sw128(k_addr + (kk >> 2) * (T * 128) + koff, 16, 1024);
-          mma_ss(tmem + ob * 128, da, db, IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + scol(i), da, db, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(a_full);
+        mma_commit(&a_full[i % NSC]);
         return true;
       };
       auto issue_kv = [&](int gci) {
@@ -286,9 +296,15 @@ __global__ void __launch_bounds__(320, 1)
           for (int hs = 0; hs < p.nsub && ok; ++hs) {
             const uint32_t ob = (uint32_t)(i & 1);
             const uint32_t ocol = ob * 128;
-            const uint32_t pcol = 256 + ob * (T / 2);
-            if (!mbar_wait(p_full, i & 1, p.status, abort_flag)) { ok = false; break; }
+            const bool last_hs = hs == p.nsub - 1;
+            const bool item_end = last_hs && n == te - tb - 1;
+            const bool has_next = !(last_item && item_end);
+            const int gnext = last_hs ? gc + 1 : gc;  // chunk step of tile i + 1
             if (hs == 0 && !mbar_wait(sb_full, gc & 1, p.status, abort_flag)) { ok = false; break; }
+            if (i >= 2 && !mbar_wait(&o_empty[ob], ((i >> 1) - 1) & 1, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const uint32_t q_addr = sQ(i), v_addr = sV(gc);
 #pragma unroll
@@ -298,28 +314,23 @@ __global__ void __launch_bounds__(320, 1)
               const uint64_t db = smem_desc_sw128(sS + kk * 2048, kHalf, 1024);
               mma_ss(tmem + ocol, da, db, IDESC_QS, kk > 0 ? 1u : 0u);
             }
+            mma_commit(&q_empty[i % QST]);  // QK(i) and QS(i) were Q(i)'s readers
+            const bool early = NSC == 2 && !item_end;
+            if (early && !issue_qk(i + 1, gnext)) { ok = false; break; }
+            if (!mbar_wait(&p_full[i % NSC], (i / NSC) & 1, p.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < T / 16; ++kk) {  // O += P V (P from TMEM)
               const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
-              mma_ts(tmem + ocol, tmem + pcol + kk * 8, db, IDESC_PV, 1u);
+              mma_ts(tmem + ocol, tmem + scol(i) + kk * 8, db, IDESC_PV, 1u);
             }
             mma_commit(&o_full[ob]);
-            mma_commit(&q_empty[i % QST]);
-            const bool last_hs = hs == p.nsub - 1;
-            const bool item_end = last_hs && n == te - tb - 1;
-            const bool has_next = !(last_item && item_end);
-            // the next tile's scores before the update only inside an item: at
-            // an item's end the update goes first, so the state hand-over to
-            // the next item does not wait for that item's first Q tile
-            const bool qk_first = kLookahead && !item_end;
-            if (!last_hs) {
-              if (!issue_qk(i + 1, gc)) ok = false;
-            } else {
-              if (qk_first && !issue_qk(i + 1, gc + 1)) ok = false;
-              if (ok) issue_kv(gc);
-              if (ok && !qk_first && has_next && !issue_qk(i + 1, gc + 1)) ok = false;
-              ++gc;
-            }
+            if (last_hs) issue_kv(gc);
+            if (!early && has_next && !issue_qk(i + 1, gnext)) { ok = false; break; }
+            if (last_hs) ++gc;
             ++i;
           }
         }
@@ -463,13 +474,12 @@ __global__ void __launch_bounds__(320, 1)
 
     if (wg1) {
       auto mask_tile = [&](int i) -> bool {
-        const uint32_t ob = (uint32_t)(i & 1);
-        const uint32_t ocol = ob * 128;
-        const uint32_t pcol = 256 + ob * (T / 2);
-        if (!warp_wait(a_full, i & 1, p.status, abort_flag)) return false;
+        const uint32_t acol = scol(i);  // scores; P goes over their first T / 2 columns
+        if (!warp_wait(&a_full[i % NSC], (i / NSC) & 1, p.status, abort_flag)) return false;
         tc_fence_after();
         // 64 score columns per round; at T = 128 blocks entirely above the
-        // diagonal of this warp's rows are not read
+        // diagonal of this warp's rows are not read.  Round h writes P to
+        // columns [32 h, 32 h + 32), which this thread read in rounds <= h.
 #pragma unroll 1
         for (int h = 0; h < T / 64; ++h) {
           uint32_t a[2][32];
@@ -478,7 +488,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int bb = 0; bb < 2; ++bb) {
             const int blk = 2 * h + bb;
             need[bb] = T == 64 || blk <= diag_blk;
-            if (need[bb]) tmem_ld32(tmem + lane_base + ocol + blk * 32, a[bb]);
+            if (need[bb]) tmem_ld32(tmem + lane_base + acol + blk * 32, a[bb]);
           }
           tmem_wait_ld();
 #pragma unroll
@@ -494,12 +504,12 @@ __global__ void __launch_bounds__(320, 1)
               const float f1 = keep1 ? __uint_as_float(a[bb][2 * m + 1]) : 0.0f;
               pk[m] = pack_bf16x2(f0, f1);
             }
-            tmem_st16(tmem + lane_base + pcol + blk * 16, pk);
+            tmem_st16(tmem + lane_base + acol + blk * 16, pk);
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[i % NSC]);
         return true;
       };
       ok = ok && mask_tile(0);
@@ -513,13 +523,15 @@ __global__ void __launch_bounds__(320, 1)
             const bool last_hs = hs == p.nsub - 1;
             const bool item_end = last_hs && n == te - tb - 1;
             const bool has_next = !(item_end && nx < 0);
-            // the MMA order decides which of the two is ready first; one call
-            // site each (two inlined copies of either spill registers at T = 128)
-            const bool step_first = last_hs && (!kLookahead || item_end);
+            // the MMA order decides which of the two is ready first (the next
+            // tile's scores ahead of the update with two score buffers inside
+            // an item); one call site each (two inlined copies of either spill
+            // registers at T = 128)
+            const bool mask_first = NSC == 2 && !item_end;
 #pragma unroll 1
             for (int ph = 0; ph < 2 && ok; ++ph) {
-              const bool do_step = last_hs && (ph == (step_first ? 0 : 1));
-              const bool do_mask = has_next && (ph == (step_first ? 1 : 0));
+              const bool do_step = last_hs && (ph == (mask_first ? 1 : 0));
+              const bool do_mask = has_next && (ph == (mask_first ? 0 : 1));
               if (do_mask && !mask_tile(i + 1)) ok = false;
               if (ok && do_step && !state_step(gc, item_end, bg, nx, k)) ok = false;
             }

@@ -94,10 +94,10 @@ struct MainLayout {
   static constexpr int kOOff = kSOff + kSBytes;
   static constexpr int kStOff = kOOff + (kDedicatedO ? kQBytes : 0);
   static constexpr int kBarOff = kStOff + (kStage ? kStateBytes : 0);
-  // q_full[QST], q_empty[QST], kv_full[KVST], kv_empty[KVST], a_full, p_full,
-  // o_full[2], o_empty[2], s_full, sb_full, mma_done, store_ready, ostage_free,
-  // st_full, st_empty, stage_done
-  static constexpr int kNumBars = 2 * QST + 2 * KVST + 14;
+  // q_full[QST], q_empty[QST], kv_full[KVST], kv_empty[KVST], a_full[2],
+  // p_full[2], o_full[2], o_empty[2], s_full, sb_full, mma_done, store_ready,
+  // ostage_free, st_full, st_empty, stage_done
+  static constexpr int kNumBars = 2 * QST + 2 * KVST + 16;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
 };

@@ -35,14 +35,18 @@ class Model:
         self.nsub = G // (128 // T)
         self.nspan, self.tiles, self.items = nspan, tiles, units * nspan
         self.grid, self.cta, self.s_out = grid, cta, s_out
-        self.lookahead = KVST >= 3
+        # score buffers in tensor memory (P is written over its scores): two
+        # of 64 columns at T = 64, which lets QK of the next tile go ahead of
+        # PV; one of 128 at T = 128
+        self.nsc = 2 if T == 64 else 1
         self.rng = random.Random(seed)
         mk = Barrier
         self.q_full = [mk(f"q_full{s}", 1) for s in range(QST)]
         self.q_empty = [mk(f"q_empty{s}", 1 if dedo else 2) for s in range(QST)]
         self.kv_full = [mk(f"kv_full{s}", 1) for s in range(KVST)]
         self.kv_empty = [mk(f"kv_empty{s}", 1) for s in range(KVST)]
-        self.a_full, self.p_full = mk("a_full", 1), mk("p_full", 1)
+        self.a_full = [mk(f"a_full{b}", 1) for b in range(self.nsc)]
+        self.p_full = [mk(f"p_full{b}", 1) for b in range(self.nsc)]
         self.o_full = [mk("o_full0", 1), mk("o_full1", 1)]
         self.o_empty = [mk("o_empty0", 1), mk("o_empty1", 1)]
         self.s_full, self.sb_full = mk("s_full", 1), mk("sb_full", 2)
@@ -56,10 +60,11 @@ class Model:
         self.state_stores = []
         self.ver = {("q", s): None for s in range(QST)}
         self.ver.update({("kv", s): None for s in range(KVST)})
-        self.ver.update({("obuf", 0): None, ("obuf", 1): None, ("p", 0): None, ("p", 1): None,
+        self.ver.update({("obuf", 0): None, ("obuf", 1): None, ("sc", 0): None, ("sc", 1): None,
                          "sS": 0, "ostage": None, ("staging", 0): None, ("staging", 1): None})
         self.stage_need = {0: None, 1: None}  # what each half of the staging tile still owes
-        self.obuf_need = {0: None, 1: None}   # scores or output a buffer still owes a reader
+        self.obuf_need = {0: None, 1: None}   # output a buffer still owes the epilogue
+        self.sc_need = {0: None, 1: None}     # scores the mask, or P the PV, has yet to read
         self.state_chunk = None   # the chunk step after which the state in TMEM is final
         self.state_ready = 0      # the chunk step whose update may run next
         self.stored = []
@@ -165,25 +170,20 @@ class Model:
     # ----------------------------------------------------------- MMA
     def mma_role(self):
         seq = list(self.steps())
-        first_gc = {}
-        for x in seq:
-            first_gc.setdefault(x["gc"], x["i"])
 
         def qk(i, gci):
-            ob = i & 1
+            sc = i % self.nsc
             yield from self.wait("mma", self.q_full[i % self.QST], i // self.QST)
             yield from self.wait("mma", self.kv_full[gci % self.KVST], gci // self.KVST)
-            if i >= 2:
-                yield from self.wait("mma", self.o_empty[ob], (i >> 1) - 1)
 
             def run():
-                assert self.obuf_need[ob] is None, (
-                    f"QK({i}) overwrites {self.obuf_need[ob]} before it was read")
-                self.ver[("obuf", ob)] = ("A", i)
-                self.obuf_need[ob] = ("A", i)
+                assert self.sc_need[sc] is None, (
+                    f"QK({i}) overwrites {self.sc_need[sc]} before it was read")
+                self.ver[("sc", sc)] = ("A", i)
+                self.sc_need[sc] = ("A", i)
             self.mma(f"QK({i})", [(("q", i % self.QST), ("Q", i)),
                                   (("kv", gci % self.KVST), gci)], run)
-            self.commit(self.a_full)
+            self.commit(self.a_full[sc])
 
         def kv(gci):
             def run():
@@ -195,32 +195,35 @@ class Model:
 
         yield from qk(0, 0)
         for x in seq:
-            i, gc, ob = x["i"], x["gc"], x["i"] & 1
-            yield from self.wait("mma", self.p_full, i)
+            i, gc, ob, sc = x["i"], x["gc"], x["i"] & 1, x["i"] % self.nsc
             if x["hs"] == 0:
                 yield from self.wait("mma", self.sb_full, gc)
+            if i >= 2:
+                yield from self.wait("mma", self.o_empty[ob], (i >> 1) - 1)
 
             def qs_run(ob=ob, i=i):
-                assert self.obuf_need[ob] is None, f"QS({i}) overwrites unread scores"
+                assert self.obuf_need[ob] is None, f"QS({i}) overwrites unread output"
                 self.ver[("obuf", ob)] = ("O", i)
 
-            def pv_run(ob=ob, i=i):
+            def pv_run(ob=ob, i=i, sc=sc):
+                self.sc_need[sc] = None
                 self.obuf_need[ob] = ("O", i)
-            self.mma(f"QS({i})", [(("q", i % self.QST), ("Q", i)), ("sS", gc),
-                                  (("obuf", ob), ("A", i))], qs_run)
-            self.mma(f"PV({i})", [(("p", ob), i), (("kv", gc % self.KVST), gc),
+            self.mma(f"QS({i})", [(("q", i % self.QST), ("Q", i)), ("sS", gc)], qs_run)
+            self.commit(self.q_empty[i % self.QST])
+            nxt = gc + 1 if x["last_hs"] else gc
+            # with two score buffers the next tile's scores go ahead of PV
+            # (inside an item; at its end the state update goes first)
+            early = self.nsc == 2 and not x["item_end"]
+            if early:
+                yield from qk(i + 1, nxt)
+            yield from self.wait("mma", self.p_full[sc], i // self.nsc)
+            self.mma(f"PV({i})", [(("sc", sc), ("P", i)), (("kv", gc % self.KVST), gc),
                                   (("obuf", ob), ("O", i))], pv_run)
             self.commit(self.o_full[ob])
-            self.commit(self.q_empty[i % self.QST])
-            qk_first = self.lookahead and not x["item_end"]
-            if not x["last_hs"]:
-                yield from qk(i + 1, gc)
-            else:
-                if qk_first:
-                    yield from qk(i + 1, gc + 1)
+            if x["last_hs"]:
                 kv(gc)
-                if not qk_first and x["has_next"]:
-                    yield from qk(i + 1, gc + 1)
+            if not early and x["has_next"]:
+                yield from qk(i + 1, nxt)
             yield
 
     # ----------------------------------------------------------- warpgroups
@@ -276,20 +279,23 @@ class Model:
         yield from self.first_state(role)
 
         def mask_tile(i):
-            ob = i & 1
-            yield from self.wait(role, self.a_full, i)
-            self.expect(("obuf", ob), ("A", i), f"mask({i})")
-            self.obuf_need[ob] = None
-            self.overwrite(("p", ob), i, f"mask({i})")
-            self.p_full.arrive()
+            sc = i % self.nsc
+            yield from self.wait(role, self.a_full[sc], i // self.nsc)
+            self.expect(("sc", sc), ("A", i), f"mask({i})")
+            self.overwrite(("sc", sc), ("P", i), f"mask({i})")  # P over its scores
+            self.sc_need[sc] = ("P", i)
+            self.p_full[sc].arrive()
 
         yield from mask_tile(0)
         for x in self.steps():
             nx = self.next_item(x["it"])
-            step_first = x["last_hs"] and (not self.lookahead or x["item_end"])
+            # the MMA order decides which is ready first: with the next tile's
+            # scores ahead of PV (two score buffers, inside an item) the mask
+            # comes before the state step
+            mask_first = self.nsc == 2 and not x["item_end"]
             for ph in (0, 1):
-                do_step = x["last_hs"] and ph == (0 if step_first else 1)
-                do_mask = x["has_next"] and ph == (1 if step_first else 0)
+                do_step = x["last_hs"] and ph == (1 if mask_first else 0)
+                do_mask = x["has_next"] and ph == (0 if mask_first else 1)
                 if do_mask:
                     yield from mask_tile(x["i"] + 1)
                 if do_step:
@@ -379,9 +385,6 @@ CONFIGS = {
     "t64_dedicated_out": dict(T=64, QST=3, KVST=2, dedo=True, staged=False),
     "t64_staged": dict(T=64, QST=2, KVST=2, dedo=False, staged=True),
     "t128": dict(T=128, QST=2, KVST=2, dedo=False, staged=False),
-    # a third K/V slot (scores of the next step before the state update):
-    # supported by the kernel, not chosen by the launcher at present
-    "t64_kv_lookahead": dict(T=64, QST=3, KVST=3, dedo=True, staged=False),
 }
 
 SHAPES = [
@@ -427,10 +430,19 @@ def test_persist_protocol(config, G, units, nspan, tiles, grid, s_out):
 MUTANTS = {
     "epilogue without o_full": (
         "            yield from self.wait(role, self.o_full[ob], i >> 1)\n", ""),
-    "QK without o_empty": (
+    "QS without o_empty": (
         "            if i >= 2:\n"
         "                yield from self.wait(\"mma\", self.o_empty[ob], (i >> 1) - 1)\n", ""),
-    "mask without a_full": ("            yield from self.wait(role, self.a_full, i)\n", ""),
+    "mask without a_full": (
+        "            yield from self.wait(role, self.a_full[sc], i // self.nsc)\n", ""),
+    "PV without p_full": (
+        "            yield from self.wait(\"mma\", self.p_full[sc], i // self.nsc)\n", ""),
+    "next scores ahead of PV with one score buffer": (
+        "            early = self.nsc == 2 and not x[\"item_end\"]\n",
+        "            early = not x[\"item_end\"]\n"),
+    "one a_full barrier for two score buffers": (
+        "        self.a_full = [mk(f\"a_full{b}\", 1) for b in range(self.nsc)]",
+        "        self.a_full = [mk(\"a_full\", 1)] * self.nsc"),
     "K/V copy without kv_empty": (
         "            if gc >= self.KVST:\n"
         "                yield from self.wait(\"kv\", self.kv_empty[s], gc // self.KVST - 1)\n", ""),
