@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(320, 1)
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
   constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, 1, 1);
   constexpr int NSC = T == 64 ? 2 : 1;  // score buffers
+  // T = 128: P handed over, and multiplied by V, in two halves of 64 keys
+  constexpr int NPH = T == 128 ? 2 : 1;
   constexpr int kDD = kHeadDim * kHeadDim;
 
   extern __shared__ uint8_t smem_raw[];
@@ -317,16 +319,21 @@ __global__ void __launch_bounds__(320, 1)
             mma_commit(&q_empty[i % QST]);  // QK(i) and QS(i) were Q(i)'s readers
             const bool early = NSC == 2 && !item_end;
             if (early && !issue_qk(i + 1, gnext)) { ok = false; break; }
-            if (!mbar_wait(&p_full[i % NSC], (i / NSC) & 1, p.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < T / 16; ++kk) {  // O += P V (P from TMEM)
-              const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
-              mma_ts(tmem + ocol, tmem + scol(i) + kk * 8, db, IDESC_PV, 1u);
+            for (int ph = 0; ph < NPH && ok; ++ph) {  // O += P V (P from TMEM), half by half
+              uint64_t* pf = NPH == 2 ? &p_full[ph] : &p_full[i % NSC];
+              if (!mbar_wait(pf, (i / NSC) & 1, p.status, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = ph * (T / 16 / NPH); kk < (ph + 1) * (T / 16 / NPH); ++kk) {
+                const uint64_t db = smem_desc_sw128(v_addr + kk * 2048, T * 128, 1024);
+                mma_ts(tmem + ocol, tmem + scol(i) + kk * 8, db, IDESC_PV, 1u);
+              }
             }
+            if (!ok) break;
             mma_commit(&o_full[ob]);
             if (last_hs) issue_kv(gc);
             if (!early && has_next && !issue_qk(i + 1, gnext)) { ok = false; break; }
@@ -506,10 +513,17 @@ __global__ void __launch_bounds__(320, 1)
             }
             tmem_st16(tmem + lane_base + acol + blk * 16, pk);
           }
+          if (NPH == 2) {  // this half of P is ready for its half of P V
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_full[h]);
+          }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[i % NSC]);
+        if (NPH == 1) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_full[i % NSC]);
+        }
         return true;
       };
       ok = ok && mask_tile(0);

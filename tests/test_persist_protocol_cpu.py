@@ -29,9 +29,12 @@ from test_walk_protocol_cpu import Barrier
 
 
 class Model:
-    def __init__(self, T, QST, KVST, dedo, staged, G, units, nspan, tiles, grid, cta, s_out,
+    def __init__(self, T, QST, KVST, out, staged, G, units, nspan, tiles, grid, cta, s_out,
                  seed):
-        self.T, self.QST, self.KVST, self.dedo, self.staged = T, QST, KVST, dedo, staged
+        # out: "dedicated" (output tile of its own), "qslot" (output staged in
+        # the tile's Q slot), "direct" (registers to global memory, no staging)
+        self.T, self.QST, self.KVST, self.out, self.staged = T, QST, KVST, out, staged
+        self.dedo = out == "dedicated"
         self.nsub = G // (128 // T)
         self.nspan, self.tiles, self.items = nspan, tiles, units * nspan
         self.grid, self.cta, self.s_out = grid, cta, s_out
@@ -39,14 +42,18 @@ class Model:
         # of 64 columns at T = 64, which lets QK of the next tile go ahead of
         # PV; one of 128 at T = 128
         self.nsc = 2 if T == 64 else 1
+        # at T = 128 the mask hands P over in two halves of 64 keys, each
+        # multiplied by V (P V in two halves) as soon as it is written
+        self.halves = 2 if T == 128 else 1
         self.rng = random.Random(seed)
         mk = Barrier
         self.q_full = [mk(f"q_full{s}", 1) for s in range(QST)]
-        self.q_empty = [mk(f"q_empty{s}", 1 if dedo else 2) for s in range(QST)]
+        self.q_empty = [mk(f"q_empty{s}", 2 if out == "qslot" else 1) for s in range(QST)]
         self.kv_full = [mk(f"kv_full{s}", 1) for s in range(KVST)]
         self.kv_empty = [mk(f"kv_empty{s}", 1) for s in range(KVST)]
         self.a_full = [mk(f"a_full{b}", 1) for b in range(self.nsc)]
-        self.p_full = [mk(f"p_full{b}", 1) for b in range(self.nsc)]
+        # per score buffer at T = 64; per half of the one buffer at T = 128
+        self.p_full = [mk(f"p_full{b}", 1) for b in range(max(self.nsc, self.halves))]
         self.o_full = [mk("o_full0", 1), mk("o_full1", 1)]
         self.o_empty = [mk("o_empty0", 1), mk("o_empty1", 1)]
         self.s_full, self.sb_full = mk("s_full", 1), mk("sb_full", 2)
@@ -62,6 +69,7 @@ class Model:
         self.ver.update({("kv", s): None for s in range(KVST)})
         self.ver.update({("obuf", 0): None, ("obuf", 1): None, ("sc", 0): None, ("sc", 1): None,
                          "sS": 0, "ostage": None, ("staging", 0): None, ("staging", 1): None})
+        self.ver.update({("ph", b, h): None for b in range(2) for h in range(2)})
         self.stage_need = {0: None, 1: None}  # what each half of the staging tile still owes
         self.obuf_need = {0: None, 1: None}   # output a buffer still owes the epilogue
         self.sc_need = {0: None, 1: None}     # scores the mask, or P the PV, has yet to read
@@ -208,6 +216,9 @@ class Model:
             def pv_run(ob=ob, i=i, sc=sc):
                 self.sc_need[sc] = None
                 self.obuf_need[ob] = ("O", i)
+
+            def pv_half_run():
+                pass
             self.mma(f"QS({i})", [(("q", i % self.QST), ("Q", i)), ("sS", gc)], qs_run)
             self.commit(self.q_empty[i % self.QST])
             nxt = gc + 1 if x["last_hs"] else gc
@@ -216,9 +227,13 @@ class Model:
             early = self.nsc == 2 and not x["item_end"]
             if early:
                 yield from qk(i + 1, nxt)
-            yield from self.wait("mma", self.p_full[sc], i // self.nsc)
-            self.mma(f"PV({i})", [(("sc", sc), ("P", i)), (("kv", gc % self.KVST), gc),
-                                  (("obuf", ob), ("O", i))], pv_run)
+            for h in range(self.halves):
+                pf = self.p_full[h] if self.halves == 2 else self.p_full[sc]
+                yield from self.wait("mma", pf, i // self.nsc)
+                last_half = h == self.halves - 1
+                self.mma(f"PV{h}({i})", [(("ph", sc, h), ("P", i)), (("kv", gc % self.KVST), gc),
+                                         (("obuf", ob), ("O", i))],
+                         pv_run if last_half else pv_half_run)
             self.commit(self.o_full[ob])
             if x["last_hs"]:
                 kv(gc)
@@ -282,9 +297,12 @@ class Model:
             sc = i % self.nsc
             yield from self.wait(role, self.a_full[sc], i // self.nsc)
             self.expect(("sc", sc), ("A", i), f"mask({i})")
-            self.overwrite(("sc", sc), ("P", i), f"mask({i})")  # P over its scores
             self.sc_need[sc] = ("P", i)
-            self.p_full[sc].arrive()
+            for h in range(self.halves):  # P over its scores, half by half
+                self.overwrite(("ph", sc, h), ("P", i), f"mask({i})")
+                (self.p_full[h] if self.halves == 2 else self.p_full[sc]).arrive()
+                if h + 1 < self.halves:
+                    yield
 
         yield from mask_tile(0)
         for x in self.steps():
@@ -320,6 +338,13 @@ class Model:
                 else:
                     self.st_empty.arrive()
             yield from self.wait(role, self.o_full[ob], i >> 1)
+            if self.out == "direct":  # registers to global memory, no tile to stage in
+                self.expect(("obuf", ob), ("O", i), f"epilogue({i})")
+                self.obuf_need[ob] = None
+                self.o_empty[ob].arrive()
+                self.stored.append((x["it"], x["n"], x["hs"]))
+                yield
+                continue
             if self.dedo and i > 0:
                 yield from self.wait(role, self.ostage_free, i - 1)
             self.expect(("obuf", ob), ("O", i), f"epilogue({i})")
@@ -382,9 +407,9 @@ class Model:
 
 
 CONFIGS = {
-    "t64_dedicated_out": dict(T=64, QST=3, KVST=2, dedo=True, staged=False),
-    "t64_staged": dict(T=64, QST=2, KVST=2, dedo=False, staged=True),
-    "t128": dict(T=128, QST=2, KVST=2, dedo=False, staged=False),
+    "t64_dedicated_out": dict(T=64, QST=3, KVST=2, out="dedicated", staged=False),
+    "t64_staged": dict(T=64, QST=2, KVST=2, out="qslot", staged=True),
+    "t128": dict(T=128, QST=2, KVST=2, out="qslot", staged=False),
 }
 
 SHAPES = [
@@ -436,7 +461,7 @@ MUTANTS = {
     "mask without a_full": (
         "            yield from self.wait(role, self.a_full[sc], i // self.nsc)\n", ""),
     "PV without p_full": (
-        "            yield from self.wait(\"mma\", self.p_full[sc], i // self.nsc)\n", ""),
+        "                yield from self.wait(\"mma\", pf, i // self.nsc)\n", ""),
     "next scores ahead of PV with one score buffer": (
         "            early = self.nsc == 2 and not x[\"item_end\"]\n",
         "            early = not x[\"item_end\"]\n"),
@@ -461,8 +486,11 @@ MUTANTS = {
         "            if x[\"hs\"] == 0:\n"
         "                yield from self.wait(\"mma\", self.sb_full, gc)\n", ""),
     "q_empty released by the MMA alone": (
-        "self.q_empty = [mk(f\"q_empty{s}\", 1 if dedo else 2) for s in range(QST)]",
+        "self.q_empty = [mk(f\"q_empty{s}\", 2 if out == \"qslot\" else 1) for s in range(QST)]",
         "self.q_empty = [mk(f\"q_empty{s}\", 1) for s in range(QST)]"),
+    "second half of P V before its half of P": (
+        "                pf = self.p_full[h] if self.halves == 2 else self.p_full[sc]\n",
+        "                pf = self.p_full[0] if self.halves == 2 else self.p_full[sc]\n"),
 }
 
 
