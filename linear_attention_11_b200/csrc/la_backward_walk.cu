@@ -17,8 +17,9 @@
 //
 // Per 128-token chunk c of a group, per 64-token key block (head h, half j):
 //   S1 = K_c Q_hj^T, S2 = V_c dO_hj^T   M=128 N=64  K=128 (SS) -> TMEM
-//   P1, P2 = bf16(triu(S1)), bf16(triu(S2))   TMEM -> registers -> smem
-//   dv += P1 dO_hj, dk += P2 Q_hj       M=128 N=128 K=64 (SS)
+//   P1, P2 = bf16(triu(S1)), bf16(triu(S2))   TMEM -> registers -> TMEM, each
+//                                             over its own scores
+//   dv += P1 dO_hj, dk += P2 Q_hj       M=128 N=128 K=64 (P from TMEM)
 //   D  += Q_hj^T dO_hj                  M=128 N=128 K=64 (SS, both MN-major)
 // and once per chunk, from the bf16 copy of D_c in smem (read MN-major for D,
 // K-major for D^T):  dv += K_c D_c,  dk += V_c D_c^T  (M=128 N=128 K=128).
@@ -28,12 +29,15 @@
 // the later spans' sums, from group_scan_kernel) is read at the item start,
 // and the item of span 0 writes dS0 at its end.
 // Roles (320 threads): warp 0 lane 0 streams key blocks (Q and dO of one head
-// half-chunk) through a three-stage ring and prefetches the blocks six ahead
+// half-chunk) through a four-stage ring and prefetches the blocks six ahead
 // into L2, lane 1 the K/V tiles of each chunk (and the next chunk's into L2);
-// warp 1 owns the tensor memory and
-// issues the MMAs, scores two blocks ahead; warps 2-5 mask S1, convert the
-// state and write dv rows out; warps 6-9 mask S2 and write dk rows out.
-// TMEM: dv at column 0, dk at 128, S1 at 256, S2 at 320, D at 384.
+// warp 1 owns the tensor memory and issues the MMAs; warps 2-5 mask S1,
+// convert the state and write dv rows out; warps 6-9 mask S2 and write dk
+// rows out.  TMEM: dv at column 0, dk at 128, S1 (then P1) at 256, S2 (then
+// P2) at 320, D at 384.  The two score streams run apart: a stream's next
+// scores are issued right after the product that reads its P, so the tensor
+// pipe's order keeps them off P, and one stream's mask overlaps the other
+// stream's MMAs.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -48,12 +52,11 @@ namespace {
 
 constexpr int kChunk = 128;                         // tokens per chunk
 constexpr int kKeyBlk = 64;                         // tokens per key block
-constexpr int kRing = 3;                            // key-block stages
+constexpr int kRing = 4;                            // key-block stages
 constexpr int kPrefetch = 6;                        // key blocks prefetched into L2 ahead
 constexpr int kChunkBytes = kChunk * kHeadDim * 2;  // 32 KB: K_c or V_c
 constexpr int kBlkBytes = kKeyBlk * kHeadDim * 2;   // 16 KB: Q or dO of one block
 constexpr int kBlkHalf = kKeyBlk * 128;             // 8 KB: 64 columns of a key block
-constexpr int kPBytes = kChunk * kKeyBlk * 2;       // 16 KB: one P tile
 constexpr uint32_t kColDv = 0, kColDk = 128, kColS1 = 256, kColS2 = 320;
 
 struct WalkLayout {
@@ -61,10 +64,9 @@ struct WalkLayout {
   static constexpr int kVOff = kChunkBytes;
   static constexpr int kRingOff = 2 * kChunkBytes;                // stage: Q block, dO block
   static constexpr int kSOff = kRingOff + kRing * 2 * kBlkBytes;  // bf16 copy of D
-  static constexpr int kPOff = kSOff + kSBytes;                   // P1, P2
-  static constexpr int kBarOff = kPOff + 2 * kPBytes;
-  // ring_full[R], ring_empty[R], kv_full, kv_empty, a_full, s_read, p_full,
-  // p_free, o_full, o_empty[2], s_full, sb_full, mma_done
+  static constexpr int kBarOff = kSOff + kSBytes;
+  // ring_full[R], ring_empty[R], kv_full, kv_empty, a_full[2], p_full[2],
+  // o_full, o_empty[2], s_full, sb_full, mma_done
   static constexpr int kNumBars = 2 * kRing + 12;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
@@ -133,14 +135,6 @@ __device__ __forceinline__ void cursor_next(const WalkParams& p, Cursor& c) {
   if (c.valid) cursor_item(p, c);
 }
 
-__device__ __forceinline__ void store_p_row(uint32_t tile, int r, const uint32_t (&pk)[32]) {
-  const uint32_t row = tile + (uint32_t)(r * 128);
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    st_shared_v4(row + (uint32_t)((c ^ (r & 7)) * 16), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                 pk[4 * c + 3]);
-}
-
 __global__ void __launch_bounds__(320, 1)
     bwd_walk_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_do,
@@ -163,11 +157,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* ring_empty = ring_full + kRing;
   uint64_t* kv_full = ring_empty + kRing;
   uint64_t* kv_empty = kv_full + 1;
-  uint64_t* a_full = kv_empty + 1;   // S1, S2 of a block computed
-  uint64_t* s_read = a_full + 1;     // ... and read out by the mask warps
-  uint64_t* p_full = s_read + 1;     // P1, P2 of a block in smem
-  uint64_t* p_free = p_full + 1;     // the P tiles read by their MMAs
-  uint64_t* o_full = p_free + 1;     // dv, dk of a chunk complete
+  uint64_t* a_full = kv_empty + 1;   // two: S1, S2 of a block computed
+  uint64_t* p_full = a_full + 2;     // two: P1, P2 of a block written over their scores
+  uint64_t* o_full = p_full + 2;     // dv, dk of a chunk complete
   uint64_t* o_empty = o_full + 1;    // two: dv, dk read out
   uint64_t* s_full = o_empty + 2;    // D updated with a chunk
   uint64_t* sb_full = s_full + 1;    // bf16 copy of D (and D itself at an item start) ready
@@ -177,7 +169,6 @@ __global__ void __launch_bounds__(320, 1)
 
   const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
   const uint32_t sS = base + L::kSOff;
-  const uint32_t sP1 = base + L::kPOff, sP2 = sP1 + kPBytes;
   auto sQ = [&](int s) { return base + (uint32_t)(L::kRingOff + s * 2 * kBlkBytes); };
   auto sDO = [&](int s) { return sQ(s) + (uint32_t)kBlkBytes; };
   const int stride = (int)gridDim.x;
@@ -192,10 +183,10 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    mbar_init(a_full, 1);
-    mbar_init(s_read, 256);
-    mbar_init(p_full, 256);
-    mbar_init(p_free, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&a_full[t], 1);
+      mbar_init(&p_full[t], 128);
+    }
     mbar_init(o_full, 1);
     mbar_init(&o_empty[0], 128);
     mbar_init(&o_empty[1], 128);
@@ -313,34 +304,33 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Tensor pipe order: S(0) S(1) | PV(0) D(0) S(2) | PV(1) D(1) S(3) | ...
-    // so the scores of block i+1 are masked while block i's products run.
-    // K_c and V_c sit in one slot: their copy for the next chunk starts once
-    // the chunk's last S and its K_c D, V_c D^T are issued, and a next chunk's
-    // first S is held back until that point.
+    // Per block k: dk += P2(k) Q(k) (a chunk's first block starts dk, then
+    // V_c D^T), the next block's S2, dv += P1(k) dO(k) (then K_c D), D += Q^T
+    // dO, the next block's S1.  Each stream's next scores come after the
+    // product that reads its P (the tensor pipe runs in issue order), and
+    // one stream's mask overlaps the other's MMAs.  K_c and V_c sit in one
+    // slot, released once the chunk's last S1 and its K_c D are issued; a
+    // next chunk's scores therefore go at the end of the block.
     if (elect_one()) {
-      Cursor a, c;  // a: next block to score; c: next block to multiply
-      cursor_init(p, a);
-      cursor_init(p, c);
-      int inter_gc = -1;   // last chunk whose K_c D, V_c D^T are issued
-      int kv_pending = -1; // chunk whose last S is issued before its K_c D
-      auto issue_s = [&](const Cursor& x) -> bool {
+      int inter_gc = -1;    // last chunk whose K_c D, V_c D^T are issued
+      int kv_pending = -1;  // chunk whose last S1 is issued before its K_c D
+      auto issue_s = [&](int t, const Cursor& x) -> bool {
         if (x.blk == 0 && !mbar_wait(kv_full, x.gc & 1, p.status, abort_flag)) return false;
         const int s = x.i % kRing;
         if (!mbar_wait(&ring_full[s], (x.i / kRing) & 1, p.status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t qa = sQ(s), doa = sDO(s);
+        const uint32_t src = t == 0 ? sK : sV;               // K_c or V_c
+        const uint32_t blk = t == 0 ? sQ(s) : sDO(s);        // Q or dO of the block
+        const uint32_t dst = tmem + (t == 0 ? kColS1 : kColS2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // S1 = K_c Q^T, S2 = V_c dO^T (all K-major)
           const uint32_t koff = (uint32_t)((kk & 3) * 32);
           const uint32_t ch = (uint32_t)(kk >> 2);
-          mma_ss(tmem + kColS1, smem_desc_sw128(sK + ch * kHalf + koff, 16, 1024),
-                 smem_desc_sw128(qa + ch * kBlkHalf + koff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-          mma_ss(tmem + kColS2, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
-                 smem_desc_sw128(doa + ch * kBlkHalf + koff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(dst, smem_desc_sw128(src + ch * kHalf + koff, 16, 1024),
+                 smem_desc_sw128(blk + ch * kBlkHalf + koff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        mma_commit(a_full);
-        if (x.blk == x.nb - 1) {
+        mma_commit(&a_full[t]);
+        if (t == 0 && x.blk == x.nb - 1) {  // the chunk's last score read of K_c, V_c
           if (inter_gc >= x.gc)
             mma_commit(kv_empty);
           else
@@ -348,34 +338,24 @@ __global__ void __launch_bounds__(320, 1)
         }
         return true;
       };
-      // score blocks up to c + 1 (the S tiles are free once the block before
-      // was read out); a chunk's first block waits for the K/V slot rule
-      auto score_ahead = [&](bool must) -> bool {
-        while (a.valid && a.i <= c.i + 1) {
-          if (a.blk == 0 && inter_gc < a.gc - 1 && !(must && a.i == c.i)) break;
-          if (a.i > 0 && !mbar_wait(s_read, (a.i - 1) & 1, p.status, abort_flag)) return false;
-          if (!issue_s(a)) return false;
-          cursor_next(p, a);
-        }
-        return true;
-      };
-      bool ok = score_ahead(true);
+      Cursor c;
+      cursor_init(p, c);
+      bool ok = !c.valid || (issue_s(1, c) && issue_s(0, c));
       while (ok && c.valid) {
-        if (a.valid && a.i == c.i && !score_ahead(true)) break;
-        const int k = c.i;
+        Cursor nx = c;
+        cursor_next(p, nx);
+        const int k = c.i, s = k % kRing;
         const bool first = c.blk == 0, last = c.blk == c.nb - 1;
-        if (!mbar_wait(p_full, k & 1, p.status, abort_flag)) break;
-        tc_fence_after();
-        const int s = k % kRing;
         const uint32_t qa = sQ(s), doa = sDO(s);
         // dk += P2 Q (a chunk's first block starts dk once it has been read
-        // out), then V_c D^T; dv += P1 dO, then K_c D
+        // out), then V_c D^T
+        if (!mbar_wait(&p_full[1], k & 1, p.status, abort_flag)) break;
         if (first && c.gc >= 1 && !mbar_wait(&o_empty[1], (c.gc - 1) & 1, p.status, abort_flag))
           break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kKeyBlk / 16; ++kk)
-          mma_ss(tmem + kColDk, smem_desc_sw128(sP2 + kk * 32, 16, 1024),
+          mma_ts(tmem + kColDk, tmem + kColS2 + kk * 8,
                  smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024), IDESC_PV,
                  (first && kk == 0) ? 0u : 1u);
         if (first) {
@@ -388,12 +368,16 @@ __global__ void __launch_bounds__(320, 1)
             mma_ss(tmem + kColDk, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
                    smem_desc_sw128(sS + ch * kHalf + koff, 16, 1024), IDESC_VDT, 1u);
           }
-          if (c.gc >= 1 && !mbar_wait(&o_empty[0], (c.gc - 1) & 1, p.status, abort_flag)) break;
-          tc_fence_after();
         }
+        if (nx.valid && nx.blk != 0 && !issue_s(1, nx)) break;
+        // dv += P1 dO, then K_c D
+        if (!mbar_wait(&p_full[0], k & 1, p.status, abort_flag)) break;
+        if (first && c.gc >= 1 && !mbar_wait(&o_empty[0], (c.gc - 1) & 1, p.status, abort_flag))
+          break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kKeyBlk / 16; ++kk)
-          mma_ss(tmem + kColDv, smem_desc_sw128(sP1 + kk * 32, 16, 1024),
+          mma_ts(tmem + kColDv, tmem + kColS1 + kk * 8,
                  smem_desc_sw128(doa + kk * 2048, kBlkHalf, 1024), IDESC_PV,
                  (first && kk == 0) ? 0u : 1u);
         if (first) {
@@ -410,7 +394,6 @@ __global__ void __launch_bounds__(320, 1)
             kv_pending = -1;
           }
         }
-        mma_commit(p_free);  // the next block's P may be stored during D's update
 #pragma unroll
         for (int kk = 0; kk < kKeyBlk / 16; ++kk)  // D += Q^T dO (both MN-major)
           mma_ss(tmem + kColS, smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024),
@@ -420,8 +403,11 @@ __global__ void __launch_bounds__(320, 1)
           mma_commit(o_full);
           mma_commit(s_full);
         }
-        cursor_next(p, c);
-        if (!score_ahead(false)) break;
+        if (nx.valid) {
+          if (nx.blk == 0 && !issue_s(1, nx)) break;
+          if (!issue_s(0, nx)) break;
+        }
+        c = nx;
       }
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0);
@@ -437,7 +423,6 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t col_s = wg1 ? kColS1 : kColS2;
     const uint32_t col_o = wg1 ? kColDv : kColDk;
-    const uint32_t sP = wg1 ? sP1 : sP2;
     __nv_bfloat16* const out_base = wg1 ? p.dv : p.dk;
     uint64_t* const my_empty = &o_empty[wg1 ? 0 : 1];
     bool ok = true;
@@ -509,42 +494,43 @@ __global__ void __launch_bounds__(320, 1)
       return true;
     };
 
-    // this warpgroup's score tile of block c -> masked bf16 P tile in smem
+    // this warpgroup's score tile of block c -> masked bf16 P over the first
+    // 32 columns of the same tensor-memory buffer (every score is in
+    // registers before P is written)
+    const int t = wg1 ? 0 : 1;
     auto mask_block = [&](const Cursor& c) -> bool {
       const int k = c.i;
       const int halves = c.nb / p.G;
       const int j = c.blk % halves;
-      if (!warp_wait(a_full, k & 1, p.status, abort_flag)) return false;
+      if (!warp_wait(&a_full[t], k & 1, p.status, abort_flag)) return false;
       tc_fence_after();
       // key column u of the block is token 64 j + u of the chunk; row r keeps
       // u >= r - 64 j.  Rows 64..127 keep nothing of the first half.
       const int rel = r - kKeyBlk * j;
       const bool none = j == 0 && quarter >= 2;
-      uint32_t pk[32];
+      uint32_t pa[16], pb[16];
       if (!none) {
         uint32_t x0[32], x1[32];
         tmem_ld32(tmem + lane_base + col_s, x0);
         tmem_ld32(tmem + lane_base + col_s + 32, x1);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(s_read);  // the score columns may be overwritten
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
           const int u = 2 * m;
-          pk[m] = pack_bf16x2(u >= rel ? __uint_as_float(x0[u]) : 0.f,
+          pa[m] = pack_bf16x2(u >= rel ? __uint_as_float(x0[u]) : 0.f,
                               u + 1 >= rel ? __uint_as_float(x0[u + 1]) : 0.f);
-          pk[16 + m] = pack_bf16x2(u + 32 >= rel ? __uint_as_float(x1[u]) : 0.f,
-                                   u + 33 >= rel ? __uint_as_float(x1[u + 1]) : 0.f);
+          pb[m] = pack_bf16x2(u + 32 >= rel ? __uint_as_float(x1[u]) : 0.f,
+                              u + 33 >= rel ? __uint_as_float(x1[u + 1]) : 0.f);
         }
       } else {
-        mbar_arrive(s_read);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) pk[m] = 0u;
+        for (int m = 0; m < 16; ++m) pa[m] = pb[m] = 0u;
       }
-      if (k >= 1 && !warp_wait(p_free, (k - 1) & 1, p.status, abort_flag)) return false;
-      store_p_row(sP, r, pk);
-      fence_proxy_async_smem();
-      mbar_arrive(p_full);
+      tmem_st16(tmem + lane_base + col_s, pa);
+      tmem_st16(tmem + lane_base + col_s + 16, pb);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
       return true;
     };
 

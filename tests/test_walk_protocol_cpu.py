@@ -13,12 +13,13 @@ scheduler interleaves the roles.  Checked for many shapes and interleavings:
   - parity: a wait for phase k of a barrier only starts, or stays blocked,
     while at most k + 1 phases have completed (a parity wait cannot tell
     phase k from phase k + 2);
-  - data: every operand an MMA reads (ring slot, K/V slot, P tile, bf16
-    state copy) holds the version it was issued for when the MMA executes,
-    and no copy, P store or state conversion overwrites a version a queued
-    MMA still needs; score tiles are read by both mask warpgroups before the
-    next scores land; the state D is reloaded or converted before the next
-    chunk's updates; dk, dv are read out before the next chunk starts them;
+  - data: every operand an MMA reads (ring slot, K/V slot, P over its scores
+    in tensor memory, bf16 state copy) holds the version it was issued for
+    when the MMA executes, and no copy, P store or state conversion
+    overwrites a version a queued MMA still needs; each score buffer's P is
+    multiplied before the next scores of its stream land; the state D is
+    reloaded or converted before the next chunk's updates; dk, dv are read
+    out before the next chunk starts them;
   - coverage: every (group, chunk, key block) is multiplied exactly once and
     every chunk's dk, dv are written exactly once.
 
@@ -29,7 +30,7 @@ import random
 
 import pytest
 
-RING = 3
+RING = 4
 CHUNK, KEYBLK = 128, 64
 
 
@@ -58,8 +59,11 @@ class Model:
         self.ring_full = [mk(f"ring_full{s}", 1) for s in range(RING)]
         self.ring_empty = [mk(f"ring_empty{s}", 1) for s in range(RING)]
         self.kv_full, self.kv_empty = mk("kv_full", 1), mk("kv_empty", 1)
-        self.a_full, self.s_read = mk("a_full", 1), mk("s_read", 2)
-        self.p_full, self.p_free = mk("p_full", 2), mk("p_free", 1)
+        # two score streams, each in its own tensor-memory buffer: S1 = K_c Q^T
+        # (masked by warpgroup 1 into P1, for dv) and S2 = V_c dO^T (warpgroup
+        # 2, P2, for dk); each P is written over its own scores
+        self.a_full = [mk("a_full1", 1), mk("a_full2", 1)]
+        self.p_full = [mk("p_full1", 1), mk("p_full2", 1)]
         self.o_full = mk("o_full", 1)
         self.o_empty = [mk("o_empty0", 1), mk("o_empty1", 1)]
         self.s_full, self.sb_full = mk("s_full", 1), mk("sb_full", 1)
@@ -68,10 +72,10 @@ class Model:
         self.copies = []       # (barrier, resource, version), landing in any order
         # resource versions
         self.ver = {("ring", s): None for s in range(RING)}
-        self.ver.update({"kv": None, "P1": None, "P2": None, "sS": 0, "S": None})
+        self.ver.update({"kv": None, "sS": 0, ("S", 0): None, ("S", 1): None})
+        self.sc_need = {0: None, 1: None}  # scores or P a buffer still owes its reader
         self.d_ready = 0              # D holds what chunk d_ready's updates need
         self.d_done = -1              # last chunk whose every update of D has executed
-        self.scores_read = {1: -1, 2: -1}  # last block whose scores each warpgroup read
         self.acc = {1: None, 2: None}      # chunk of the last product into dv (1), dk (2)
         self.acc_read = {1: -1, 2: -1}     # last chunk each warpgroup wrote out
         self.multiplied, self.written = [], []
@@ -120,6 +124,9 @@ class Model:
         assert not stale, f"{who}: overwrites {res} while queued MMAs still need {stale}"
         self.ver[res] = version
 
+    def expect(self, res, v, who):
+        assert self.ver[res] == v, f"{who}: {res} holds {self.ver[res]}, wants {v}"
+
     def land(self, res, v):
         self.overwrite(res, v, f"copy into {res}")
 
@@ -155,23 +162,29 @@ class Model:
                 yield
 
     def mma_role(self):
+        # Per block k: dk += P2(k) Q(k) (+ V_c D^T at a chunk's first block),
+        # the next block's S2, dv += P1(k) dO(k) (+ K_c D), D += Q(k)^T dO(k),
+        # the next block's S1.  A stream's next scores follow its product, so
+        # the tensor pipe's order keeps them off P until P has been used.
         seq = list(self.blocks())
-        st = {"inter_gc": -1, "kv_pending": -1, "a": 0}
+        st = {"inter_gc": -1, "kv_pending": -1}
 
-        def scores(i):
+        def scores(t, i):
             def run():
-                for wg in (1, 2):
-                    assert self.scores_read[wg] >= i - 1, (
-                        f"S({i}) lands before warpgroup {wg} read S({i - 1})")
-                self.ver["S"] = i
+                assert self.sc_need[t] is None, (
+                    f"S{t + 1}({i}) lands on {self.sc_need[t]} before it was used")
+                self.ver[("S", t)] = ("A", i)
+                self.sc_need[t] = ("A", i)
             return run
 
-        def product(wg, gc, first):
+        def product(wg, gc, first, t=None):
             def run():
                 if first:
                     assert self.acc_read[wg] >= gc - 1, (
                         f"chunk {gc} starts accumulator {wg} before chunk {gc - 1} was read out")
                 self.acc[wg] = gc
+                if t is not None:
+                    self.sc_need[t] = None
             return run
 
         def update(gc, last):
@@ -181,60 +194,62 @@ class Model:
                     self.d_done = gc
             return run
 
-        def issue_s(x):
+        def issue_s(t, x):
             if x["blk"] == 0:
                 yield from self.wait("mma", self.kv_full, x["gc"])
             s = x["i"] % RING
             yield from self.wait("mma", self.ring_full[s], x["i"] // RING)
-            self.mma(f"S({x['i']})", [(("ring", s), x["i"]), ("kv", x["gc"])], scores(x["i"]))
-            self.commit(self.a_full)
-            if x["blk"] == x["nb"] - 1:
+            self.mma(f"S{t + 1}({x['i']})", [(("ring", s), x["i"]), ("kv", x["gc"])],
+                     scores(t, x["i"]))
+            self.commit(self.a_full[t])
+            # S1 of a chunk's last block is the K/V slot's last score reader
+            if t == 0 and x["blk"] == x["nb"] - 1:
                 if st["inter_gc"] >= x["gc"]:
                     self.commit(self.kv_empty)
                 else:
                     st["kv_pending"] = x["gc"]
 
-        def score_ahead(c_i, must):
-            while st["a"] < len(seq) and st["a"] <= c_i + 1:
-                x = seq[st["a"]]
-                if x["blk"] == 0 and st["inter_gc"] < x["gc"] - 1 and not (must and x["i"] == c_i):
-                    break
-                if x["i"] > 0:
-                    yield from self.wait("mma", self.s_read, x["i"] - 1)
-                yield from issue_s(x)
-                st["a"] += 1
-
-        yield from score_ahead(0, True)
-        for c in seq:
+        if seq:
+            yield from issue_s(1, seq[0])
+            yield from issue_s(0, seq[0])
+        for idx, c in enumerate(seq):
             k, gc, s = c["i"], c["gc"], c["i"] % RING
-            if st["a"] == k:
-                yield from score_ahead(k, True)
+            nxt = seq[idx + 1] if idx + 1 < len(seq) else None
             first, last = c["blk"] == 0, c["blk"] == c["nb"] - 1
-            yield from self.wait("mma", self.p_full, k)
+            yield from self.wait("mma", self.p_full[1], k)
             if first and gc >= 1:
                 yield from self.wait("mma", self.o_empty[1], gc - 1)
-            self.mma(f"dk+=P2Q({k})", [(("ring", s), k), ("P2", k)], product(2, gc, first))
+            self.mma(f"dk+=P2Q({k})", [(("ring", s), k), (("S", 1), ("P", k))],
+                     product(2, gc, first, 1))
             if first:
                 yield from self.wait("mma", self.sb_full, gc)
                 self.mma(f"dk+=VD^T({gc})", [("kv", gc), ("sS", gc)], product(2, gc, False))
-                if gc >= 1:
-                    yield from self.wait("mma", self.o_empty[0], gc - 1)
-            self.mma(f"dv+=P1dO({k})", [(("ring", s), k), ("P1", k)], product(1, gc, first))
+            # a next chunk's scores wait for the K/V slot, whose release needs
+            # this chunk's K_c D issued: at a chunk boundary both go last
+            if nxt and nxt["blk"] != 0:
+                yield from issue_s(1, nxt)
+            yield from self.wait("mma", self.p_full[0], k)
+            if first and gc >= 1:
+                yield from self.wait("mma", self.o_empty[0], gc - 1)
+            self.mma(f"dv+=P1dO({k})", [(("ring", s), k), (("S", 0), ("P", k))],
+                     product(1, gc, first, 0))
             if first:
                 self.mma(f"dv+=KD({gc})", [("kv", gc), ("sS", gc)], product(1, gc, False))
                 st["inter_gc"] = gc
                 if st["kv_pending"] == gc:
                     self.commit(self.kv_empty)
                     st["kv_pending"] = -1
-            self.commit(self.p_free)
             self.mma(f"D+=QdO({k})", [(("ring", s), k)], update(gc, last))
             self.commit(self.ring_empty[s])
             if last:
                 self.commit(self.o_full)
                 self.commit(self.s_full)
             self.multiplied.append((c["bg"], c["cs"], c["blk"]))
+            if nxt:
+                if nxt["blk"] == 0:
+                    yield from issue_s(1, nxt)
+                yield from issue_s(0, nxt)
             yield
-            yield from score_ahead(k + 1, False)
 
     def warpgroup(self, wg):
         role = f"wg{wg}"
@@ -259,16 +274,14 @@ class Model:
 
         if wg == 1:
             state_ready(0)
+        t = wg - 1
         for c in self.blocks():
             k = c["i"]
-            yield from self.wait(role, self.a_full, k)
-            assert self.ver["S"] == k, f"{role}: scores of block {k} replaced by {self.ver['S']}"
-            self.scores_read[wg] = k
-            self.s_read.arrive()
-            if k >= 1:
-                yield from self.wait(role, self.p_free, k - 1)
-            self.overwrite(f"P{wg}", k, role)
-            self.p_full.arrive()
+            yield from self.wait(role, self.a_full[t], k)
+            self.expect(("S", t), ("A", k), f"{role}: mask({k})")
+            self.overwrite(("S", t), ("P", k), role)  # P over its scores
+            self.sc_need[t] = ("P", k)
+            self.p_full[t].arrive()
             yield
             if c["blk"] == 0 and prev is not None:
                 if wg == 1:
