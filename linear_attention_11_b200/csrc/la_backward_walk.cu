@@ -304,16 +304,19 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per block k: dk += P2(k) Q(k) (a chunk's first block starts dk, then
-    // V_c D^T), the next block's S2, dv += P1(k) dO(k) (then K_c D), D += Q^T
-    // dO, the next block's S1.  Each stream's next scores come after the
-    // product that reads its P (the tensor pipe runs in issue order), and
-    // one stream's mask overlaps the other's MMAs.  K_c and V_c sit in one
-    // slot, released once the chunk's last S1 and its K_c D are issued; a
-    // next chunk's scores therefore go at the end of the block.
+    // Per block k: dv += P1(k) dO(k) (a chunk's first block starts dv once it
+    // has been read out), the next block's S1, dk += P2(k) Q(k), the next
+    // block's S2, at a chunk's first block K_c D and V_c D^T, then D += Q^T dO.
+    // Each stream's next scores come after the product that reads its P (the
+    // tensor pipe runs in issue order), and each mask has the other stream's
+    // product and scores and D's update to run under it.  The bf16 copy of D
+    // is waited for only before K_c D; D's first update of a chunk follows it
+    // (the conversion reads D).  K_c and V_c sit in one slot, released once
+    // the chunk's last S2 and its K_c D, V_c D^T are issued; a next chunk's
+    // scores therefore go at the end of the block.
     if (elect_one()) {
       int inter_gc = -1;    // last chunk whose K_c D, V_c D^T are issued
-      int kv_pending = -1;  // chunk whose last S1 is issued before its K_c D
+      int kv_pending = -1;  // chunk whose last S2 is issued before its K_c D
       auto issue_s = [&](int t, const Cursor& x) -> bool {
         if (x.blk == 0 && !mbar_wait(kv_full, x.gc & 1, p.status, abort_flag)) return false;
         const int s = x.i % kRing;
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(320, 1)
                  smem_desc_sw128(blk + ch * kBlkHalf + koff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
         mma_commit(&a_full[t]);
-        if (t == 0 && x.blk == x.nb - 1) {  // the chunk's last score read of K_c, V_c
+        if (t == 1 && x.blk == x.nb - 1) {  // the chunk's last score read of K_c, V_c
           if (inter_gc >= x.gc)
             mma_commit(kv_empty);
           else
@@ -340,37 +343,15 @@ __global__ void __launch_bounds__(320, 1)
       };
       Cursor c;
       cursor_init(p, c);
-      bool ok = !c.valid || (issue_s(1, c) && issue_s(0, c));
+      bool ok = !c.valid || (issue_s(0, c) && issue_s(1, c));
       while (ok && c.valid) {
         Cursor nx = c;
         cursor_next(p, nx);
         const int k = c.i, s = k % kRing;
         const bool first = c.blk == 0, last = c.blk == c.nb - 1;
+        const bool nx_same = nx.valid && nx.blk != 0;  // the next block is in this chunk
         const uint32_t qa = sQ(s), doa = sDO(s);
-        // dk += P2 Q (a chunk's first block starts dk once it has been read
-        // out), then V_c D^T
-        if (!mbar_wait(&p_full[1], k & 1, p.status, abort_flag)) break;
-        if (first && c.gc >= 1 && !mbar_wait(&o_empty[1], (c.gc - 1) & 1, p.status, abort_flag))
-          break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kKeyBlk / 16; ++kk)
-          mma_ts(tmem + kColDk, tmem + kColS2 + kk * 8,
-                 smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024), IDESC_PV,
-                 (first && kk == 0) ? 0u : 1u);
-        if (first) {
-          if (!mbar_wait(sb_full, c.gc & 1, p.status, abort_flag)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (uint32_t)((kk & 3) * 32);
-            const uint32_t ch = (uint32_t)(kk >> 2);
-            mma_ss(tmem + kColDk, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
-                   smem_desc_sw128(sS + ch * kHalf + koff, 16, 1024), IDESC_VDT, 1u);
-          }
-        }
-        if (nx.valid && nx.blk != 0 && !issue_s(1, nx)) break;
-        // dv += P1 dO, then K_c D
+        // dv += P1 dO
         if (!mbar_wait(&p_full[0], k & 1, p.status, abort_flag)) break;
         if (first && c.gc >= 1 && !mbar_wait(&o_empty[0], (c.gc - 1) & 1, p.status, abort_flag))
           break;
@@ -380,13 +361,34 @@ __global__ void __launch_bounds__(320, 1)
           mma_ts(tmem + kColDv, tmem + kColS1 + kk * 8,
                  smem_desc_sw128(doa + kk * 2048, kBlkHalf, 1024), IDESC_PV,
                  (first && kk == 0) ? 0u : 1u);
-        if (first) {
+        if (nx_same && !issue_s(0, nx)) break;
+        // dk += P2 Q
+        if (!mbar_wait(&p_full[1], k & 1, p.status, abort_flag)) break;
+        if (first && c.gc >= 1 && !mbar_wait(&o_empty[1], (c.gc - 1) & 1, p.status, abort_flag))
+          break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kKeyBlk / 16; ++kk)
+          mma_ts(tmem + kColDk, tmem + kColS2 + kk * 8,
+                 smem_desc_sw128(qa + kk * 2048, kBlkHalf, 1024), IDESC_PV,
+                 (first && kk == 0) ? 0u : 1u);
+        if (nx_same && !issue_s(1, nx)) break;
+        if (first) {  // the state's terms: dv += K_c D, dk += V_c D^T
+          if (!mbar_wait(sb_full, c.gc & 1, p.status, abort_flag)) break;
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t koff = (uint32_t)((kk & 3) * 32);
             const uint32_t ch = (uint32_t)(kk >> 2);
             mma_ss(tmem + kColDv, smem_desc_sw128(sK + ch * kHalf + koff, 16, 1024),
                    smem_desc_sw128(sS + kk * 2048, kHalf, 1024), IDESC_KD, 1u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (uint32_t)((kk & 3) * 32);
+            const uint32_t ch = (uint32_t)(kk >> 2);
+            mma_ss(tmem + kColDk, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
+                   smem_desc_sw128(sS + ch * kHalf + koff, 16, 1024), IDESC_VDT, 1u);
           }
           inter_gc = c.gc;
           if (kv_pending == c.gc) {
@@ -403,9 +405,8 @@ __global__ void __launch_bounds__(320, 1)
           mma_commit(o_full);
           mma_commit(s_full);
         }
-        if (nx.valid) {
-          if (nx.blk == 0 && !issue_s(1, nx)) break;
-          if (!issue_s(0, nx)) break;
+        if (nx.valid && !nx_same) {
+          if (!issue_s(0, nx) || !issue_s(1, nx)) break;
         }
         c = nx;
       }
@@ -581,16 +582,18 @@ __global__ void __launch_bounds__(320, 1)
     cursor_init(p, c);
     int prev_it = -1, prev_gc = -1, prev_bg = 0, prev_cs = 0;
     for (; c.valid && ok; cursor_next(p, c)) {
+      // the chunk before ended: its accumulator goes out first (the new
+      // chunk's first product waits for it), then this block's mask, then
+      // the state step (the bf16 copy is first used later in the block)
+      const bool boundary = c.blk == 0 && prev_gc >= 0;
+      if (boundary && !write_out(prev_gc, prev_bg, prev_cs)) { ok = false; break; }
       if (!mask_block(c)) { ok = false; break; }
-      // the chunk before ended: its state step and output, after this
-      // block's mask (which the next MMAs need first)
-      if (c.blk == 0 && prev_gc >= 0) {
+      if (boundary) {
         const bool item_end = c.it != prev_it;
         if (wg1 && !state_step(prev_gc, item_end, prev_it, item_end ? c.it : -1)) {
           ok = false;
           break;
         }
-        if (!write_out(prev_gc, prev_bg, prev_cs)) { ok = false; break; }
       }
       prev_it = c.it;
       prev_gc = c.gc;

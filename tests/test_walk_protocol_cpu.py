@@ -162,10 +162,12 @@ class Model:
                 yield
 
     def mma_role(self):
-        # Per block k: dk += P2(k) Q(k) (+ V_c D^T at a chunk's first block),
-        # the next block's S2, dv += P1(k) dO(k) (+ K_c D), D += Q(k)^T dO(k),
-        # the next block's S1.  A stream's next scores follow its product, so
-        # the tensor pipe's order keeps them off P until P has been used.
+        # Per block k: dv += P1(k) dO(k), the next block's S1, dk += P2(k) Q(k),
+        # the next block's S2, at a chunk's first block K_c D and V_c D^T, then
+        # D += Q(k)^T dO(k).  A stream's next scores follow its product, so the
+        # tensor pipe's order keeps them off P until P has been used, and each
+        # mask has the other stream's product and scores and D's update to run
+        # under it.
         seq = list(self.blocks())
         st = {"inter_gc": -1, "kv_pending": -1}
 
@@ -202,39 +204,44 @@ class Model:
             self.mma(f"S{t + 1}({x['i']})", [(("ring", s), x["i"]), ("kv", x["gc"])],
                      scores(t, x["i"]))
             self.commit(self.a_full[t])
-            # S1 of a chunk's last block is the K/V slot's last score reader
-            if t == 0 and x["blk"] == x["nb"] - 1:
+            # S2 of a chunk's last block is the K/V slot's last score reader
+            if t == 1 and x["blk"] == x["nb"] - 1:
                 if st["inter_gc"] >= x["gc"]:
                     self.commit(self.kv_empty)
                 else:
                     st["kv_pending"] = x["gc"]
 
         if seq:
-            yield from issue_s(1, seq[0])
             yield from issue_s(0, seq[0])
+            yield from issue_s(1, seq[0])
         for idx, c in enumerate(seq):
             k, gc, s = c["i"], c["gc"], c["i"] % RING
             nxt = seq[idx + 1] if idx + 1 < len(seq) else None
             first, last = c["blk"] == 0, c["blk"] == c["nb"] - 1
+            yield from self.wait("mma", self.p_full[0], k)
+            # (implied by P1 since warpgroup 1 reads dv out before this mask;
+            # the kernel keeps the direct wait as well)
+            if first and gc >= 1:
+                yield from self.wait("mma", self.o_empty[0], gc - 1)
+            self.mma(f"dv+=P1dO({k})", [(("ring", s), k), (("S", 0), ("P", k))],
+                     product(1, gc, first, 0))
+            # a next chunk's scores wait for the K/V slot, whose release needs
+            # this chunk's K_c D, V_c D^T issued: at a chunk boundary they go last
+            if nxt and nxt["blk"] != 0:
+                yield from issue_s(0, nxt)
             yield from self.wait("mma", self.p_full[1], k)
             if first and gc >= 1:
                 yield from self.wait("mma", self.o_empty[1], gc - 1)
             self.mma(f"dk+=P2Q({k})", [(("ring", s), k), (("S", 1), ("P", k))],
                      product(2, gc, first, 1))
-            if first:
-                yield from self.wait("mma", self.sb_full, gc)
-                self.mma(f"dk+=VD^T({gc})", [("kv", gc), ("sS", gc)], product(2, gc, False))
-            # a next chunk's scores wait for the K/V slot, whose release needs
-            # this chunk's K_c D issued: at a chunk boundary both go last
             if nxt and nxt["blk"] != 0:
                 yield from issue_s(1, nxt)
-            yield from self.wait("mma", self.p_full[0], k)
-            if first and gc >= 1:
-                yield from self.wait("mma", self.o_empty[0], gc - 1)
-            self.mma(f"dv+=P1dO({k})", [(("ring", s), k), (("S", 0), ("P", k))],
-                     product(1, gc, first, 0))
             if first:
+                # the bf16 copy of D for this chunk; D's first update of the
+                # chunk waits for it too (the conversion reads D)
+                yield from self.wait("mma", self.sb_full, gc)
                 self.mma(f"dv+=KD({gc})", [("kv", gc), ("sS", gc)], product(1, gc, False))
+                self.mma(f"dk+=VD^T({gc})", [("kv", gc), ("sS", gc)], product(2, gc, False))
                 st["inter_gc"] = gc
                 if st["kv_pending"] == gc:
                     self.commit(self.kv_empty)
@@ -245,10 +252,9 @@ class Model:
                 self.commit(self.o_full)
                 self.commit(self.s_full)
             self.multiplied.append((c["bg"], c["cs"], c["blk"]))
-            if nxt:
-                if nxt["blk"] == 0:
-                    yield from issue_s(1, nxt)
+            if nxt and nxt["blk"] == 0:
                 yield from issue_s(0, nxt)
+                yield from issue_s(1, nxt)
             yield
 
     def warpgroup(self, wg):
@@ -277,17 +283,21 @@ class Model:
         t = wg - 1
         for c in self.blocks():
             k = c["i"]
+            # at a chunk boundary the previous chunk's accumulator is read out
+            # first (the chunk's first product waits for it), the state
+            # converted after the mask (its first use comes later)
+            boundary = c["blk"] == 0 and prev is not None
+            if boundary:
+                yield from write_out(prev)
             yield from self.wait(role, self.a_full[t], k)
             self.expect(("S", t), ("A", k), f"{role}: mask({k})")
             self.overwrite(("S", t), ("P", k), role)  # P over its scores
             self.sc_need[t] = ("P", k)
             self.p_full[t].arrive()
             yield
-            if c["blk"] == 0 and prev is not None:
-                if wg == 1:
-                    yield from self.wait(role, self.s_full, prev["gc"])
-                    state_ready(c["gc"])
-                yield from write_out(prev)
+            if boundary and wg == 1:
+                yield from self.wait(role, self.s_full, prev["gc"])
+                state_ready(c["gc"])
             prev = c
         if prev is not None:
             if wg == 1:
@@ -395,3 +405,60 @@ def test_planner_spans_fit_the_chunks():
             for G in (1, 4, 16):
                 ns = _walk_spans(units, tiles, 148, G)
                 assert 1 <= ns <= tiles
+
+
+# Planted mistakes: each removes or weakens one wait, moves one issue, or
+# merges two barriers, as a plausible slip would, and must fail the model.
+MUTANTS = {
+    "dv without its P1": (
+        "            yield from self.wait(\"mma\", self.p_full[0], k)\n", ""),
+    "dk without its P2": (
+        "            yield from self.wait(\"mma\", self.p_full[1], k)\n", ""),
+    "mask without its scores": (
+        "            yield from self.wait(role, self.a_full[t], k)\n", ""),
+    "state terms before the bf16 copy of D": (
+        "                yield from self.wait(\"mma\", self.sb_full, gc)\n", ""),
+    "key block copied into a busy stage": (
+        "                yield from self.wait(\"ring\", self.ring_empty[s], x[\"i\"] // RING - 1)\n",
+        "                pass\n"),
+    "K/V copied into the busy slot": (
+        "                    yield from self.wait(\"kv\", self.kv_empty, gc - 1)\n",
+        "                    pass\n"),
+    "next S1 ahead of the dv that reads P1": (
+        "            self.mma(f\"dv+=P1dO({k})\", [((\"ring\", s), k), ((\"S\", 0), (\"P\", k))],\n"
+        "                     product(1, gc, first, 0))\n"
+        "            # a next chunk's scores wait for the K/V slot, whose release needs\n"
+        "            # this chunk's K_c D, V_c D^T issued: at a chunk boundary they go last\n"
+        "            if nxt and nxt[\"blk\"] != 0:\n"
+        "                yield from issue_s(0, nxt)\n",
+        "            if nxt and nxt[\"blk\"] != 0:\n"
+        "                yield from issue_s(0, nxt)\n"
+        "            self.mma(f\"dv+=P1dO({k})\", [((\"ring\", s), k), ((\"S\", 0), (\"P\", k))],\n"
+        "                     product(1, gc, first, 0))\n"),
+    "K/V released at the last S1 instead of the last S2": (
+        "            if t == 1 and x[\"blk\"] == x[\"nb\"] - 1:\n",
+        "            if t == 0 and x[\"blk\"] == x[\"nb\"] - 1:\n"),
+    "one p_full barrier for both streams": (
+        "        self.p_full = [mk(\"p_full1\", 1), mk(\"p_full2\", 1)]",
+        "        self.p_full = [mk(\"p_full\", 1)] * 2"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_walk_mistakes(name):
+    import inspect
+    import sys
+    old, new = MUTANTS[name]
+    src = inspect.getsource(sys.modules[__name__])
+    src = src[:src.index("\n# Planted mistakes")]
+    assert src.count(old) == 1, name
+    ns = {"__name__": f"walk_mutant_{abs(hash(name))}"}
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), ns)
+    caught = False
+    for shape in ns["SHAPES"]:
+        try:
+            ns["test_walk_protocol"](*shape)
+        except AssertionError:
+            caught = True
+            break
+    assert caught, f"planted mistake '{name}' passed the model"
