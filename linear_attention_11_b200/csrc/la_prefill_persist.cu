@@ -317,7 +317,8 @@ __global__ void __launch_bounds__(320, 1)
               mma_ss(tmem + ocol, da, db, IDESC_QS, kk > 0 ? 1u : 0u);
             }
             mma_commit(&q_empty[i % QST]);  // QK(i) and QS(i) were Q(i)'s readers
-            const bool early = NSC == 2 && !item_end;
+            // (not with staged states: their items are a tile or two long)
+            const bool early = NSC == 2 && !kStage && !item_end;
             if (early && !issue_qk(i + 1, gnext)) { ok = false; break; }
 #pragma unroll
             for (int ph = 0; ph < NPH && ok; ++ph) {  // O += P V (P from TMEM), half by half
@@ -541,7 +542,7 @@ __global__ void __launch_bounds__(320, 1)
             // tile's scores ahead of the update with two score buffers inside
             // an item); one call site each (two inlined copies of either spill
             // registers at T = 128)
-            const bool mask_first = NSC == 2 && !item_end;
+            const bool mask_first = NSC == 2 && !kStage && !item_end;
 #pragma unroll 1
             for (int ph = 0; ph < 2 && ok; ++ph) {
               const bool do_step = last_hs && (ph == (mask_first ? 1 : 0));

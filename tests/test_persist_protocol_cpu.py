@@ -224,7 +224,7 @@ class Model:
             nxt = gc + 1 if x["last_hs"] else gc
             # with two score buffers the next tile's scores go ahead of PV
             # (inside an item; at its end the state update goes first)
-            early = self.nsc == 2 and not x["item_end"]
+            early = self.nsc == 2 and not self.staged and not x["item_end"]
             if early:
                 yield from qk(i + 1, nxt)
             for h in range(self.halves):
@@ -310,7 +310,7 @@ class Model:
             # the MMA order decides which is ready first: with the next tile's
             # scores ahead of PV (two score buffers, inside an item) the mask
             # comes before the state step
-            mask_first = self.nsc == 2 and not x["item_end"]
+            mask_first = self.nsc == 2 and not self.staged and not x["item_end"]
             for ph in (0, 1):
                 do_step = x["last_hs"] and ph == (1 if mask_first else 0)
                 do_mask = x["has_next"] and ph == (0 if mask_first else 1)
@@ -463,7 +463,7 @@ MUTANTS = {
     "PV without p_full": (
         "                yield from self.wait(\"mma\", pf, i // self.nsc)\n", ""),
     "next scores ahead of PV with one score buffer": (
-        "            early = self.nsc == 2 and not x[\"item_end\"]\n",
+        "            early = self.nsc == 2 and not self.staged and not x[\"item_end\"]\n",
         "            early = not x[\"item_end\"]\n"),
     "one a_full barrier for two score buffers": (
         "        self.a_full = [mk(f\"a_full{b}\", 1) for b in range(self.nsc)]",
