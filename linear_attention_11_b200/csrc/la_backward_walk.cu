@@ -535,43 +535,36 @@ __global__ void __launch_bounds__(320, 1)
       return true;
     };
 
-    // this warpgroup's accumulator of chunk gcd (rows of chunk cs of group
-    // bg) -> bf16 rows in global memory, released once read out
-    auto write_out = [&](int gcd, int bg, int cs) -> bool {
+    // this warpgroup's accumulator of chunk gcd -> bf16 row r in registers;
+    // the accumulator is released as soon as it is read, before any store
+    auto read_out = [&](int gcd, uint32_t (&row_bf)[64]) -> bool {
       if (!warp_wait(o_full, gcd & 1, p.status, abort_flag)) return false;
       tc_fence_after();
-      const int64_t row = (int64_t)cs * kChunk + r;
-      const bool valid = row < p.N;
-      uint4* dst = reinterpret_cast<uint4*>(out_base + ((size_t)bg * p.N + (valid ? row : 0)) *
-                                                           kHeadDim);
-#pragma unroll 1
+#pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t x0[32], x1[32];
         tmem_ld32(tmem + lane_base + col_o + hh * 64, x0);
         tmem_ld32(tmem + lane_base + col_o + hh * 64 + 32, x1);
         tmem_wait_ld();
-        if (hh == 1) {
-          tc_fence_before();
-          mbar_arrive(my_empty);
-        }
-        if (valid) {
 #pragma unroll
-          for (int m = 0; m < 4; ++m)
-            dst[hh * 8 + m] = make_uint4(
-                pack_bf16x2(__uint_as_float(x0[8 * m]), __uint_as_float(x0[8 * m + 1])),
-                pack_bf16x2(__uint_as_float(x0[8 * m + 2]), __uint_as_float(x0[8 * m + 3])),
-                pack_bf16x2(__uint_as_float(x0[8 * m + 4]), __uint_as_float(x0[8 * m + 5])),
-                pack_bf16x2(__uint_as_float(x0[8 * m + 6]), __uint_as_float(x0[8 * m + 7])));
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            dst[hh * 8 + 4 + m] = make_uint4(
-                pack_bf16x2(__uint_as_float(x1[8 * m]), __uint_as_float(x1[8 * m + 1])),
-                pack_bf16x2(__uint_as_float(x1[8 * m + 2]), __uint_as_float(x1[8 * m + 3])),
-                pack_bf16x2(__uint_as_float(x1[8 * m + 4]), __uint_as_float(x1[8 * m + 5])),
-                pack_bf16x2(__uint_as_float(x1[8 * m + 6]), __uint_as_float(x1[8 * m + 7])));
+        for (int m = 0; m < 16; ++m) {
+          row_bf[hh * 32 + m] = pack_bf16x2(__uint_as_float(x0[2 * m]), __uint_as_float(x0[2 * m + 1]));
+          row_bf[hh * 32 + 16 + m] =
+              pack_bf16x2(__uint_as_float(x1[2 * m]), __uint_as_float(x1[2 * m + 1]));
         }
       }
+      tc_fence_before();
+      mbar_arrive(my_empty);
       return true;
+    };
+    // row r of chunk cs of group bg to global memory (rows past N dropped)
+    auto store_out = [&](int bg, int cs, const uint32_t (&row_bf)[64]) {
+      const int64_t row = (int64_t)cs * kChunk + r;
+      if (row >= p.N) return;
+      uint4* dst = reinterpret_cast<uint4*>(out_base + ((size_t)bg * p.N + row) * kHeadDim);
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        dst[m] = make_uint4(row_bf[4 * m], row_bf[4 * m + 1], row_bf[4 * m + 2], row_bf[4 * m + 3]);
     };
 
     if (wg1) {
@@ -581,12 +574,14 @@ __global__ void __launch_bounds__(320, 1)
     Cursor c;
     cursor_init(p, c);
     int prev_it = -1, prev_gc = -1, prev_bg = 0, prev_cs = 0;
+    uint32_t row_bf[64];
     for (; c.valid && ok; cursor_next(p, c)) {
-      // the chunk before ended: its accumulator goes out first (the new
+      // the chunk before ended: its accumulator is read out first (the new
       // chunk's first product waits for it), then this block's mask, then
-      // the state step (the bf16 copy is first used later in the block)
+      // the state step (the bf16 copy is first used later in the block), and
+      // only then the read-out rows go to global memory
       const bool boundary = c.blk == 0 && prev_gc >= 0;
-      if (boundary && !write_out(prev_gc, prev_bg, prev_cs)) { ok = false; break; }
+      if (boundary && !read_out(prev_gc, row_bf)) { ok = false; break; }
       if (!mask_block(c)) { ok = false; break; }
       if (boundary) {
         const bool item_end = c.it != prev_it;
@@ -594,6 +589,7 @@ __global__ void __launch_bounds__(320, 1)
           ok = false;
           break;
         }
+        store_out(prev_bg, prev_cs, row_bf);
       }
       prev_it = c.it;
       prev_gc = c.gc;
@@ -602,7 +598,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (ok && prev_gc >= 0) {
       if (wg1) ok = state_step(prev_gc, true, prev_it, -1);
-      if (ok) write_out(prev_gc, prev_bg, prev_cs);
+      if (ok && read_out(prev_gc, row_bf)) store_out(prev_bg, prev_cs, row_bf);
     }
   }
 
