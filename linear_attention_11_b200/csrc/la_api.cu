@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdint>
 #include <mutex>
 
 #include "la.h"
@@ -268,12 +269,24 @@ bool stage_states_pays(const PrefillGeometry& g) {
 
 int span_parts(const la_plan& plan, int units, int sms) {
   if (plan.nspan <= 1) return 1;
-  // the forward computes the states of the first nspan - 1 spans; cut each
-  // into parts until those CTAs cover the SMs, keeping two tiles per part
+  // the forward computes the states of the first nspan - 1 spans, one CTA
+  // per SM at a time; cut each span into the number of parts (at least two
+  // tiles each) whose CTAs finish soonest: waves x (tiles per part + a fixed
+  // cost of about three tiles per CTA: pipeline fill, state write-out), the
+  // fewest parts on a tie
   const int64_t ctas = (int64_t)units * (plan.nspan - 1);
-  int64_t parts = (sms + ctas - 1) / ctas;
-  parts = std::min<int64_t>(parts, std::max<int64_t>(1, plan.tiles_total / (2 * plan.nspan)));
-  return (int)std::max<int64_t>(1, std::min<int64_t>(parts, 64));
+  const int64_t span_tiles = (plan.tiles_total + plan.nspan - 1) / plan.nspan;
+  const int64_t max_parts = std::max<int64_t>(1, std::min<int64_t>(64, span_tiles / 2));
+  int64_t best = 1, best_cost = INT64_MAX;
+  for (int64_t parts = 1; parts <= max_parts; ++parts) {
+    const int64_t waves = (ctas * parts + sms - 1) / sms;
+    const int64_t cost = waves * ((span_tiles + parts - 1) / parts + 3);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = parts;
+    }
+  }
+  return (int)best;
 }
 
 size_t forward_workspace_bytes(const la_plan& plan) {

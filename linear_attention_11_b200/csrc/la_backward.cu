@@ -94,7 +94,7 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
     return LA_ERR_CUDA;
   const int tiles_w = (int)((N + 127) / 128);
   const int nspan_w = walk_spans(B * Hkv, tiles_w, sms, G);
-  const size_t sq_bytes = round((size_t)B * Hkv * dd * 4);
+  const size_t sq_bytes = S0 ? round((size_t)B * Hkv * dd * 4) : 0;
   const size_t wsq_bytes = forward_workspace_bytes(plan_q);
   const size_t wsq = round(wsq_bytes);
   const size_t wsh = nspan_w > 1 ? round((size_t)B * Hq * nspan_w * dd * 4) : 0;
@@ -105,7 +105,7 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
   if (cudaMallocAsync(reinterpret_cast<void**>(&pool), total, s) != cudaSuccess) return LA_ERR_CUDA;
   char* cur = pool;
   auto take = [&](size_t n) { char* p = cur; cur += n; return p; };
-  float* S_q = reinterpret_cast<float*>(take(sq_bytes));
+  float* S_q = S0 ? reinterpret_cast<float*>(take(sq_bytes)) : nullptr;
   void* ws_q = take(wsq);
   float* ws_h = wsh ? reinterpret_cast<float*>(take(wsh)) : nullptr;
   float* ent = ent_bytes ? reinterpret_cast<float*>(take(ent_bytes)) : nullptr;
@@ -114,8 +114,8 @@ LA_EXPORT la_status la_backward(const la_bf16* q, const la_bf16* k, const la_bf1
     if (e != cudaSuccess && st == LA_OK) st = LA_ERR_CUDA;
   };
 
-  // ---- dq: the forward pass on (dO, V, K) from S0^T
-  cu(place_states(S0, S_q, B, Hkv, 1, d, 1, s));
+  // ---- dq: the forward pass on (dO, V, K) from S0^T (from zero without S0)
+  if (S0) cu(place_states(S0, S_q, B, Hkv, 1, d, 1, s));
   if (st == LA_OK)
     st = forward_dispatch(dO, v, k, dq, S_q, B, Hq, Hkv, N, plan_q, ws_q, wsq_bytes, s, false);
 
