@@ -347,7 +347,7 @@ la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v,
   const bool final_state = S != nullptr && final_out;
   cudaError_t e = launch_span_states(g, maps.k, maps.v, ws, status, stream, !final_state, parts);
   if (e == cudaSuccess)
-    e = launch_state_scan(ws, S, B * Hkv, nsub_spans, kHeadDim, stream, 0,
+    e = launch_state_scan(ws, S, B * Hkv, nsub_spans, kHeadDim, stream,
                           final_state ? nsub_spans : nsub_spans - parts);
   if (e == cudaSuccess)
     e = launch_prefill_persist(g, maps, ws, nullptr, status, sms, stream, true, false, parts);

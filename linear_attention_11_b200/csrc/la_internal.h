@@ -98,12 +98,12 @@ la_status forward_dispatch(const la_bf16* q, const la_bf16* k, const la_bf16* v,
 cudaError_t launch_prefill_fused(const PrefillGeometry& g, const PrefillMaps& maps, float* S,
                                  void* workspace, unsigned* status, int num_sms, int lookahead,
                                  cudaStream_t stream);
-// reverse: ws[j] <- S0 + sum_{i>j} ws[i] (the state entering span j of a
-// backwards walk); S receives S0 + sum_i ws[i] either way.  nread < nspan
-// (forward only): entries from nread on are not read, ws[nread] receives its
-// entering state and S is only read (S0); nread < 0 means nspan.
+// ws[j] <- S0 + sum_{i<j} ws[i] (the state entering entry j; S0 = *S or
+// zero), and S receives S0 + sum_i ws[i].  nread < nspan: entries from nread
+// on are not read, ws[nread] receives its entering state and S is only read
+// (S0); nread < 0 means nspan.
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
-                              cudaStream_t stream, int reverse = 0, int nread = -1);
+                              cudaStream_t stream, int nread = -1);
 // S = S0 (nullable) + sum_{i < seg} states[i * per_seg_floats ...] (float4-wise).
 cudaError_t launch_state_prefix(const float* states, const float* S0, float* S, int seg,
                                 size_t per_seg_floats, cudaStream_t stream);

@@ -6,10 +6,14 @@
 // kv_sum over the whole sequence).  When the chunk loop writes the final state
 // itself, the last span's K^T V is never computed (nread < nspan) and only the
 // entering states are written.  Elementwise fp32 adds, HBM/L2-bound: one
-// thread owns one float4 of the d x d matrix of one unit and walks the spans
-// in order, loading eight spans ahead to keep loads in flight.  Launched as a
-// programmatic dependent of the span-state kernel: it lets the chunk-loop
-// kernel start its copies, then waits for the span states.
+// thread owns two float4 of the d x d matrix of one unit and walks the spans
+// in order, eight spans at a time with all their loads issued before the
+// stores, so a short scan costs one round trip to memory, not one per span.
+// Two float4 per thread keep the grid small (at most a few 256-thread CTAs
+// per SM), so the chunk-loop kernel, launched behind it, finds room to start
+// its copies early.  Launched as a programmatic dependent of the span-state
+// kernel: it lets the chunk-loop kernel start its copies, then waits for the
+// span states.
 #include <cuda_runtime.h>
 
 #include "la_internal.h"
@@ -22,58 +26,62 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
+constexpr int kScanVec = 1;  // float4 per thread
+constexpr int kScanBatch = 4;  // spans whose loads are issued together
+
 __global__ void __launch_bounds__(256)
     state_scan_kernel(float4* __restrict__ ws, float4* __restrict__ S, int nspan, int n4,
-                      int blocks_per_unit, int reverse, int nread) {
+                      int blocks_per_unit, int nread) {
   griddep_launch_dependents();  // the chunk-loop kernel may start its copies
   griddep_wait();               // the span states are complete
   const size_t unit = blockIdx.x / blocks_per_unit;
-  const int p = (blockIdx.x % blocks_per_unit) * blockDim.x + threadIdx.x;
-  if (p >= n4) return;
-  float4* w = ws + unit * (size_t)nspan * n4 + p;
-  float4 carry = S ? S[unit * n4 + p] : make_float4(0.f, 0.f, 0.f, 0.f);
-  if (reverse) {  // spans from the last to the first
-    for (int j = nspan - 1; j >= 0; --j) {
-      const float4 x = w[(size_t)j * n4];
-      w[(size_t)j * n4] = carry;
-      carry = add4(carry, x);
-    }
-    if (S) S[unit * n4 + p] = carry;
-    return;
+  const int p0 = (blockIdx.x % blocks_per_unit) * (blockDim.x * kScanVec) + threadIdx.x;
+  float4* w = ws + unit * (size_t)nspan * n4;
+  int pos[kScanVec];
+  bool in[kScanVec];
+  float4 carry[kScanVec];
+#pragma unroll
+  for (int e = 0; e < kScanVec; ++e) {
+    pos[e] = p0 + e * (int)blockDim.x;
+    in[e] = pos[e] < n4;
+    carry[e] = (S && in[e]) ? S[unit * n4 + pos[e]] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   // nread < nspan: entries from nread on were not computed (they only feed
   // the final state); the entering state of entry nread is written, no final
-  int j = 0;
-  for (; j + 8 <= nread; j += 8) {
-    float4 x[8];
+  for (int j = 0; j < nread; j += kScanBatch) {
+    float4 x[kScanVec][kScanBatch];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = w[(size_t)(j + u) * n4];
+    for (int e = 0; e < kScanVec; ++e)
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      w[(size_t)(j + u) * n4] = carry;
-      carry = add4(carry, x[u]);
-    }
+      for (int u = 0; u < kScanBatch; ++u)
+        if (in[e] && j + u < nread) x[e][u] = w[(size_t)(j + u) * n4 + pos[e]];
+#pragma unroll
+    for (int e = 0; e < kScanVec; ++e)
+#pragma unroll
+      for (int u = 0; u < kScanBatch; ++u)
+        if (in[e] && j + u < nread) {
+          w[(size_t)(j + u) * n4 + pos[e]] = carry[e];
+          carry[e] = add4(carry[e], x[e][u]);
+        }
   }
-  for (; j < nread; ++j) {
-    const float4 x = w[(size_t)j * n4];
-    w[(size_t)j * n4] = carry;
-    carry = add4(carry, x);
+#pragma unroll
+  for (int e = 0; e < kScanVec; ++e) {
+    if (!in[e]) continue;
+    if (nread < nspan)
+      w[(size_t)nread * n4 + pos[e]] = carry[e];
+    else if (S)
+      S[unit * n4 + pos[e]] = carry[e];
   }
-  if (nread < nspan) {
-    w[(size_t)nread * n4] = carry;
-    return;
-  }
-  if (S) S[unit * n4 + p] = carry;
 }
 
 }  // namespace
 
 cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
-                              cudaStream_t stream, int reverse, int nread) {
+                              cudaStream_t stream, int nread) {
   if (nread < 0) nread = nspan;
-  if (nread < 1 || nread > nspan || (reverse && nread != nspan)) return cudaErrorInvalidValue;
+  if (nread < 1 || nread > nspan) return cudaErrorInvalidValue;
   const int n4 = d * d / 4;
-  const int bpu = (n4 + 255) / 256;
+  const int bpu = (n4 + 256 * kScanVec - 1) / (256 * kScanVec);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(units * bpu));
   cfg.blockDim = dim3(256);
@@ -85,7 +93,7 @@ cudaError_t launch_state_scan(float* ws, float* S, int units, int nspan, int d,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, state_scan_kernel, reinterpret_cast<float4*>(ws),
-                            reinterpret_cast<float4*>(S), nspan, n4, bpu, reverse, nread);
+                            reinterpret_cast<float4*>(S), nspan, n4, bpu, nread);
 }
 
 namespace {
