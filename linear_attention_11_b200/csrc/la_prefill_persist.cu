@@ -61,14 +61,14 @@ struct PersistParams {
 // loaded an item ahead by a third copy lane; without it the math warps read
 // and write them row by row.  kDedO: a dedicated output staging tile (else
 // the output goes through the Q slot).
-template <int T, int QST, int KVST, bool kDedO, bool kStage>
+template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kHalfKV>
 __global__ void __launch_bounds__(320, 1)
     prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
                            const __grid_constant__ CUtensorMap map_k,
                            const __grid_constant__ CUtensorMap map_v,
                            const __grid_constant__ CUtensorMap map_o,
                            const __grid_constant__ CUtensorMap map_s, const PersistParams p) {
-  using L = MainLayout<T, QST, KVST, kDedO, kStage>;
+  using L = MainLayout<T, QST, KVST, kDedO, kStage, kHalfKV>;
   constexpr int HPT = kTileRows / T;
   constexpr bool kDedicatedO = L::kDedicatedO;
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, T, 0, 0);
@@ -108,8 +108,18 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t sSt = base + L::kStOff;
   const bool staged = kStage && p.ws != nullptr;
   auto sQ = [&](int i) { return base + (uint32_t)((i % QST) * kQBytes); };
-  auto sK = [&](int c) { return base + (uint32_t)(L::kKVOff + (c % KVST) * L::kKVBytes); };
-  auto sV = [&](int c) { return sK(c) + (uint32_t)L::kKBytes; };
+  // K/V ring: slot c % KVST holds chunk step c's K and V tiles; with
+  // kHalfKV the tiles take slots apart, copy 2c (K) and 2c + 1 (V) of the
+  // ring, so a K tile can be refilled while the V tile of its step is in use
+  auto kcopy = [&](int c) { return kHalfKV ? 2 * c : c; };
+  auto vcopy = [&](int c) { return kHalfKV ? 2 * c + 1 : c; };
+  auto sK = [&](int c) {
+    return base + (uint32_t)(L::kKVOff + (kcopy(c) % KVST) * L::kKVBytes);
+  };
+  auto sV = [&](int c) {
+    return kHalfKV ? base + (uint32_t)(L::kKVOff + (vcopy(c) % KVST) * L::kKVBytes)
+                   : sK(c) + (uint32_t)L::kKBytes;
+  };
   auto sO = [&](int i) { return kDedicatedO ? base + (uint32_t)L::kOOff : sQ(i); };
   // TMEM column of tile i's score buffer (its P over the first T / 2 columns)
   auto scol = [&](int i) { return (uint32_t)(256 + (i % NSC) * T); };
@@ -205,30 +215,39 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t pol_kv = policy_evict_first();
       int gc = 0;
       bool go = true;
+      int u = 0;  // copies into the ring so far
       for (int it = blockIdx.x; it < p.items && go; it += stride) {
         int bg, tb, te;
         span_of(it, bg, tb, te);
         const int nx = next_item(it);
         if (!staged && p.ws && nx >= 0)  // next item's entering state, read at this item's end
           prefetch_l2_bulk(p.ws + (size_t)nx * p.ws_stride * kDD, (uint32_t)(kDD * sizeof(float)));
-        for (int n = 0; n < te - tb; ++n, ++gc) {
+        for (int n = 0; n < te - tb && go; ++n, ++gc) {
           const int cs = tb + n;
-          const int s = gc % KVST;
-          if (gc >= KVST && !mbar_wait(&kv_empty[s], ((gc / KVST) - 1) & 1, p.status, abort_flag)) {
-            go = false;
-            break;
+#pragma unroll
+          for (int part = 0; part < (kHalfKV ? 2 : 1); ++part, ++u) {
+            const int s = u % KVST;
+            if (u >= KVST &&
+                !mbar_wait(&kv_empty[s], ((u / KVST) - 1) & 1, p.status, abort_flag)) {
+              go = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&kv_full[s], L::kKVBytes);
+            if (!kHalfKV || part == 0) {
+              uint8_t* k_dst = sm + (sK(gc) - base);
+              tma_load_3d(k_dst, &map_k, &kv_full[s], 0, cs * T, bg, pol_kv);
+              tma_load_3d(k_dst + T * 128, &map_k, &kv_full[s], 64, cs * T, bg, pol_kv);
+            }
+            if (!kHalfKV || part == 1) {
+              uint8_t* v_dst = sm + (sV(gc) - base);
+              tma_load_3d(v_dst, &map_v, &kv_full[s], 0, cs * T, bg, pol_kv);
+              tma_load_3d(v_dst + T * 128, &map_v, &kv_full[s], 64, cs * T, bg, pol_kv);
+            }
           }
-          mbar_arrive_expect_tx(&kv_full[s], L::kKVBytes);
-          uint8_t* k_dst = sm + (sK(gc) - base);
-          uint8_t* v_dst = sm + (sV(gc) - base);
-          tma_load_3d(k_dst, &map_k, &kv_full[s], 0, cs * T, bg, pol_kv);
-          tma_load_3d(k_dst + T * 128, &map_k, &kv_full[s], 64, cs * T, bg, pol_kv);
-          tma_load_3d(v_dst, &map_v, &kv_full[s], 0, cs * T, bg, pol_kv);
-          tma_load_3d(v_dst + T * 128, &map_v, &kv_full[s], 64, cs * T, bg, pol_kv);
         }
       }
       if (*abort_flag) {
-        for (int k = (gc > KVST ? gc - KVST : 0); k < gc; ++k)
+        for (int k = (u > KVST ? u - KVST : 0); k < u; ++k)
           mbar_wait_drain(&kv_full[k % KVST], (k / KVST) & 1);
       }
     } else if (lane == 2 && staged) {
@@ -262,9 +281,18 @@ __global__ void __launch_bounds__(320, 1)
     // QS(i + 1).  At an item's end the update goes first, so the state
     // hand-over to the next item does not wait for that item's first tiles.
     if (elect_one()) {
+      // wait for the K (or K/V) tile of chunk step c, or its V tile
+      auto wait_k = [&](int c) {
+        const int u = kcopy(c);
+        return mbar_wait(&kv_full[u % KVST], (u / KVST) & 1, p.status, abort_flag);
+      };
+      auto wait_v = [&](int c) {
+        const int u = vcopy(c);
+        return mbar_wait(&kv_full[u % KVST], (u / KVST) & 1, p.status, abort_flag);
+      };
       auto issue_qk = [&](int i, int gci) -> bool {
         if (!mbar_wait(&q_full[i % QST], (i / QST) & 1, p.status, abort_flag)) return false;
-        if (!mbar_wait(&kv_full[gci % KVST], (gci / KVST) & 1, p.status, abort_flag)) return false;
+        if (!wait_k(gci)) return false;
         tc_fence_after();
         const uint32_t q_addr = sQ(i), k_addr = sK(gci);
 #pragma unroll
@@ -277,7 +305,9 @@ __global__ void __launch_bounds__(320, 1)
         mma_commit(&a_full[i % NSC]);
         return true;
       };
-      auto issue_kv = [&](int gci) {
+      auto issue_kv = [&](int gci) -> bool {
+        if (kHalfKV && !wait_v(gci)) return false;
+        tc_fence_after();
         const uint32_t k_addr = sK(gci), v_addr = sV(gci);
 #pragma unroll
         for (int kk = 0; kk < T / 16; ++kk) {  // S += K^T V (both MN-major)
@@ -286,7 +316,10 @@ __global__ void __launch_bounds__(320, 1)
           mma_ss(tmem + kColS, da, db, IDESC_KV, 1u);
         }
         mma_commit(s_full);
-        mma_commit(&kv_empty[gci % KVST]);
+        // the K tile's last reader (with kHalfKV; else the K/V slot's, as the
+        // update follows the step's last P V)
+        mma_commit(&kv_empty[kcopy(gci) % KVST]);
+        return true;
       };
       int i = 0, gc = 0;
       bool ok = issue_qk(0, 0);
@@ -320,6 +353,10 @@ __global__ void __launch_bounds__(320, 1)
             // (not with staged states: their items are a tile or two long)
             const bool early = NSC == 2 && !kStage && !item_end;
             if (early && !issue_qk(i + 1, gnext)) { ok = false; break; }
+            // with K and V apart the step's update goes before its last P V,
+            // which frees the K slot (its last reader) a tile earlier
+            if (kHalfKV && last_hs && !issue_kv(gc)) { ok = false; break; }
+            if (kHalfKV && !wait_v(gc)) { ok = false; break; }
 #pragma unroll
             for (int ph = 0; ph < NPH && ok; ++ph) {  // O += P V (P from TMEM), half by half
               uint64_t* pf = NPH == 2 ? &p_full[ph] : &p_full[i % NSC];
@@ -336,7 +373,8 @@ __global__ void __launch_bounds__(320, 1)
             }
             if (!ok) break;
             mma_commit(&o_full[ob]);
-            if (last_hs) issue_kv(gc);
+            if (kHalfKV && last_hs) mma_commit(&kv_empty[vcopy(gc) % KVST]);  // V's last reader
+            if (!kHalfKV && last_hs && !issue_kv(gc)) { ok = false; break; }
             if (!early && has_next && !issue_qk(i + 1, gnext)) { ok = false; break; }
             if (last_hs) ++gc;
             ++i;
@@ -656,12 +694,13 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int T, int QST, int KVST, bool kDedO, bool kStage>
+template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kHalfKV = false>
 cudaError_t launch_persist(dim3 grid, cudaStream_t stream, const PrefillMaps& maps,
                            const CUtensorMap& map_s, const PersistParams& p, bool dependent) {
-  using L = MainLayout<T, QST, KVST, kDedO, kStage>;
+  using L = MainLayout<T, QST, KVST, kDedO, kStage, kHalfKV>;
   static_assert(L::kBytes <= 232448, "shared memory");
-  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage>;
+  static_assert(!kHalfKV || KVST >= 3, "K and V tiles apart need three slots");
+  auto kernel = prefill_persist_kernel<T, QST, KVST, kDedO, kStage, kHalfKV>;
   cudaError_t e = set_smem(kernel, L::kBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -700,6 +739,11 @@ cudaError_t launch_prefill_persist(const PrefillGeometry& g, const PrefillMaps& 
     return launch_persist<64, 2, 2, false, true>(grid, stream, maps, map_s, p, dependent);
   }
   if (g.tile == 64) return launch_persist<64, 3, 2, true, false>(grid, stream, maps, maps.q, p, dependent);
+  // 128-token tiles: with several tiles per chunk step (grouped heads), K and
+  // V apart in a three-slot ring, which leaves room for a third Q slot; with
+  // one tile per step, K/V tiles together in two slots
+  if (nsub > 1)
+    return launch_persist<128, 3, 3, false, false, true>(grid, stream, maps, maps.q, p, dependent);
   return launch_persist<128, 2, 2, false, false>(grid, stream, maps, maps.q, p, dependent);
 }
 

@@ -83,12 +83,15 @@ __device__ __forceinline__ void store_row16_sw128(uint32_t base, int r, int q,
 // With kStage (persistent kernel, one span per sequence) a 64 KB fp32 state
 // tile follows, through which entering states arrive and final states leave
 // by bulk tensor copies.
-template <int T, int QST, int KVST, bool DedicatedO = (T == 64), bool Stage = false>
+template <int T, int QST, int KVST, bool DedicatedO = (T == 64), bool Stage = false,
+          bool HalfKV = false>
 struct MainLayout {
   static constexpr bool kDedicatedO = DedicatedO;
   static constexpr bool kStage = Stage;
   static constexpr int kKBytes = T * kHeadDim * 2;
-  static constexpr int kKVBytes = 2 * kKBytes;
+  // bytes per K/V slot: a K and a V tile, or one of them (HalfKV: K and V
+  // tiles take separate slots of one ring)
+  static constexpr int kKVBytes = HalfKV ? kKBytes : 2 * kKBytes;
   static constexpr int kKVOff = QST * kQBytes;
   static constexpr int kSOff = kKVOff + KVST * kKVBytes;
   static constexpr int kOOff = kSOff + kSBytes;

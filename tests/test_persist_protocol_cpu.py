@@ -1,8 +1,11 @@
 """The synchronisation of the prefill's persistent chunk-loop kernel
 (prefill_persist_kernel in linear_attention_11_b200/csrc/la_prefill_persist.cu),
-modelled on the CPU, for the three forward configurations the launcher
+modelled on the CPU, for the four forward configurations the launcher
 instantiates: 64-token tiles with a dedicated output tile, 64-token tiles with
-staged states (output through the Q slot), and 128-token tiles.
+staged states (output through the Q slot), 128-token tiles with one tile per
+chunk step (K and V tiles together in two slots), and 128-token tiles with
+several (K and V tiles apart in a three-slot ring, three Q slots, the state
+update ahead of the step's last P V).
 
 Each role of one CTA (Q copies, K/V copies, staged-state copies, MMA issue,
 the mask warpgroup, the output warpgroup; both warpgroups convert the state)
@@ -30,10 +33,13 @@ from test_walk_protocol_cpu import Barrier
 
 class Model:
     def __init__(self, T, QST, KVST, out, staged, G, units, nspan, tiles, grid, cta, s_out,
-                 seed):
+                 seed, halfkv=False):
         # out: "dedicated" (output tile of its own), "qslot" (output staged in
         # the tile's Q slot), "direct" (registers to global memory, no staging)
         self.T, self.QST, self.KVST, self.out, self.staged = T, QST, KVST, out, staged
+        # halfkv: K of chunk step c is copy 2c of the K/V ring, V copy 2c + 1
+        # (else one copy c holds both)
+        self.halfkv = halfkv
         self.dedo = out == "dedicated"
         self.nsub = G // (128 // T)
         self.nspan, self.tiles, self.items = nspan, tiles, units * nspan
@@ -158,15 +164,31 @@ class Model:
             self.copies.append((self.q_full[s], ("q", s), ("Q", i)))
             yield
 
+    def kcopy(self, gc):
+        return 2 * gc if self.halfkv else gc
+
+    def vcopy(self, gc):
+        return 2 * gc + 1 if self.halfkv else gc
+
+    def kver(self, gc):
+        return ("K", gc) if self.halfkv else gc
+
+    def vver(self, gc):
+        return ("V", gc) if self.halfkv else gc
+
     def kv_lane(self):
+        u = 0
         for x in self.steps():
             if not x["last_hs"]:
                 continue
-            gc, s = x["gc"], x["gc"] % self.KVST
-            if gc >= self.KVST:
-                yield from self.wait("kv", self.kv_empty[s], gc // self.KVST - 1)
-            self.copies.append((self.kv_full[s], ("kv", s), gc))
-            yield
+            gc = x["gc"]
+            for ver in ((self.kver(gc), self.vver(gc)) if self.halfkv else (gc,)):
+                s = u % self.KVST
+                if u >= self.KVST:
+                    yield from self.wait("kv", self.kv_empty[s], u // self.KVST - 1)
+                self.copies.append((self.kv_full[s], ("kv", s), ver))
+                u += 1
+                yield
 
     def stage_lane(self):
         for k, _it in enumerate(range(self.cta, self.items, self.grid)):
@@ -181,8 +203,9 @@ class Model:
 
         def qk(i, gci):
             sc = i % self.nsc
+            ku = self.kcopy(gci)
             yield from self.wait("mma", self.q_full[i % self.QST], i // self.QST)
-            yield from self.wait("mma", self.kv_full[gci % self.KVST], gci // self.KVST)
+            yield from self.wait("mma", self.kv_full[ku % self.KVST], ku // self.KVST)
 
             def run():
                 assert self.sc_need[sc] is None, (
@@ -190,16 +213,25 @@ class Model:
                 self.ver[("sc", sc)] = ("A", i)
                 self.sc_need[sc] = ("A", i)
             self.mma(f"QK({i})", [(("q", i % self.QST), ("Q", i)),
-                                  (("kv", gci % self.KVST), gci)], run)
+                                  (("kv", ku % self.KVST), self.kver(gci))], run)
             self.commit(self.a_full[sc])
 
+        def wait_v(gci):
+            vu = self.vcopy(gci)
+            yield from self.wait("mma", self.kv_full[vu % self.KVST], vu // self.KVST)
+
         def kv(gci):
+            if self.halfkv:
+                yield from wait_v(gci)
+
             def run():
                 assert self.state_ready >= gci, f"KV({gci}) before the state was ready"
                 self.state_chunk = gci
-            self.mma(f"KV({gci})", [(("kv", gci % self.KVST), gci)], run)
+            ku, vu = self.kcopy(gci), self.vcopy(gci)
+            self.mma(f"KV({gci})", [(("kv", ku % self.KVST), self.kver(gci)),
+                                    (("kv", vu % self.KVST), self.vver(gci))], run)
             self.commit(self.s_full)
-            self.commit(self.kv_empty[gci % self.KVST])
+            self.commit(self.kv_empty[ku % self.KVST])  # K's last reader
 
         yield from qk(0, 0)
         for x in seq:
@@ -227,16 +259,28 @@ class Model:
             early = self.nsc == 2 and not self.staged and not x["item_end"]
             if early:
                 yield from qk(i + 1, nxt)
+            vu = self.vcopy(gc)
+            # with K and V apart the update goes before the step's last P V
+            if self.halfkv and x["last_hs"]:
+                yield from kv(gc)
+            if self.halfkv:
+                yield from wait_v(gc)
+            release_v_early = False
+            if release_v_early and self.halfkv and x["last_hs"]:
+                self.commit(self.kv_empty[vu % self.KVST])
             for h in range(self.halves):
                 pf = self.p_full[h] if self.halves == 2 else self.p_full[sc]
                 yield from self.wait("mma", pf, i // self.nsc)
                 last_half = h == self.halves - 1
-                self.mma(f"PV{h}({i})", [(("ph", sc, h), ("P", i)), (("kv", gc % self.KVST), gc),
+                self.mma(f"PV{h}({i})", [(("ph", sc, h), ("P", i)),
+                                         (("kv", vu % self.KVST), self.vver(gc)),
                                          (("obuf", ob), ("O", i))],
                          pv_run if last_half else pv_half_run)
             self.commit(self.o_full[ob])
-            if x["last_hs"]:
-                kv(gc)
+            if self.halfkv and x["last_hs"] and not release_v_early:
+                self.commit(self.kv_empty[vu % self.KVST])  # V's last reader
+            if not self.halfkv and x["last_hs"]:
+                yield from kv(gc)
             if not early and x["has_next"]:
                 yield from qk(i + 1, nxt)
             yield
@@ -410,6 +454,7 @@ CONFIGS = {
     "t64_dedicated_out": dict(T=64, QST=3, KVST=2, out="dedicated", staged=False),
     "t64_staged": dict(T=64, QST=2, KVST=2, out="qslot", staged=True),
     "t128": dict(T=128, QST=2, KVST=2, out="qslot", staged=False),
+    "t128_half_kv": dict(T=128, QST=3, KVST=3, out="qslot", staged=False, halfkv=True),
 }
 
 SHAPES = [
@@ -469,8 +514,14 @@ MUTANTS = {
         "        self.a_full = [mk(f\"a_full{b}\", 1) for b in range(self.nsc)]",
         "        self.a_full = [mk(\"a_full\", 1)] * self.nsc"),
     "K/V copy without kv_empty": (
-        "            if gc >= self.KVST:\n"
-        "                yield from self.wait(\"kv\", self.kv_empty[s], gc // self.KVST - 1)\n", ""),
+        "                if u >= self.KVST:\n"
+        "                    yield from self.wait(\"kv\", self.kv_empty[s], u // self.KVST - 1)\n",
+        ""),
+    "P V without its V tile": (
+        "            if self.halfkv:\n"
+        "                yield from wait_v(gc)\n", ""),
+    "V tile released before its last P V": (
+        "            release_v_early = False\n", "            release_v_early = True\n"),
     "Q copy without q_empty": (
         "            if i >= self.QST:\n"
         "                yield from self.wait(\"q\", self.q_empty[s], i // self.QST - 1)\n", ""),
