@@ -29,7 +29,9 @@
 // the later spans' sums, from group_scan_kernel) is read at the item start,
 // and the item of span 0 writes dS0 at its end.
 // Roles (320 threads): warp 0 lane 0 streams key blocks (Q and dO of one head
-// half-chunk) through a four-stage ring, lane 1 the K/V tiles of each chunk;
+// half-chunk) through a four-stage ring, lane 1 the K and V tiles of each
+// chunk (K a chunk ahead, into the region the bf16 copy of D leaves once the
+// chunk's first block has used it);
 // warp 1 owns the tensor memory and issues the MMAs; warps 2-5 mask S1,
 // convert the state and write dv rows out; warps 6-9 mask S2 and write dk
 // rows out.  TMEM: dv at column 0, dk at 128, S1 (then P1) at 256, S2 (then
@@ -57,15 +59,20 @@ constexpr int kBlkBytes = kKeyBlk * kHeadDim * 2;   // 16 KB: Q or dO of one blo
 constexpr int kBlkHalf = kKeyBlk * 128;             // 8 KB: 64 columns of a key block
 constexpr uint32_t kColDv = 0, kColDk = 128, kColS1 = 256, kColS2 = 320;
 
+// Two 32 KB regions take turns holding K_c and the bf16 copy of D: for the
+// CTA's chunk n, K_n sits in region n % 2 and D's copy in region (n + 1) % 2.
+// D's copy is read only by K_n D and V_n D^T at the chunk's first block, so
+// K_{n+1} is loaded into its region as soon as those have run, a chunk ahead;
+// the copy for chunk n + 1 then goes into K_n's region once the chunk's last
+// scores and updates have run.  V_c keeps a region of its own.
 struct WalkLayout {
-  static constexpr int kKOff = 0;
-  static constexpr int kVOff = kChunkBytes;
-  static constexpr int kRingOff = 2 * kChunkBytes;                // stage: Q block, dO block
-  static constexpr int kSOff = kRingOff + kRing * 2 * kBlkBytes;  // bf16 copy of D
-  static constexpr int kBarOff = kSOff + kSBytes;
-  // ring_full[R], ring_empty[R], kv_full, kv_empty, a_full[2], p_full[2],
-  // o_full, o_empty[2], s_full, sb_full, mma_done
-  static constexpr int kNumBars = 2 * kRing + 12;
+  static constexpr int kRegOff = 0;                  // regions 0 and 1: K_c or D
+  static constexpr int kVOff = 2 * kChunkBytes;
+  static constexpr int kRingOff = 3 * kChunkBytes;   // stage: Q block, dO block
+  static constexpr int kBarOff = kRingOff + kRing * 2 * kBlkBytes;
+  // ring_full[R], ring_empty[R], k_full, v_full, d_free, v_free, a_full[2],
+  // p_full[2], o_full, o_empty[2], s_full, sb_full, mma_done
+  static constexpr int kNumBars = 2 * kRing + 14;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -152,9 +159,11 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBarOff);
   uint64_t* ring_full = bars;
   uint64_t* ring_empty = ring_full + kRing;
-  uint64_t* kv_full = ring_empty + kRing;
-  uint64_t* kv_empty = kv_full + 1;
-  uint64_t* a_full = kv_empty + 1;   // two: S1, S2 of a block computed
+  uint64_t* k_full = ring_empty + kRing;  // K_c of a chunk landed
+  uint64_t* v_full = k_full + 1;          // V_c of a chunk landed
+  uint64_t* d_free = v_full + 1;          // a chunk's K_c D, V_c D^T done: D's region free
+  uint64_t* v_free = d_free + 1;          // a chunk's last V_c reader done
+  uint64_t* a_full = v_free + 1;     // two: S1, S2 of a block computed
   uint64_t* p_full = a_full + 2;     // two: P1, P2 of a block written over their scores
   uint64_t* o_full = p_full + 2;     // dv, dk of a chunk complete
   uint64_t* o_empty = o_full + 1;    // two: dv, dk read out
@@ -164,8 +173,10 @@ __global__ void __launch_bounds__(320, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMiscOff + 4);
 
-  const uint32_t sK = base + L::kKOff, sV = base + L::kVOff;
-  const uint32_t sS = base + L::kSOff;
+  // region of K_n and of D's bf16 copy for the CTA's chunk n; V_c's region
+  auto sK = [&](int n) { return base + (uint32_t)(L::kRegOff + (n & 1) * kChunkBytes); };
+  auto sS = [&](int n) { return base + (uint32_t)(L::kRegOff + ((n + 1) & 1) * kChunkBytes); };
+  const uint32_t sV = base + L::kVOff;
   auto sQ = [&](int s) { return base + (uint32_t)(L::kRingOff + s * 2 * kBlkBytes); };
   auto sDO = [&](int s) { return sQ(s) + (uint32_t)kBlkBytes; };
   const int stride = (int)gridDim.x;
@@ -178,8 +189,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
     }
-    mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1);
+    mbar_init(k_full, 1);
+    mbar_init(v_full, 1);
+    mbar_init(d_free, 1);
+    mbar_init(v_free, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&a_full[t], 1);
       mbar_init(&p_full[t], 128);
@@ -242,7 +255,7 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&map_k);
       prefetch_tmap(&map_v);
       const uint64_t pol = policy_evict_first();
-      int gc = 0;
+      int gc = 0, k_issued = 0, v_issued = 0;
       bool go = true;
       for (int it = blockIdx.x; it < p.items && go; it += stride) {
         int bg, tb, te;
@@ -252,20 +265,32 @@ __global__ void __launch_bounds__(320, 1)
           prefetch_l2_bulk(p.ws + (size_t)nx * kDD, (uint32_t)(kDD * sizeof(float)));
         for (int n = 0; n < te - tb; ++n, ++gc) {
           const int cs = te - 1 - n;
-          if (gc >= 1 && !mbar_wait(kv_empty, (gc - 1) & 1, p.status, abort_flag)) {
+          // K_c into the region chunk gc - 1's D copy held (free once that
+          // chunk's K_c D, V_c D^T have run), then V_c into its own region
+          if (gc >= 1 && !mbar_wait(d_free, (gc - 1) & 1, p.status, abort_flag)) {
             go = false;
             break;
           }
-          mbar_arrive_expect_tx(kv_full, 2 * kChunkBytes);
-          uint8_t* k_dst = sm + (sK - base);
+          mbar_arrive_expect_tx(k_full, kChunkBytes);
+          uint8_t* k_dst = sm + (sK(gc) - base);
+          tma_load_3d(k_dst, &map_k, k_full, 0, cs * kChunk, bg, pol);
+          tma_load_3d(k_dst + kHalf, &map_k, k_full, 64, cs * kChunk, bg, pol);
+          ++k_issued;
+          if (gc >= 1 && !mbar_wait(v_free, (gc - 1) & 1, p.status, abort_flag)) {
+            go = false;
+            break;
+          }
+          mbar_arrive_expect_tx(v_full, kChunkBytes);
           uint8_t* v_dst = sm + (sV - base);
-          tma_load_3d(k_dst, &map_k, kv_full, 0, cs * kChunk, bg, pol);
-          tma_load_3d(k_dst + kHalf, &map_k, kv_full, 64, cs * kChunk, bg, pol);
-          tma_load_3d(v_dst, &map_v, kv_full, 0, cs * kChunk, bg, pol);
-          tma_load_3d(v_dst + kHalf, &map_v, kv_full, 64, cs * kChunk, bg, pol);
+          tma_load_3d(v_dst, &map_v, v_full, 0, cs * kChunk, bg, pol);
+          tma_load_3d(v_dst + kHalf, &map_v, v_full, 64, cs * kChunk, bg, pol);
+          ++v_issued;
         }
       }
-      if (*abort_flag && gc > 0) mbar_wait_drain(kv_full, (gc - 1) & 1);
+      if (*abort_flag) {  // let copies already issued land before the block exits
+        if (k_issued > 0) mbar_wait_drain(k_full, (k_issued - 1) & 1);
+        if (v_issued > 0) mbar_wait_drain(v_full, (v_issued - 1) & 1);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -277,18 +302,20 @@ __global__ void __launch_bounds__(320, 1)
     // tensor pipe runs in issue order), and each mask has the other stream's
     // product and scores and D's update to run under it.  The bf16 copy of D
     // is waited for only before K_c D; D's first update of a chunk follows it
-    // (the conversion reads D).  K_c and V_c sit in one slot, released once
-    // the chunk's last S2 and its K_c D, V_c D^T are issued; a next chunk's
-    // scores therefore go at the end of the block.
+    // (the conversion reads D).  After K_c D, V_c D^T the region of D's copy
+    // is released (the next chunk's K_c goes there); V_c's region once the
+    // chunk's last S2 and V_c D^T are issued.  A next chunk's scores go at the
+    // end of the block.
     if (elect_one()) {
       int inter_gc = -1;    // last chunk whose K_c D, V_c D^T are issued
-      int kv_pending = -1;  // chunk whose last S2 is issued before its K_c D
+      int kv_pending = -1;  // chunk whose last S2 is issued before its V_c D^T
       auto issue_s = [&](int t, const Cursor& x) -> bool {
-        if (x.blk == 0 && !mbar_wait(kv_full, x.gc & 1, p.status, abort_flag)) return false;
+        if (x.blk == 0 && !mbar_wait(t == 0 ? k_full : v_full, x.gc & 1, p.status, abort_flag))
+          return false;
         const int s = x.i % kRing;
         if (!mbar_wait(&ring_full[s], (x.i / kRing) & 1, p.status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t src = t == 0 ? sK : sV;               // K_c or V_c
+        const uint32_t src = t == 0 ? sK(x.gc) : sV;         // K_c or V_c
         const uint32_t blk = t == 0 ? sQ(s) : sDO(s);        // Q or dO of the block
         const uint32_t dst = tmem + (t == 0 ? kColS1 : kColS2);
 #pragma unroll
@@ -299,9 +326,9 @@ __global__ void __launch_bounds__(320, 1)
                  smem_desc_sw128(blk + ch * kBlkHalf + koff, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
         mma_commit(&a_full[t]);
-        if (t == 1 && x.blk == x.nb - 1) {  // the chunk's last score read of K_c, V_c
+        if (t == 1 && x.blk == x.nb - 1) {  // the chunk's last score read of V_c
           if (inter_gc >= x.gc)
-            mma_commit(kv_empty);
+            mma_commit(v_free);
           else
             kv_pending = x.gc;
         }
@@ -342,23 +369,25 @@ __global__ void __launch_bounds__(320, 1)
         if (first) {  // the state's terms: dv += K_c D, dk += V_c D^T
           if (!mbar_wait(sb_full, c.gc & 1, p.status, abort_flag)) break;
           tc_fence_after();
+          const uint32_t ka = sK(c.gc), da = sS(c.gc);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t koff = (uint32_t)((kk & 3) * 32);
             const uint32_t ch = (uint32_t)(kk >> 2);
-            mma_ss(tmem + kColDv, smem_desc_sw128(sK + ch * kHalf + koff, 16, 1024),
-                   smem_desc_sw128(sS + kk * 2048, kHalf, 1024), IDESC_KD, 1u);
+            mma_ss(tmem + kColDv, smem_desc_sw128(ka + ch * kHalf + koff, 16, 1024),
+                   smem_desc_sw128(da + kk * 2048, kHalf, 1024), IDESC_KD, 1u);
           }
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t koff = (uint32_t)((kk & 3) * 32);
             const uint32_t ch = (uint32_t)(kk >> 2);
             mma_ss(tmem + kColDk, smem_desc_sw128(sV + ch * kHalf + koff, 16, 1024),
-                   smem_desc_sw128(sS + ch * kHalf + koff, 16, 1024), IDESC_VDT, 1u);
+                   smem_desc_sw128(da + ch * kHalf + koff, 16, 1024), IDESC_VDT, 1u);
           }
+          mma_commit(d_free);  // D's copy read: its region takes the next K_c
           inter_gc = c.gc;
           if (kv_pending == c.gc) {
-            mma_commit(kv_empty);
+            mma_commit(v_free);
             kv_pending = -1;
           }
         }
@@ -395,7 +424,8 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
 
     // entering state of item it -> D in tensor memory and its bf16 copy
-    auto load_state = [&](int it) {
+    auto load_state = [&](int it, int gcd) {  // for the CTA's chunk gcd
+      const uint32_t dcopy = sS(gcd);
       const float4* src =
           p.ws ? reinterpret_cast<const float4*>(p.ws + (size_t)it * kDD + (size_t)r * kHeadDim)
                : nullptr;
@@ -412,7 +442,7 @@ __global__ void __launch_bounds__(320, 1)
           v[4 * m + 3] = __float_as_uint(f.w);
         }
         tmem_st32(tmem + lane_base + kColS + blk * 32, v);
-        store_row32_sw128(sS, r, blk, v);
+        store_row32_sw128(dcopy, r, blk, v);
       }
       tmem_wait_st();
       fence_proxy_async_smem();
@@ -433,8 +463,8 @@ __global__ void __launch_bounds__(320, 1)
           tmem_ld32(tmem + lane_base + kColS + blk * 32, v0);
           tmem_ld32(tmem + lane_base + kColS + (blk + 1) * 32, v1);
           tmem_wait_ld();
-          store_row32_sw128(sS, r, blk, v0);
-          store_row32_sw128(sS, r, blk + 1, v1);
+          store_row32_sw128(sS(gcd + 1), r, blk, v0);
+          store_row32_sw128(sS(gcd + 1), r, blk + 1, v1);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -457,7 +487,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       tc_fence_before();
-      if (next_it >= 0) load_state(next_it);
+      if (next_it >= 0) load_state(next_it, gcd + 1);
       return true;
     };
 
@@ -535,7 +565,7 @@ __global__ void __launch_bounds__(320, 1)
 
     if (wg1) {
       griddep_wait();  // entering states come from the kernel before
-      load_state(blockIdx.x);
+      load_state(blockIdx.x, 0);
     }
     Cursor c;
     cursor_init(p, c);

@@ -58,7 +58,10 @@ class Model:
         mk = Barrier
         self.ring_full = [mk(f"ring_full{s}", 1) for s in range(RING)]
         self.ring_empty = [mk(f"ring_empty{s}", 1) for s in range(RING)]
-        self.kv_full, self.kv_empty = mk("kv_full", 1), mk("kv_empty", 1)
+        # K_n and the bf16 copy of D take turns in two regions (K_n in region
+        # n % 2, D's copy for chunk n in region (n + 1) % 2); V has its own
+        self.k_full, self.v_full = mk("k_full", 1), mk("v_full", 1)
+        self.d_free, self.v_free = mk("d_free", 1), mk("v_free", 1)
         # two score streams, each in its own tensor-memory buffer: S1 = K_c Q^T
         # (masked by warpgroup 1 into P1, for dv) and S2 = V_c dO^T (warpgroup
         # 2, P2, for dk); each P is written over its own scores
@@ -72,7 +75,8 @@ class Model:
         self.copies = []       # (barrier, resource, version), landing in any order
         # resource versions
         self.ver = {("ring", s): None for s in range(RING)}
-        self.ver.update({"kv": None, "sS": 0, ("S", 0): None, ("S", 1): None})
+        self.ver.update({("R", 0): None, ("R", 1): None, "V": None, ("S", 0): None,
+                         ("S", 1): None})
         self.sc_need = {0: None, 1: None}  # scores or P a buffer still owes its reader
         self.d_ready = 0              # D holds what chunk d_ready's updates need
         self.d_done = -1              # last chunk whose every update of D has executed
@@ -155,9 +159,14 @@ class Model:
         for it in range(self.cta, self.items, self.grid):
             _, tb, te = self.span_of(it)
             for _n in range(te - tb):
+                # K into the region the previous chunk's D copy held, then V
                 if gc >= 1:
-                    yield from self.wait("kv", self.kv_empty, gc - 1)
-                self.copies.append((self.kv_full, "kv", gc))
+                    yield from self.wait("kv", self.d_free, gc - 1)
+                self.copies.append((self.k_full, ("R", gc % 2), ("K", gc)))
+                yield
+                if gc >= 1:
+                    yield from self.wait("kv", self.v_free, gc - 1)
+                self.copies.append((self.v_full, "V", gc))
                 gc += 1
                 yield
 
@@ -197,17 +206,18 @@ class Model:
             return run
 
         def issue_s(t, x):
+            gc = x["gc"]
             if x["blk"] == 0:
-                yield from self.wait("mma", self.kv_full, x["gc"])
+                yield from self.wait("mma", self.k_full if t == 0 else self.v_full, gc)
             s = x["i"] % RING
             yield from self.wait("mma", self.ring_full[s], x["i"] // RING)
-            self.mma(f"S{t + 1}({x['i']})", [(("ring", s), x["i"]), ("kv", x["gc"])],
-                     scores(t, x["i"]))
+            src = (("R", gc % 2), ("K", gc)) if t == 0 else ("V", gc)
+            self.mma(f"S{t + 1}({x['i']})", [(("ring", s), x["i"]), src], scores(t, x["i"]))
             self.commit(self.a_full[t])
-            # S2 of a chunk's last block is the K/V slot's last score reader
+            # S2 of a chunk's last block is V's last score reader
             if t == 1 and x["blk"] == x["nb"] - 1:
                 if st["inter_gc"] >= x["gc"]:
-                    self.commit(self.kv_empty)
+                    self.commit(self.v_free)
                 else:
                     st["kv_pending"] = x["gc"]
 
@@ -225,8 +235,9 @@ class Model:
                 yield from self.wait("mma", self.o_empty[0], gc - 1)
             self.mma(f"dv+=P1dO({k})", [(("ring", s), k), (("S", 0), ("P", k))],
                      product(1, gc, first, 0))
-            # a next chunk's scores wait for the K/V slot, whose release needs
-            # this chunk's K_c D, V_c D^T issued: at a chunk boundary they go last
+            # a next chunk's scores wait for its K and V, whose regions free up
+            # with this chunk's K_c D, V_c D^T and last S2: at a chunk
+            # boundary they go last
             if nxt and nxt["blk"] != 0:
                 yield from issue_s(0, nxt)
             yield from self.wait("mma", self.p_full[1], k)
@@ -240,11 +251,13 @@ class Model:
                 # the bf16 copy of D for this chunk; D's first update of the
                 # chunk waits for it too (the conversion reads D)
                 yield from self.wait("mma", self.sb_full, gc)
-                self.mma(f"dv+=KD({gc})", [("kv", gc), ("sS", gc)], product(1, gc, False))
-                self.mma(f"dk+=VD^T({gc})", [("kv", gc), ("sS", gc)], product(2, gc, False))
+                kreg, dreg = (("R", gc % 2), ("K", gc)), (("R", (gc + 1) % 2), ("D", gc))
+                self.mma(f"dv+=KD({gc})", [kreg, dreg], product(1, gc, False))
+                self.mma(f"dk+=VD^T({gc})", [("V", gc), dreg], product(2, gc, False))
+                self.commit(self.d_free)
                 st["inter_gc"] = gc
                 if st["kv_pending"] == gc:
-                    self.commit(self.kv_empty)
+                    self.commit(self.v_free)
                     st["kv_pending"] = -1
             self.mma(f"D+=QdO({k})", [(("ring", s), k)], update(gc, last))
             self.commit(self.ring_empty[s])
@@ -277,7 +290,8 @@ class Model:
             # now serve chunk gc
             if gc > 0:
                 assert self.d_done == gc - 1, f"{role}: reads D for chunk {gc} after chunk {self.d_done}"
-            self.overwrite("sS", gc, role)
+            d_region = ("R", (gc + 1) % 2)
+            self.overwrite(d_region, ("D", gc), role)
             self.d_ready = gc
             self.sb_full.arrive()
 
@@ -424,21 +438,28 @@ MUTANTS = {
     "key block copied into a busy stage": (
         "                yield from self.wait(\"ring\", self.ring_empty[s], x[\"i\"] // RING - 1)\n",
         "                pass\n"),
-    "K/V copied into the busy slot": (
-        "                    yield from self.wait(\"kv\", self.kv_empty, gc - 1)\n",
+    "K copied over D's copy before its readers ran": (
+        "                    yield from self.wait(\"kv\", self.d_free, gc - 1)\n",
         "                    pass\n"),
+    "V copied into the busy region": (
+        "                    yield from self.wait(\"kv\", self.v_free, gc - 1)\n",
+        "                    pass\n"),
+    "D's copy written over the chunk's own K": (
+        "            d_region = (\"R\", (gc + 1) % 2)\n",
+        "            d_region = (\"R\", gc % 2)\n"),
     "next S1 ahead of the dv that reads P1": (
         "            self.mma(f\"dv+=P1dO({k})\", [((\"ring\", s), k), ((\"S\", 0), (\"P\", k))],\n"
         "                     product(1, gc, first, 0))\n"
-        "            # a next chunk's scores wait for the K/V slot, whose release needs\n"
-        "            # this chunk's K_c D, V_c D^T issued: at a chunk boundary they go last\n"
+        "            # a next chunk's scores wait for its K and V, whose regions free up\n"
+        "            # with this chunk's K_c D, V_c D^T and last S2: at a chunk\n"
+        "            # boundary they go last\n"
         "            if nxt and nxt[\"blk\"] != 0:\n"
         "                yield from issue_s(0, nxt)\n",
         "            if nxt and nxt[\"blk\"] != 0:\n"
         "                yield from issue_s(0, nxt)\n"
         "            self.mma(f\"dv+=P1dO({k})\", [((\"ring\", s), k), ((\"S\", 0), (\"P\", k))],\n"
         "                     product(1, gc, first, 0))\n"),
-    "K/V released at the last S1 instead of the last S2": (
+    "V released at the last S1 instead of the last S2": (
         "            if t == 1 and x[\"blk\"] == x[\"nb\"] - 1:\n",
         "            if t == 0 and x[\"blk\"] == x[\"nb\"] - 1:\n"),
     "one p_full barrier for both streams": (
