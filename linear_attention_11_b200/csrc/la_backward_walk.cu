@@ -554,13 +554,26 @@ __global__ void __launch_bounds__(320, 1)
       return true;
     };
     // row r of chunk cs of group bg to global memory (rows past N dropped)
-    auto store_out = [&](int bg, int cs, const uint32_t (&row_bf)[64]) {
+    // quarter qt (64 bytes) of row r of chunk cs of group bg to global
+    // memory (rows past N dropped)
+    auto store_quarter = [&](int bg, int cs, const uint32_t (&row_bf)[64], int qt) {
       const int64_t row = (int64_t)cs * kChunk + r;
       if (row >= p.N) return;
       uint4* dst = reinterpret_cast<uint4*>(out_base + ((size_t)bg * p.N + row) * kHeadDim);
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        dst[m] = make_uint4(row_bf[4 * m], row_bf[4 * m + 1], row_bf[4 * m + 2], row_bf[4 * m + 3]);
+      switch (qt) {  // constant register indices in each case
+#define LA_STORE_QUARTER(Q)                                                             \
+  case Q:                                                                               \
+    _Pragma("unroll") for (int m = 4 * Q; m < 4 * Q + 4; ++m) dst[m] =                 \
+        make_uint4(row_bf[4 * m], row_bf[4 * m + 1], row_bf[4 * m + 2], row_bf[4 * m + 3]); \
+    break;
+        LA_STORE_QUARTER(0)
+        LA_STORE_QUARTER(1)
+        LA_STORE_QUARTER(2)
+        LA_STORE_QUARTER(3)
+#undef LA_STORE_QUARTER
+        default:
+          break;
+      }
     };
 
     if (wg1) {
@@ -571,13 +584,20 @@ __global__ void __launch_bounds__(320, 1)
     cursor_init(p, c);
     int prev_it = -1, prev_gc = -1, prev_bg = 0, prev_cs = 0;
     uint32_t row_bf[64];
+    // the read-out row goes to global memory a quarter per block, after each
+    // of the next four masks: stored all at once, the warpgroups' 16-byte
+    // stores slowed the MMA thread's issue for the chunk's first block
+    int stored = 4, out_bg = 0, out_cs = 0;
     for (; c.valid && ok; cursor_next(p, c)) {
-      // the chunk before ended: its accumulator is read out first (the new
-      // chunk's first product waits for it), then this block's mask, then
-      // the state step (the bf16 copy is first used later in the block), and
-      // only then the read-out rows go to global memory
+      // the chunk before ended: the rest of the row before it goes out, its
+      // accumulator is read out (the new chunk's first product waits for
+      // it), then this block's mask, then the state step (the bf16 copy is
+      // first used later in the block)
       const bool boundary = c.blk == 0 && prev_gc >= 0;
-      if (boundary && !read_out(prev_gc, row_bf)) { ok = false; break; }
+      if (boundary) {
+        for (; stored < 4; ++stored) store_quarter(out_bg, out_cs, row_bf, stored);
+        if (!read_out(prev_gc, row_bf)) { ok = false; break; }
+      }
       if (!mask_block(c)) { ok = false; break; }
       if (boundary) {
         const bool item_end = c.it != prev_it;
@@ -585,16 +605,21 @@ __global__ void __launch_bounds__(320, 1)
           ok = false;
           break;
         }
-        store_out(prev_bg, prev_cs, row_bf);
+        stored = 0;
+        out_bg = prev_bg;
+        out_cs = prev_cs;
       }
+      if (stored < 4) store_quarter(out_bg, out_cs, row_bf, stored++);
       prev_it = c.it;
       prev_gc = c.gc;
       prev_bg = c.bg;
       prev_cs = c.cs;
     }
     if (ok && prev_gc >= 0) {
+      for (; stored < 4; ++stored) store_quarter(out_bg, out_cs, row_bf, stored);
       if (wg1) ok = state_step(prev_gc, true, prev_it, -1);
-      if (ok && read_out(prev_gc, row_bf)) store_out(prev_bg, prev_cs, row_bf);
+      if (ok && read_out(prev_gc, row_bf))
+        for (int qt = 0; qt < 4; ++qt) store_quarter(prev_bg, prev_cs, row_bf, qt);
     }
   }
 
