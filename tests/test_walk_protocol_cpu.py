@@ -276,8 +276,8 @@ class Model:
 
         def write_out(p):
             # the accumulator is read into registers and released; the rows
-            # go to global memory later (after the next mask), outside the
-            # protocol
+            # go to global memory later (a quarter after each of the next four
+            # masks), outside the protocol
             yield from self.wait(role, self.o_full, p["gc"])
             assert self.acc[wg] == p["gc"], f"{role}: reads chunk {p['gc']}, holds {self.acc[wg]}"
             self.acc_read[wg] = p["gc"]
