@@ -60,7 +60,9 @@ struct PersistParams {
 // memory by bulk tensor copies (map_s over the states, [units, 128, 128]),
 // loaded an item ahead by a third copy lane; without it the math warps read
 // and write them row by row.  kDedO: a dedicated output staging tile (else
-// the output goes through the Q slot).
+// the output goes through the Q slot).  kHalfKV: K and V tiles take separate
+// slots of the K/V ring (used at T = 128 with several tiles per chunk step,
+// where the 32 KB this saves holds a third Q slot).
 template <int T, int QST, int KVST, bool kDedO, bool kStage, bool kHalfKV>
 __global__ void __launch_bounds__(320, 1)
     prefill_persist_kernel(const __grid_constant__ CUtensorMap map_q,
@@ -280,6 +282,9 @@ __global__ void __launch_bounds__(320, 1)
     // whose P(i) P V(i) still reads) after P V(i), so the next mask overlaps
     // QS(i + 1).  At an item's end the update goes first, so the state
     // hand-over to the next item does not wait for that item's first tiles.
+    // With K and V apart (kHalfKV) the update of a chunk step goes right
+    // after the last tile's QS, ahead of its P V: the update is then K's last
+    // reader and releases K's slot, V's goes after that P V.
     if (elect_one()) {
       // wait for the K (or K/V) tile of chunk step c, or its V tile
       auto wait_k = [&](int c) {
