@@ -553,7 +553,6 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(my_empty);
       return true;
     };
-    // row r of chunk cs of group bg to global memory (rows past N dropped)
     // quarter qt (64 bytes) of row r of chunk cs of group bg to global
     // memory (rows past N dropped)
     auto store_quarter = [&](int bg, int cs, const uint32_t (&row_bf)[64], int qt) {
